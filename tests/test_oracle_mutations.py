@@ -1,0 +1,76 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case copies the oracle into a temporary directory, plants one mistake
+in the copy's C source (a dropped term, a wrong sign, a transposed operand,
+a wrong index), and runs the pin suite against the copy in a subprocess.
+The suite must fail for every planted mistake and pass for the unmodified
+copy.  Nothing here touches the real oracle or any GPU.
+"""
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
+
+MUTATIONS = {
+    "no_softmax_scale": ("s[j] = scale * dot;", "s[j] = dot;"),
+    "no_softmax_normalisation": ("o[c] /= l;", "o[c] /= 1.0;"),
+    "value_row_index": ("const double* vj = v + IDX4(b, j, h, 0, L, H, d);",
+                        "const double* vj = v + IDX4(b, i, h, 0, L, H, d);"),
+    "phi_q_transposed": ("acc += qi[a] * Wq[(size_t)a * d + c];",
+                         "acc += qi[a] * Wq[(size_t)c * d + a];"),
+    "read_state_transposed": ("acc += qp[c] * S[(size_t)c * d + n];",
+                              "acc += qp[c] * S[(size_t)n * d + c];"),
+    "phi_kv_transposed": ("for (int a = 0; a < d; ++a) acc += xr[a] * W[(size_t)a * d + c];",
+                          "for (int a = 0; a < d; ++a) acc += xr[a] * W[(size_t)c * d + a];"),
+    "no_key_normalisation": ("if (l2norm) {", "if (0) {"),
+    "residual_sign": ("r[(size_t)t * d + n] = vp[(size_t)t * d + n] - acc;",
+                      "r[(size_t)t * d + n] = vp[(size_t)t * d + n] + acc;"),
+    "residual_dropped": ("r[(size_t)t * d + n] = vp[(size_t)t * d + n] - acc;",
+                         "r[(size_t)t * d + n] = vp[(size_t)t * d + n];"),
+    "alpha_dropped": ("S[(size_t)c * d + n] = a * S[(size_t)c * d + n] + dS[(size_t)c * d + n];",
+                      "S[(size_t)c * d + n] = S[(size_t)c * d + n] + dS[(size_t)c * d + n];"),
+    "beta_dropped": ("acc += bt[t] * kp[(size_t)t * d + c] * r[(size_t)t * d + n];",
+                     "acc += kp[(size_t)t * d + c] * r[(size_t)t * d + n];"),
+    "update_outer_product_transposed": (
+        "acc += bt[t] * kp[(size_t)t * d + c] * r[(size_t)t * d + n];",
+        "acc += bt[t] * kp[(size_t)t * d + n] * r[(size_t)t * d + c];"),
+    "update_on_every_pass": ("if (clean) return arl2_oracle_state_update(",
+                             "if (1) return arl2_oracle_state_update("),
+}
+
+
+def _run_pins_on_copy(tmp_path, mutation):
+    dst = tmp_path / "oracle"
+    shutil.copytree(os.path.join(ROOT, "oracle"), dst,
+                    ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    src = dst / "arl2_oracle.c"
+    text = src.read_text()
+    if mutation is not None:
+        old, new = mutation
+        assert text.count(old) == 1, f"mutation anchor not unique: {old!r}"
+        src.write_text(text.replace(old, new))
+    env = dict(os.environ)
+    env["PYTHONPATH"] = str(tmp_path) + os.pathsep + env.get("PYTHONPATH", "")
+    env["OMP_NUM_THREADS"] = "2"
+    cmd = [sys.executable, "-c",
+           "import sys, pytest; import oracle; assert oracle.__file__.startswith(sys.argv[1]); "
+           "sys.exit(pytest.main(['-q', '-x', '-p', 'no:cacheprovider', sys.argv[2]]))",
+           str(tmp_path), PINS]
+    return subprocess.run(cmd, env=env, cwd=str(tmp_path), capture_output=True, text=True,
+                          timeout=300)
+
+
+def test_unmodified_copy_passes(tmp_path):
+    r = _run_pins_on_copy(tmp_path, None)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(tmp_path, name):
+    r = _run_pins_on_copy(tmp_path, MUTATIONS[name])
+    assert r.returncode != 0, f"pins did not catch mutation {name}"

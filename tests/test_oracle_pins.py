@@ -1,0 +1,336 @@
+"""Pins of the CPU oracle against what the ARL2 pages and mathematics fix.
+
+None of these tests compares the oracle with a retyped copy of itself.  Each
+pin is one of: a case worked out by hand (tests/golden), a special case that
+reduces to a library routine (torch's scaled_dot_product_attention), a
+closed form of the update (orthonormal keys), or an invariant the method
+implies (frame-level sharing, clean-pass-only updates, independence of
+streams and heads, scale invariance of the k' normalisation).
+
+Method text: "Attend Locally, Remember Linearly", technical summary
+section 2.1 (branches, phi maps, state update, read) and section 2.2
+(frame-level access, clean-pass updates).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_worked_cases.json")
+
+
+def rnd(rng, *shape, scale=1.0):
+    return rng.standard_normal(shape) * scale
+
+
+def eye_w(H, d):
+    return np.broadcast_to(np.eye(d), (H, d, d)).copy()
+
+
+def make(rng, B=2, L=7, H=3, d=8, wscale=0.3):
+    q, k, v = (rnd(rng, B, L, H, d) for _ in range(3))
+    wq, wk, wv = (np.eye(d)[None] + rnd(rng, H, d, d, scale=wscale) for _ in range(3))
+    alpha = 1.0 / (1.0 + np.exp(-(2.0 + 0.5 * rnd(rng, B, H))))
+    beta = 1.0 / (1.0 + np.exp(-rnd(rng, B, H, L))) / L
+    S = rnd(rng, B, H, d, d, scale=0.1)
+    return dict(q=q, k=k, v=v, wq=wq, wk=wk, wv=wv, alpha=alpha, beta=beta, S=S)
+
+
+def run(x, clean, S=None, **over):
+    a = dict(x)
+    a.update(over)
+    return oracle.frame_pass(a["q"], a["k"], a["v"], a["wq"], a["wk"], a["wv"], a["alpha"],
+                             a["beta"], a["S"] if S is None else S, clean)
+
+
+def as_blhd(m):
+    """[L][d] (one stream, one head) -> [1][L][1][d]."""
+    m = np.asarray(m, dtype=np.float64)
+    return m[None, :, None, :]
+
+
+def w_from(spec, d):
+    if spec == "identity":
+        return np.eye(d)[None]
+    return np.asarray(spec, dtype=np.float64)[None]
+
+
+def s_from(spec, d):
+    if spec == "zero":
+        return np.zeros((1, 1, d, d))
+    return np.asarray(spec, dtype=np.float64)[None, None]
+
+
+# --------------------------------------------------------------------------
+# Hand-worked cases (tests/golden)
+# --------------------------------------------------------------------------
+
+def golden_cases():
+    with open(GOLDEN) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", golden_cases(), ids=lambda c: c["name"])
+def test_hand_worked_case(case):
+    d, L = case["d"], case["L"]
+    zeros = np.zeros((L, d))
+    q = as_blhd(case.get("q", zeros))
+    k = as_blhd(case["k"])
+    v = as_blhd(case["v"])
+    wq = w_from(case.get("w_q", "identity"), d)
+    wk = w_from(case.get("w_k", "identity"), d)
+    wv = w_from(case.get("w_v", "identity"), d)
+    S = s_from(case.get("S_prev", "zero"), d)
+    alpha = np.array([[case.get("alpha", 1.0)]])
+    beta = np.asarray(case.get("beta", [0.0] * L), dtype=np.float64)[None, None]
+    clean = "expected_S" in case
+    out, S_new = oracle.frame_pass(q, k, v, wq, wk, wv, alpha, beta, S, clean)
+    if "expected_out" in case:
+        np.testing.assert_allclose(out[0, :, 0, :], case["expected_out"], rtol=0, atol=1e-12)
+    if clean:
+        np.testing.assert_allclose(S_new[0, 0], case["expected_S"], rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Intra branch: textbook softmax attention
+# --------------------------------------------------------------------------
+
+def test_intra_equals_library_sdpa_when_state_is_zero():
+    rng = np.random.default_rng(1)
+    x = make(rng, B=2, L=13, H=3, d=8)
+    S0 = np.zeros_like(x["S"])
+    out, _ = run(x, clean=False, S=S0)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a.transpose(0, 2, 1, 3)))  # [B,H,L,d]
+    ref = torch.nn.functional.scaled_dot_product_attention(t(x["q"]), t(x["k"]), t(x["v"]))
+    np.testing.assert_allclose(out, ref.numpy().transpose(0, 2, 1, 3), rtol=0, atol=1e-12)
+
+
+def test_single_token_frame_returns_its_value():
+    rng = np.random.default_rng(2)
+    x = make(rng, B=1, L=1, H=2, d=5)
+    out, _ = run(x, clean=False, S=np.zeros_like(x["S"]))
+    np.testing.assert_allclose(out, x["v"], rtol=0, atol=1e-14)
+
+
+def test_identical_keys_average_the_values():
+    rng = np.random.default_rng(3)
+    x = make(rng, B=1, L=9, H=2, d=6)
+    k = np.broadcast_to(x["k"][:, :1], x["k"].shape).copy()
+    out, _ = run(x, clean=False, S=np.zeros_like(x["S"]), k=k)
+    mean_v = np.broadcast_to(x["v"].mean(axis=1, keepdims=True), x["v"].shape)
+    np.testing.assert_allclose(out, mean_v, rtol=0, atol=1e-13)
+
+
+def test_dominant_key_selects_its_value():
+    rng = np.random.default_rng(4)
+    B, L, H, d = 1, 6, 1, 4
+    q = np.zeros((B, L, H, d)); q[..., 0] = 1.0
+    k = np.zeros((B, L, H, d)); k[0, 3, 0, 0] = 200.0   # score 100 vs 0 after the 1/2 scale
+    v = rnd(rng, B, L, H, d)
+    out, _ = oracle.frame_pass(q, k, v, eye_w(H, d), eye_w(H, d), eye_w(H, d), None, None,
+                               np.zeros((B, H, d, d)), False)
+    np.testing.assert_allclose(out[0, :, 0], np.broadcast_to(v[0, 3, 0], (L, d)), atol=1e-30)
+
+
+# --------------------------------------------------------------------------
+# Inter read
+# --------------------------------------------------------------------------
+
+def test_zero_state_adds_nothing_and_read_is_linear_in_state():
+    rng = np.random.default_rng(5)
+    x = make(rng)
+    o0, _ = run(x, clean=False, S=np.zeros_like(x["S"]))
+    o1, _ = run(x, clean=False, S=x["S"])
+    o2, _ = run(x, clean=False, S=2.0 * x["S"])
+    # O(S) - O(0) is linear in S: O(2S) - O(0) = 2 (O(S) - O(0))
+    np.testing.assert_allclose(o2 - o0, 2.0 * (o1 - o0), rtol=0, atol=1e-12)
+    assert np.max(np.abs(o1 - o0)) > 1e-3
+
+
+def test_read_with_shift_map_and_identity_state():
+    # W_q[a][a+1] = 1 shifts features right by one; with S = I and v = 0
+    # the output is the shifted query: o[:, c] = q[:, c-1], o[:, 0] = 0.
+    rng = np.random.default_rng(6)
+    B, L, H, d = 1, 5, 2, 6
+    q = rnd(rng, B, L, H, d)
+    k = rnd(rng, B, L, H, d)
+    v = np.zeros((B, L, H, d))
+    shift = np.zeros((d, d))
+    for a in range(d - 1):
+        shift[a, a + 1] = 1.0
+    wq = np.broadcast_to(shift, (H, d, d)).copy()
+    S = np.broadcast_to(np.eye(d), (B, H, d, d)).copy()
+    out, _ = oracle.frame_pass(q, k, v, wq, eye_w(H, d), eye_w(H, d), None, None, S, False)
+    np.testing.assert_allclose(out[..., 1:], q[..., :-1], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(out[..., 0], 0.0, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# State update: closed forms
+# --------------------------------------------------------------------------
+
+def test_alpha_one_beta_zero_leaves_state_unchanged():
+    rng = np.random.default_rng(7)
+    x = make(rng)
+    _, S1 = run(x, clean=True, alpha=np.ones_like(x["alpha"]), beta=np.zeros_like(x["beta"]))
+    assert np.array_equal(S1, x["S"])
+
+
+def test_one_token_unit_key_alpha_beta_one_stores_value():
+    # k' S_N = v' for ||k'|| = 1 and alpha = beta = 1, whatever S_{N-1}.
+    rng = np.random.default_rng(8)
+    B, L, H, d = 2, 1, 3, 8
+    x = make(rng, B=B, L=L, H=H, d=d)
+    # identity maps, so k' = k / ||k|| and v' = v independently of phi
+    _, S1 = run(x, clean=True, wk=eye_w(H, d), wv=eye_w(H, d), alpha=np.ones((B, H)),
+                beta=np.ones((B, H, L)))
+    for b in range(B):
+        for h in range(H):
+            kp = x["k"][b, 0, h] / np.linalg.norm(x["k"][b, 0, h])
+            np.testing.assert_allclose(kp @ S1[b, h], x["v"][b, 0, h], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("L", [1, 4, 8])
+def test_orthonormal_keys_closed_form(L):
+    # With orthonormal k' rows (L <= d): k'_i S_N = alpha k'_i S + beta_i (v'_i - k'_i S).
+    # Rows of K are orthonormal rows scaled by positive factors, W_k = I, so
+    # the L2 normalisation must undo the scaling.
+    rng = np.random.default_rng(10 + L)
+    B, H, d = 1, 2, 8
+    x = make(rng, B=B, L=L, H=H, d=d)
+    k = np.zeros((B, L, H, d))
+    for h in range(H):
+        qmat, _ = np.linalg.qr(rng.standard_normal((d, d)))
+        k[0, :, h, :] = qmat[:L] * rng.uniform(0.5, 3.0, size=(L, 1))
+    beta = rng.uniform(0.1, 0.9, size=(B, H, L))
+    alpha = rng.uniform(0.3, 0.95, size=(B, H))
+    _, S1 = run(x, clean=True, k=k, wk=eye_w(H, d), wv=eye_w(H, d), beta=beta, alpha=alpha)
+    vp = x["v"]
+    for h in range(H):
+        kp = k[0, :, h, :] / np.linalg.norm(k[0, :, h, :], axis=1, keepdims=True)
+        S0 = x["S"][0, h]
+        lhs = kp @ S1[0, h]
+        rhs = alpha[0, h] * (kp @ S0) + beta[0, h][:, None] * (vp[0, :, h] - kp @ S0)
+        np.testing.assert_allclose(lhs, rhs, rtol=0, atol=1e-12)
+
+
+def test_update_from_zero_state_is_rank_L_outer_product_sum():
+    # S_{N-1} = 0: S_N = sum_i beta_i k'_i^T v'_i, so S_N lies in span(k'_i)
+    # on the row side and span(v'_i) on the column side.
+    rng = np.random.default_rng(11)
+    B, L, H, d = 1, 3, 1, 8
+    x = make(rng, B=B, L=L, H=H, d=d)
+    _, S1 = run(x, clean=True, S=np.zeros((B, H, d, d)))
+    kp = oracle.phi(x["k"], x["wk"], True)[0, :, 0]
+    vp = oracle.phi(x["v"], x["wv"], False)[0, :, 0]
+    assert np.linalg.matrix_rank(S1[0, 0], tol=1e-10) == L
+    # project out span(k') from the rows: nothing is left
+    Qk, _ = np.linalg.qr(kp.T)
+    np.testing.assert_allclose(S1[0, 0] - Qk @ (Qk.T @ S1[0, 0]), 0.0, atol=1e-12)
+    Qv, _ = np.linalg.qr(vp.T)
+    np.testing.assert_allclose(S1[0, 0] - (S1[0, 0] @ Qv) @ Qv.T, 0.0, atol=1e-12)
+
+
+def test_key_normalisation_is_scale_invariant():
+    rng = np.random.default_rng(12)
+    x = make(rng)
+    _, S1 = run(x, clean=True)
+    c = rng.uniform(0.25, 4.0, size=x["k"].shape[:3] + (1,))
+    _, S2 = run(x, clean=True, k=x["k"] * c)
+    np.testing.assert_allclose(S2, S1, rtol=0, atol=1e-13)
+    _, S3 = run(x, clean=True, wk=3.0 * x["wk"])
+    np.testing.assert_allclose(S3, S1, rtol=0, atol=1e-13)
+
+
+def test_phi_k_rows_have_unit_norm_and_phi_v_is_unnormalised():
+    rng = np.random.default_rng(13)
+    x = make(rng)
+    kp = oracle.phi(x["k"], x["wk"], True)
+    np.testing.assert_allclose(np.linalg.norm(kp, axis=-1), 1.0, atol=1e-13)
+    vp = oracle.phi(x["v"], x["wv"], False)
+    np.testing.assert_allclose(oracle.phi(2.0 * x["v"], x["wv"], False), 2.0 * vp, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# Clean-pass updates and frame-level access (section 2.2)
+# --------------------------------------------------------------------------
+
+def test_non_clean_pass_keeps_state_bit_identical():
+    rng = np.random.default_rng(14)
+    x = make(rng)
+    _, S1 = run(x, clean=False)
+    assert np.array_equal(S1, x["S"])
+
+
+def test_clean_pass_output_reads_pre_update_state():
+    rng = np.random.default_rng(15)
+    x = make(rng)
+    o_read, _ = run(x, clean=False)
+    o_clean, S1 = run(x, clean=True)
+    assert np.array_equal(o_read, o_clean)
+    assert not np.array_equal(S1, x["S"])
+
+
+def test_token_permutation_permutes_output_and_keeps_state():
+    rng = np.random.default_rng(16)
+    x = make(rng, L=11)
+    perm = rng.permutation(11)
+    o1, S1 = run(x, clean=True)
+    o2, S2 = run(x, clean=True, q=x["q"][:, perm], k=x["k"][:, perm], v=x["v"][:, perm],
+                 beta=x["beta"][:, :, perm])
+    np.testing.assert_allclose(o2, o1[:, perm], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(S2, S1, rtol=0, atol=1e-14)
+
+
+def test_streams_and_heads_are_independent():
+    rng = np.random.default_rng(17)
+    x = make(rng, B=3, H=2)
+    o, S = run(x, clean=True)
+    for b in range(3):
+        for h in range(2):
+            sl = dict(q=x["q"][b:b + 1, :, h:h + 1], k=x["k"][b:b + 1, :, h:h + 1],
+                      v=x["v"][b:b + 1, :, h:h + 1], wq=x["wq"][h:h + 1], wk=x["wk"][h:h + 1],
+                      wv=x["wv"][h:h + 1], alpha=x["alpha"][b:b + 1, h:h + 1],
+                      beta=x["beta"][b:b + 1, h:h + 1], S=x["S"][b:b + 1, h:h + 1])
+            ob, Sb = run(sl, clean=True)
+            np.testing.assert_array_equal(ob[0, :, 0], o[b, :, h])
+            np.testing.assert_array_equal(Sb[0, 0], S[b, h])
+
+
+def test_rows_entry_matches_full_pass_rows():
+    rng = np.random.default_rng(18)
+    x = make(rng, B=2, L=9)
+    o, _ = run(x, clean=False)
+    rb, rt = [0, 1, 1, 0], [0, 8, 3, 5]
+    r = oracle.rows(x["q"], x["k"], x["v"], x["wq"], x["S"], rb, rt)
+    for i, (b, t) in enumerate(zip(rb, rt)):
+        np.testing.assert_array_equal(r[i], o[b, t])
+
+
+def test_state_stays_bounded_over_a_long_stream():
+    # alpha < 1 and beta ~ 1/L keep the state bounded: a 200-frame stream of
+    # the tiny workload's distributions must not grow without limit.
+    rng = np.random.default_rng(19)
+    B, L, H, d = 1, 16, 1, 16
+    S = np.zeros((B, H, d, d))
+    wq, wk, wv = (np.eye(d)[None] + rnd(rng, H, d, d, scale=0.02) for _ in range(3))
+    norms = []
+    for f in range(200):
+        k, v = rnd(rng, B, L, H, d), rnd(rng, B, L, H, d)
+        alpha = 1 / (1 + np.exp(-(2 + 0.5 * rnd(rng, B, H))))
+        beta = 1 / (1 + np.exp(-rnd(rng, B, H, L))) / L
+        S = oracle.state_update(k, v, wk, wv, alpha, beta, S)
+        norms.append(np.linalg.norm(S))
+    assert max(norms[100:]) < 3.0 * max(norms[:100]) + 1e-9
+    assert all(math.isfinite(n) for n in norms)
+
+
+def test_oracle_rejects_bad_arguments():
+    with pytest.raises(RuntimeError):
+        oracle.rows(np.zeros((1, 2, 1, 4)), np.zeros((1, 2, 1, 4)), np.zeros((1, 2, 1, 4)),
+                    np.zeros((1, 4, 4)), np.zeros((1, 1, 4, 4)), [0], [2])
