@@ -1,0 +1,394 @@
+"""Benchmark of the ARL2 hybrid attention layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 480p_bf16]
+                    [--impl reference]
+
+One step = one whole stream of the workload through the C ABI: state reset,
+then every frame's denoising passes (read-only passes, then the clean pass
+that updates the state).  For the default 480p workload that is 21 latent
+frames x 4 passes of 12 heads x 128 dims x 1560 tokens.  Inputs for every
+pass are generated once, resident in HBM (1.2 GB, larger than the 126 MB L2)
+before timing starts.
+
+Printed (rank 0, one JSON line): frames/s over all ranks, the fused
+attention kernel's roofline (algorithmic FLOPs per launch over its
+CUDA-event duration, against the measured bf16 tensor peak), SM clocks
+sampled during the timed region, an end-to-end number through the
+host-buffer entry point, and the CPU oracle's frames/s on a bounded sample.
+
+N > 1 (torchrun): every rank runs its own independent stream (replicas, no
+collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+import workloads
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+
+
+# ----------------------------------------------------------------- flops --
+def attn_flops(w: workloads.Workload) -> float:
+    """Algorithmic FLOPs of one fused-kernel launch: intra-frame softmax
+    attention 4 L^2 d H plus the state read 2 L d^2 H, per stream."""
+    L, d, H, B = w.tokens, w.head_dim, w.heads, w.batch
+    return (4.0 * L * L * d * H + 2.0 * L * d * d * H) * B
+
+
+def frame_flops(w: workloads.Workload) -> float:
+    """Algorithmic FLOPs of one frame: every pass 4L^2dH + 2Ld^2H + 2Ld^2H
+    (intra, read, phi_q); the clean pass adds 4Ld^2H (phi_k, phi_v) and
+    4Ld^2H (update)."""
+    L, d, H, B = w.tokens, w.head_dim, w.heads, w.batch
+    per_pass = 4.0 * L * L * d * H + 4.0 * L * d * d * H
+    return B * (w.passes * per_pass + 8.0 * L * d * d * H)
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ---------------------------------------------------------------- clocks --
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            out_dir = os.path.join(ROOT, "gpurun_out") if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else "/tmp"
+            self.path = os.path.join(out_dir, f"clocks_{os.getpid()}.csv")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", ident, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        try:
+            rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
+        except Exception:
+            return None
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = max(mx, float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() in ("active", "0x1") or v == "1":
+                    reasons.add(n)
+        if not sm:
+            return None
+        loaded = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ distributed --
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# -------------------------------------------------------------- CPU side --
+def oracle_frame_seconds(w: workloads.Workload, budget_s: float = 12.0):
+    """Time the CPU oracle on a bounded sample of one frame and scale it to
+    a whole frame: the clean pass's full state update, plus R sampled output
+    rows (all heads) for each pass, scaled by L / R.  Returns
+    (seconds per frame, threads, description)."""
+    import oracle
+    wq, wk, wv = workloads.phi_weights(w, 0)
+    alpha, beta = workloads.frame_gates(w, 0, 0)
+    ins = [workloads.pass_inputs(w, 0, 0, p) for p in range(w.passes)]
+    S = oracle.zero_state(w.batch, w.heads, w.head_dim)
+    q, k, v = ins[-1]
+    t0 = time.perf_counter()
+    S = oracle.state_update(k, v, wk, wv, alpha, beta, S)
+    t_update = time.perf_counter() - t0
+    R = 8
+    while True:
+        rt = np.arange(R) % w.tokens
+        rb = np.zeros(R, dtype=np.int64)
+        t0 = time.perf_counter()
+        for p in range(w.passes):
+            q, k, v = ins[p]
+            oracle.rows(q, k, v, wq, S, rb, rt)
+        t_rows = time.perf_counter() - t0
+        if t_rows > 0.25 * budget_s or R >= w.tokens:
+            break
+        R = min(w.tokens, R * 4)
+    per_frame = w.batch * (t_update / w.batch + t_rows * (w.tokens / R))
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    desc = (f"oracle fp64: one full clean-pass state update ({t_update:.2f} s) plus {R} output rows x "
+            f"{w.passes} passes ({t_rows:.2f} s), rows scaled by L/R={w.tokens / R:.1f} to one frame")
+    return per_frame, threads, desc
+
+
+def run_reference(args, w: workloads.Workload):
+    """--impl reference: the CPU oracle as it stands, on a bounded sample per step."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    wq, wk, wv = workloads.phi_weights(w, 0)
+    alpha, beta = workloads.frame_gates(w, 0, 0)
+    ins = [workloads.pass_inputs(w, 0, 0, p) for p in range(w.passes)]
+    R = 16
+    rb = np.zeros(R, dtype=np.int64)
+    rt = (np.arange(R) * 97) % w.tokens
+
+    def step(S):
+        t0 = time.perf_counter()
+        for p in range(w.passes):
+            q, k, v = ins[p]
+            oracle.rows(q, k, v, wq, S, rb, rt)
+        t_rows = time.perf_counter() - t0
+        t1 = time.perf_counter()
+        q, k, v = ins[-1]
+        S = oracle.state_update(k, v, wk, wv, alpha, beta, S)
+        t_up = time.perf_counter() - t1
+        return S, t_up + t_rows * (w.tokens / R)  # oracle seconds for one whole frame
+
+    S = oracle.zero_state(w.batch, w.heads, w.head_dim)
+    for _ in range(args.warmup):
+        S, _ = step(S)
+    frame_secs = []
+    for _ in range(args.steps):
+        S, fs = step(S)
+        frame_secs.append(fs)
+    spf = float(np.mean(frame_secs))
+    value = w.batch / spf
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = (f"per step: one full clean-pass state update plus {R} output rows x {w.passes} passes "
+              f"of one {w.name} frame, rows scaled by L/R to a whole frame")
+    line = {
+        "impl": "reference", "metric": "hybrid-attn frames/s", "value": value, "unit": "frames/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": spf * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
+                   "tokens_per_frame": w.tokens, "frames": w.frames, "passes": w.passes},
+        "cpu_baseline": {"value": value, "unit": "frames/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------------- GPU side --
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="480p_bf16")
+    ap.add_argument("--impl", default="arl2", choices=["arl2", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = workloads.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    if args.warmup < 3:
+        raise SystemExit("at least 3 warm-up steps")
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from hybrid_softmax_gated_b200 import Arl2Layer
+
+    stream_idx = rank  # each rank: its own independent stream (replica)
+    wq, wk, wv = workloads.phi_weights(w, 0)
+    lay = Arl2Layer(w.batch, w.heads, w.head_dim, w.tokens, wq.cuda(), wk.cuda(), wv.cuda(),
+                    dtype=w.torch_dtype, host_staging=True)
+    # all inputs of the stream, resident in HBM before timing
+    ins, gates = [], []
+    for f in range(w.frames):
+        a, b = workloads.frame_gates(w, stream_idx, f)
+        gates.append((a.cuda(), b.cuda()))
+        for p in range(w.passes):
+            ins.append(workloads.pass_inputs(w, stream_idx, f, p, device="cuda"))
+    out = torch.empty_like(ins[0][0])
+    st = torch.cuda.current_stream()
+    n_read = w.frames * (w.passes - 1)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n_read)]
+
+    def step(time_kernels: bool):
+        lay.state_reset()
+        i = r = 0
+        for f in range(w.frames):
+            a, b = gates[f]
+            for p in range(w.passes):
+                q, k, v = ins[i]
+                i += 1
+                clean = workloads.is_clean(w, p)
+                if time_kernels and not clean:
+                    ev[r][0].record(st)
+                lay.forward(q, k, v, a, b, clean_pass=clean, out=out)
+                if time_kernels and not clean:
+                    ev[r][1].record(st)
+                    r += 1
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    assert lay.device_status() == 0
+
+    clocks = ClockSampler(local)
+    kernel_ms = []
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    start.record(st)
+    for _ in range(args.steps):
+        step(True)
+        # per-launch durations of the fused kernel (read-only passes launch only it)
+        stop.record(st)
+        stop.synchronize()
+        kernel_ms.extend(e0.elapsed_time(e1) for e0, e1 in ev)
+    torch.cuda.synchronize()
+    barrier(ws)
+    elapsed_ms = start.elapsed_time(stop)
+    clk = clocks.stop()
+    status = lay.device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status}")
+    t_max = max_over_ranks(elapsed_ms, ws)
+    frames_total = args.steps * w.frames * w.batch * ws
+    value = frames_total / (t_max / 1e3)
+
+    # end to end: host (pinned) buffers through arl2_frame_forward_host
+    ring = 8
+    host_in = [tuple(t.cpu().pin_memory() for t in ins[i]) for i in range(ring)]
+    host_gates = [tuple(t.cpu().pin_memory() for t in gates[f]) for f in range(min(ring, w.frames))]
+    host_out = torch.empty(ins[0][0].shape, dtype=ins[0][0].dtype).pin_memory()
+    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h2d = d2h = 0
+    tok_bytes = ins[0][0].numel() * ins[0][0].element_size()
+    gate_bytes = (gates[0][0].numel() + gates[0][1].numel()) * 4
+
+    def e2e_step():
+        lay.state_reset()
+        i = 0
+        for f in range(w.frames):
+            a, b = host_gates[f % len(host_gates)]
+            for p in range(w.passes):
+                q, k, v = host_in[i % ring]
+                i += 1
+                lay.forward_host(q, k, v, a, b, workloads.is_clean(w, p), host_out)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e_start.record(st)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e_stop.record(st)
+    e_stop.synchronize()
+    barrier(ws)
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_stop), ws)
+    h2d = w.frames * (w.passes * 3 * tok_bytes + gate_bytes)
+    d2h = w.frames * w.passes * tok_bytes
+    e2e_value = args.e2e_steps * w.frames * w.batch * ws / (e2e_ms / 1e3)
+
+    peaks = load_peaks()
+    k_ms = float(np.mean(kernel_ms))
+    achieved = attn_flops(w) / (k_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None, "kernel": "attn_tc_kernel",
+                "kernel_ms": k_ms, "flops_per_launch": attn_flops(w),
+                "peak_kind": f"bf16 sustained ({peaks['source']})",
+                "frac_of_burst": achieved / peaks["bf16_tflops"]}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        spf, threads, desc = oracle_frame_seconds(w)
+        cpu = {"value": w.batch / spf, "unit": "frames/s", "cores": threads, "kind": "oracle",
+               "sample": desc}
+
+    launches_per_step = (w.frames * (w.passes - 1)) * 1 + w.frames * (1 + 5)
+    line = {
+        "metric": "hybrid-attn frames/s (12h x 128d, 1560 tok/frame) & % of B200 BF16 tensor peak",
+        "value": value, "unit": "frames/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
+                   "tokens_per_frame": w.tokens, "frames_per_step": w.frames, "passes": w.passes,
+                   "parallelism": f"replicas{ws}", "l2": "inputs larger than L2 (1.2 GB ring)"},
+        "tokens_per_s": value * w.tokens,
+        "tflops_per_frame_algorithmic": frame_flops(w) / 1e12,
+        "roofline": roofline, "clocks": clk,
+        "e2e": {"value": e2e_value, "unit": "frames/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * launches_per_step * ws,
+        "cpu_baseline": cpu,
+        "peak_device_bytes": torch.cuda.max_memory_allocated() + lay.device_bytes(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    lay.close()
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,241 @@
+"""ARL2 hybrid attention layer on B200: Python binding of libarl2.so.
+
+Argument marshalling only: every step of the layer runs in the CUDA
+kernels of ``libarl2.so`` (C ABI in ``include/arl2.h``).  PyTorch supplies
+device memory and streams.  If the library is missing, importing this
+package raises; there is no other implementation to fall back on.
+
+The layer ("Attend Locally, Remember Linearly", technical summary §2.1 and
+§2.2), per stream b and head h of one latent frame and denoising pass:
+
+    out = softmax(Q K^T / sqrt(d)) V + (Q W_q[h]) S_{N-1}
+    clean pass only, after the read:
+    S_N = alpha S_{N-1} + K'^T diag(beta) (V' - K' S_{N-1}),
+    K' = rownorm(K W_k[h]), V' = V W_v[h]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libarl2.so")
+
+ARL2_OK = 0
+ARL2_ERR_TIMEOUT = -6
+ARL2_BF16, ARL2_FP32 = 0, 1
+ARL2_IMPL_AUTO, ARL2_IMPL_SIMT = 0, 1
+
+EXPORTED = (
+    "arl2_create", "arl2_frame_forward", "arl2_frame_forward_host", "arl2_state_reset",
+    "arl2_state_get", "arl2_state_set", "arl2_phi_apply", "arl2_device_status",
+    "arl2_device_bytes", "arl2_destroy", "arl2_status_string", "arl2_version",
+)
+
+
+class Arl2Config(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int), ("heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+        ("tokens_per_frame", ctypes.c_int), ("dtype", ctypes.c_int),
+        ("w_q", ctypes.c_void_p), ("w_k", ctypes.c_void_p), ("w_v", ctypes.c_void_p),
+        ("softmax_scale", ctypes.c_float), ("host_staging", ctypes.c_int), ("impl", ctypes.c_int),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m hybrid_softmax_gated_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    H = ctypes.c_void_p
+    sig = {
+        "arl2_create": ([ctypes.POINTER(Arl2Config), P, ctypes.POINTER(H)], I),
+        "arl2_frame_forward": ([H, P, P, P, P, P, I, P, P], I),
+        "arl2_frame_forward_host": ([H, P, P, P, P, P, I, P, P], I),
+        "arl2_state_reset": ([H, P], I),
+        "arl2_state_get": ([H, P, P], I),
+        "arl2_state_set": ([H, P, P], I),
+        "arl2_phi_apply": ([H, I, P, P, P], I),
+        "arl2_device_status": ([H, P], I),
+        "arl2_device_bytes": ([H], S),
+        "arl2_destroy": ([H], None),
+        "arl2_status_string": ([I], ctypes.c_char_p),
+        "arl2_version": ([], I),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+class Arl2Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_lib.arl2_status_string(status).decode()} ({status})")
+
+
+def _check(status: int, what: str) -> None:
+    if status != ARL2_OK:
+        raise Arl2Error(status, what)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def version() -> int:
+    return _lib.arl2_version()
+
+
+class Arl2Layer:
+    """One ARL2 hybrid attention layer: B streams, H heads, width d, L tokens.
+
+    w_q, w_k, w_v: CUDA tensors [H, d, d] in the layer dtype (bf16 or fp32),
+    row = input feature.  The handle copies them and owns the fp32 state
+    S [B, H, d, d] (zero at creation).
+    """
+
+    def __init__(self, batch: int, heads: int, head_dim: int, tokens: int, w_q, w_k, w_v, *,
+                 dtype: torch.dtype = torch.bfloat16, softmax_scale: float = 0.0,
+                 host_staging: bool = False, impl: str = "auto", stream=None):
+        if dtype not in (torch.bfloat16, torch.float32):
+            raise ValueError("dtype must be torch.bfloat16 or torch.float32")
+        for w in (w_q, w_k, w_v):
+            if not (w.is_cuda and w.is_contiguous() and w.dtype == dtype):
+                raise ValueError("feature maps must be contiguous CUDA tensors of the layer dtype")
+            if tuple(w.shape) != (heads, head_dim, head_dim):
+                raise ValueError("feature maps must be [H, d, d]")
+        self.shape = (batch, tokens, heads, head_dim)
+        self.dtype = dtype
+        self.device = w_q.device
+        cfg = Arl2Config(batch, heads, head_dim, tokens,
+                         ARL2_BF16 if dtype == torch.bfloat16 else ARL2_FP32,
+                         w_q.data_ptr(), w_k.data_ptr(), w_v.data_ptr(), float(softmax_scale),
+                         1 if host_staging else 0,
+                         {"auto": ARL2_IMPL_AUTO, "simt": ARL2_IMPL_SIMT}[impl])
+        h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            _check(_lib.arl2_create(ctypes.byref(cfg), _stream(stream), ctypes.byref(h)), "arl2_create")
+        self._h = h
+
+    # -- helpers --------------------------------------------------------
+    def _tok(self, t, name):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == self.dtype):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor of the layer dtype")
+        if tuple(t.shape) != self.shape:
+            raise ValueError(f"{name} must have shape {self.shape}")
+        return t
+
+    @property
+    def handle(self):
+        if self._h is None:
+            raise RuntimeError("layer is closed")
+        return self._h
+
+    # -- C ABI calls ----------------------------------------------------
+    def forward(self, q, k, v, alpha=None, beta=None, clean_pass: bool = False, out=None,
+                stream=None):
+        """One denoising pass; returns out [B, L, H, d].  alpha [B, H] and
+        beta [B, H, L] (fp32 CUDA) are needed on the clean pass only."""
+        self._tok(q, "q"), self._tok(k, "k"), self._tok(v, "v")
+        if out is None:
+            out = torch.empty_like(q)
+        self._tok(out, "out")
+        B, L, H, _ = self.shape
+        if clean_pass:
+            if alpha is None or beta is None:
+                raise ValueError("the clean pass needs alpha and beta")
+            if not (alpha.is_cuda and alpha.dtype == torch.float32 and alpha.is_contiguous()
+                    and tuple(alpha.shape) == (B, H)):
+                raise ValueError("alpha must be a contiguous fp32 CUDA tensor [B, H]")
+            if not (beta.is_cuda and beta.dtype == torch.float32 and beta.is_contiguous()
+                    and tuple(beta.shape) == (B, H, L)):
+                raise ValueError("beta must be a contiguous fp32 CUDA tensor [B, H, L]")
+        _check(_lib.arl2_frame_forward(self.handle, _ptr(q), _ptr(k), _ptr(v),
+                                       _ptr(alpha) if clean_pass else None,
+                                       _ptr(beta) if clean_pass else None,
+                                       1 if clean_pass else 0, _ptr(out), _stream(stream)),
+               "arl2_frame_forward")
+        return out
+
+    def forward_host(self, q, k, v, alpha, beta, clean_pass: bool, out, stream=None):
+        """arl2_frame_forward_host: q, k, v, alpha, beta, out are host (pinned) tensors."""
+        for t in (q, k, v, out):
+            if t.is_cuda or not t.is_contiguous() or tuple(t.shape) != self.shape or t.dtype != self.dtype:
+                raise ValueError("host token tensors must be contiguous CPU tensors of the layer shape")
+        if clean_pass and (alpha is None or beta is None or alpha.is_cuda or beta.is_cuda):
+            raise ValueError("the clean pass needs host alpha and beta")
+        _check(_lib.arl2_frame_forward_host(self.handle, _ptr(q), _ptr(k), _ptr(v),
+                                            _ptr(alpha) if clean_pass else None,
+                                            _ptr(beta) if clean_pass else None,
+                                            1 if clean_pass else 0, _ptr(out), _stream(stream)),
+               "arl2_frame_forward_host")
+        return out
+
+    def state_reset(self, stream=None) -> None:
+        _check(_lib.arl2_state_reset(self.handle, _stream(stream)), "arl2_state_reset")
+
+    def state_get(self, out=None, stream=None):
+        B, _, H, d = self.shape
+        if out is None:
+            out = torch.empty(B, H, d, d, dtype=torch.float32, device=self.device)
+        _check(_lib.arl2_state_get(self.handle, _ptr(out), _stream(stream)), "arl2_state_get")
+        return out
+
+    def state_set(self, src, stream=None) -> None:
+        B, _, H, d = self.shape
+        if not (src.is_cuda and src.dtype == torch.float32 and src.is_contiguous()
+                and tuple(src.shape) == (B, H, d, d)):
+            raise ValueError("state must be a contiguous fp32 CUDA tensor [B, H, d, d]")
+        _check(_lib.arl2_state_set(self.handle, _ptr(src), _stream(stream)), "arl2_state_set")
+
+    def phi_apply(self, which: str, x, out=None, stream=None):
+        """which in {"q", "k", "v"}: x W_q, rownorm(x W_k) or x W_v."""
+        self._tok(x, "x")
+        if out is None:
+            out = torch.empty_like(x)
+        self._tok(out, "out")
+        _check(_lib.arl2_phi_apply(self.handle, {"q": 0, "k": 1, "v": 2}[which], _ptr(x), _ptr(out),
+                                   _stream(stream)), "arl2_phi_apply")
+        return out
+
+    def device_status(self, stream=None) -> int:
+        """Synchronise and return the device status code (0, or ARL2_ERR_TIMEOUT)."""
+        return _lib.arl2_device_status(self.handle, _stream(stream))
+
+    def device_bytes(self) -> int:
+        return int(_lib.arl2_device_bytes(self.handle))
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None:
+            _lib.arl2_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()

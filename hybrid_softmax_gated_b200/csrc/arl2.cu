@@ -1,0 +1,332 @@
+// Host side of libarl2.so: the C ABI declared in include/arl2.h.
+//
+// The handle owns the fp32 state S[B][H][d][d], its bf16 derived copies
+// for the tensor-core kernels, copies of the three feature maps, and every
+// workspace.  All of it is allocated in arl2_create; no later call
+// allocates, which keeps device memory flat over arbitrarily long streams
+// (the constant-memory property the ARL2 pages claim for the fixed-size
+// state, technical summary §1 and §4 "Memory").
+#include "arl2.h"
+#include "internal.h"
+#include "attn_tc.h"
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+using arl2::Dims;
+
+struct arl2_handle {
+    int device = -1;
+    Dims dm{};
+    arl2_dtype dtype = ARL2_BF16;
+    arl2_impl impl = ARL2_IMPL_AUTO;
+    bool use_tc = false;      // tensor-core kernels for attention and update
+    float scale = 0.f;
+    size_t esz = 0;           // bytes per element of dtype
+    size_t n_tok = 0;         // B*L*H*d
+    size_t n_state = 0;       // B*H*d*d
+    size_t bytes = 0;         // device bytes held
+    void* w[3] = {nullptr, nullptr, nullptr};  // feature-map copies [H][d][d] dtype
+    float* S = nullptr;       // fp32 master state
+    void* Mt = nullptr;       // bf16 (W_q S)^T, tensor-core read
+    void* St = nullptr;       // bf16 S^T, tensor-core update
+    float* qp = nullptr;      // fp32 workspaces [B][L][H][d]
+    float* kp = nullptr;
+    float* vp = nullptr;
+    void* stage_tok[4] = {nullptr, nullptr, nullptr, nullptr};  // q, k, v, out
+    float* stage_alpha = nullptr;
+    float* stage_beta = nullptr;
+    int* err = nullptr;       // device error word
+    arl2::AttnTc* tc = nullptr;
+};
+
+namespace {
+
+constexpr int kMaxHeads = 1024;
+constexpr int kMaxBatch = 65535;
+constexpr int kMaxTokens = 1 << 20;
+constexpr int kMaxHeadDim = 128;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+arl2_status check_device(const arl2_handle* h) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ARL2_ERR_CUDA;
+    return dev == h->device ? ARL2_OK : ARL2_ERR_INVALID_ARG;
+}
+
+template <typename T>
+arl2_status dalloc(arl2_handle* h, T** p, size_t bytes) {
+    void* q = nullptr;
+    if (cudaMalloc(&q, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return ARL2_ERR_OOM;
+    }
+    *p = static_cast<T*>(q);
+    h->bytes += bytes;
+    return ARL2_OK;
+}
+
+void release(arl2_handle* h) {
+    if (!h) return;
+    if (h->tc) arl2::attn_tc_destroy(h->tc);
+    void* ptrs[] = {h->w[0], h->w[1], h->w[2], h->S, h->Mt, h->St, h->qp, h->kp, h->vp,
+                    h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], h->stage_tok[3],
+                    h->stage_alpha, h->stage_beta, h->err};
+    for (void* p : ptrs)
+        if (p) cudaFree(p);
+    delete h;
+}
+
+// Recompute the tensor-core copies of the state after it changed.
+arl2_status refresh_derived(arl2_handle* h, cudaStream_t st) {
+    if (!h->use_tc) return ARL2_OK;
+    if (arl2::launch_fold_state(h->w[0], h->S, h->Mt, h->St, h->dm, st) != cudaSuccess)
+        return ARL2_ERR_CUDA;
+    return ARL2_OK;
+}
+
+arl2_status clean_update(arl2_handle* h, const void* k, const void* v, const float* alpha,
+                         const float* beta, cudaStream_t st) {
+    const bool bf16 = h->dtype == ARL2_BF16;
+    if (arl2::launch_phi_simt(bf16, k, h->w[1], true, h->kp, nullptr, h->dm, st) != cudaSuccess)
+        return ARL2_ERR_CUDA;
+    if (arl2::launch_phi_simt(bf16, v, h->w[2], false, h->vp, nullptr, h->dm, st) != cudaSuccess)
+        return ARL2_ERR_CUDA;
+    if (arl2::launch_residual_simt(h->kp, h->vp, h->S, h->dm, st) != cudaSuccess)
+        return ARL2_ERR_CUDA;
+    if (arl2::launch_accum_simt(h->kp, h->vp, alpha, beta, h->S, h->dm, st) != cudaSuccess)
+        return ARL2_ERR_CUDA;
+    return refresh_derived(h, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int arl2_version(void) { return 10000; }
+
+const char* arl2_status_string(arl2_status s) {
+    switch (s) {
+        case ARL2_OK: return "ok";
+        case ARL2_ERR_INVALID_ARG: return "invalid argument";
+        case ARL2_ERR_SHAPE: return "unsupported shape";
+        case ARL2_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case ARL2_ERR_CUDA: return "CUDA error";
+        case ARL2_ERR_OOM: return "device out of memory";
+        case ARL2_ERR_TIMEOUT: return "kernel wait timed out";
+        case ARL2_ERR_UNSUPPORTED: return "unsupported dtype or head_dim for these kernels";
+    }
+    return "unknown status";
+}
+
+arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle** out) {
+    if (!cfg || !out) return ARL2_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (cfg->dtype != ARL2_BF16 && cfg->dtype != ARL2_FP32) return ARL2_ERR_INVALID_ARG;
+    if (cfg->impl != ARL2_IMPL_AUTO && cfg->impl != ARL2_IMPL_SIMT) return ARL2_ERR_INVALID_ARG;
+    if (!cfg->w_q || !cfg->w_k || !cfg->w_v) return ARL2_ERR_INVALID_ARG;
+    if (cfg->batch < 1 || cfg->batch > kMaxBatch || cfg->heads < 1 || cfg->heads > kMaxHeads ||
+        cfg->tokens_per_frame < 1 || cfg->tokens_per_frame > kMaxTokens || cfg->head_dim < 1 ||
+        cfg->head_dim > kMaxHeadDim)
+        return ARL2_ERR_SHAPE;
+    if (!(cfg->softmax_scale >= 0.f) || std::isinf(cfg->softmax_scale)) return ARL2_ERR_INVALID_ARG;
+    if (!aligned16(cfg->w_q) || !aligned16(cfg->w_k) || !aligned16(cfg->w_v)) return ARL2_ERR_ALIGN;
+    const bool use_tc = cfg->impl == ARL2_IMPL_AUTO && cfg->dtype == ARL2_BF16;
+    if (use_tc && cfg->head_dim != 128) return ARL2_ERR_UNSUPPORTED;
+
+    arl2_handle* h = new (std::nothrow) arl2_handle();
+    if (!h) return ARL2_ERR_OOM;
+    if (cudaGetDevice(&h->device) != cudaSuccess) {
+        delete h;
+        return ARL2_ERR_CUDA;
+    }
+    h->dm = Dims{cfg->batch, cfg->heads, cfg->head_dim, cfg->tokens_per_frame};
+    h->dtype = cfg->dtype;
+    h->impl = cfg->impl;
+    h->use_tc = use_tc;
+    h->scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->head_dim);
+    h->esz = cfg->dtype == ARL2_BF16 ? 2 : 4;
+    const Dims& dm = h->dm;
+    h->n_tok = (size_t)dm.B * dm.L * dm.H * dm.d;
+    h->n_state = (size_t)dm.B * dm.H * dm.d * dm.d;
+    const size_t wbytes = (size_t)dm.H * dm.d * dm.d * h->esz;
+
+    arl2_status s = ARL2_OK;
+    for (int i = 0; i < 3 && s == ARL2_OK; ++i) s = dalloc(h, &h->w[i], wbytes);
+    if (s == ARL2_OK) s = dalloc(h, &h->S, h->n_state * sizeof(float));
+    if (s == ARL2_OK && use_tc) s = dalloc(h, &h->Mt, h->n_state * 2);
+    if (s == ARL2_OK && use_tc) s = dalloc(h, &h->St, h->n_state * 2);
+    if (s == ARL2_OK && !use_tc) s = dalloc(h, &h->qp, h->n_tok * sizeof(float));
+    if (s == ARL2_OK) s = dalloc(h, &h->kp, h->n_tok * sizeof(float));
+    if (s == ARL2_OK) s = dalloc(h, &h->vp, h->n_tok * sizeof(float));
+    if (s == ARL2_OK) s = dalloc(h, &h->err, sizeof(int));
+    if (s == ARL2_OK && cfg->host_staging) {
+        for (int i = 0; i < 4 && s == ARL2_OK; ++i) s = dalloc(h, &h->stage_tok[i], h->n_tok * h->esz);
+        if (s == ARL2_OK) s = dalloc(h, &h->stage_alpha, (size_t)dm.B * dm.H * sizeof(float));
+        if (s == ARL2_OK) s = dalloc(h, &h->stage_beta, (size_t)dm.B * dm.H * dm.L * sizeof(float));
+    }
+    if (s == ARL2_OK && arl2::simt_init() != cudaSuccess) s = ARL2_ERR_CUDA;
+    if (s == ARL2_OK && use_tc) {
+        h->tc = arl2::attn_tc_create(dm);
+        if (!h->tc) s = ARL2_ERR_CUDA;
+    }
+    if (s != ARL2_OK) {
+        release(h);
+        return s;
+    }
+    const void* src[3] = {cfg->w_q, cfg->w_k, cfg->w_v};
+    for (int i = 0; i < 3; ++i)
+        if (cudaMemcpyAsync(h->w[i], src[i], wbytes, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+            s = ARL2_ERR_CUDA;
+    if (s == ARL2_OK && cudaMemsetAsync(h->S, 0, h->n_state * sizeof(float), stream) != cudaSuccess)
+        s = ARL2_ERR_CUDA;
+    if (s == ARL2_OK && use_tc &&
+        (cudaMemsetAsync(h->Mt, 0, h->n_state * 2, stream) != cudaSuccess ||
+         cudaMemsetAsync(h->St, 0, h->n_state * 2, stream) != cudaSuccess))
+        s = ARL2_ERR_CUDA;
+    if (s == ARL2_OK && cudaMemsetAsync(h->err, 0, sizeof(int), stream) != cudaSuccess)
+        s = ARL2_ERR_CUDA;
+    if (s != ARL2_OK) {
+        cudaStreamSynchronize(stream);
+        release(h);
+        return s;
+    }
+    *out = h;
+    return ARL2_OK;
+}
+
+arl2_status arl2_frame_forward(arl2_handle* h, const void* q, const void* k, const void* v,
+                               const float* alpha, const float* beta, int clean_pass, void* out,
+                               cudaStream_t stream) {
+    if (!h || !q || !k || !v || !out) return ARL2_ERR_INVALID_ARG;
+    if (clean_pass && (!alpha || !beta)) return ARL2_ERR_INVALID_ARG;
+    if (out == q || out == k || out == v) return ARL2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ARL2_ERR_ALIGN;
+    arl2_status s = check_device(h);
+    if (s != ARL2_OK) return s;
+    const bool bf16 = h->dtype == ARL2_BF16;
+    if (h->use_tc) {
+        if (arl2::attn_tc_launch(h->tc, q, k, v, h->Mt, out, h->scale, h->err, stream) != cudaSuccess)
+            return ARL2_ERR_CUDA;
+    } else {
+        if (arl2::launch_phi_simt(bf16, q, h->w[0], false, h->qp, nullptr, h->dm, stream) != cudaSuccess)
+            return ARL2_ERR_CUDA;
+        if (arl2::launch_attn_simt(bf16, q, k, v, h->qp, h->S, out, h->scale, h->dm, stream) !=
+            cudaSuccess)
+            return ARL2_ERR_CUDA;
+    }
+    if (clean_pass) return clean_update(h, k, v, alpha, beta, stream);
+    return ARL2_OK;
+}
+
+arl2_status arl2_frame_forward_host(arl2_handle* h, const void* q, const void* k, const void* v,
+                                    const float* alpha, const float* beta, int clean_pass,
+                                    void* out, cudaStream_t stream) {
+    if (!h || !q || !k || !v || !out) return ARL2_ERR_INVALID_ARG;
+    if (!h->stage_tok[0]) return ARL2_ERR_INVALID_ARG;
+    if (clean_pass && (!alpha || !beta)) return ARL2_ERR_INVALID_ARG;
+    arl2_status s = check_device(h);
+    if (s != ARL2_OK) return s;
+    const size_t tb = h->n_tok * h->esz;
+    const void* src[3] = {q, k, v};
+    for (int i = 0; i < 3; ++i)
+        if (cudaMemcpyAsync(h->stage_tok[i], src[i], tb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+            return ARL2_ERR_CUDA;
+    const float* a_dev = nullptr;
+    const float* b_dev = nullptr;
+    if (clean_pass) {
+        const Dims& dm = h->dm;
+        if (cudaMemcpyAsync(h->stage_alpha, alpha, (size_t)dm.B * dm.H * sizeof(float),
+                            cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+            cudaMemcpyAsync(h->stage_beta, beta, (size_t)dm.B * dm.H * dm.L * sizeof(float),
+                            cudaMemcpyHostToDevice, stream) != cudaSuccess)
+            return ARL2_ERR_CUDA;
+        a_dev = h->stage_alpha;
+        b_dev = h->stage_beta;
+    }
+    s = arl2_frame_forward(h, h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], a_dev, b_dev,
+                           clean_pass, h->stage_tok[3], stream);
+    if (s != ARL2_OK) return s;
+    if (cudaMemcpyAsync(out, h->stage_tok[3], tb, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return ARL2_ERR_CUDA;
+    return ARL2_OK;
+}
+
+arl2_status arl2_state_reset(arl2_handle* h, cudaStream_t stream) {
+    if (!h) return ARL2_ERR_INVALID_ARG;
+    arl2_status s = check_device(h);
+    if (s != ARL2_OK) return s;
+    if (cudaMemsetAsync(h->S, 0, h->n_state * sizeof(float), stream) != cudaSuccess)
+        return ARL2_ERR_CUDA;
+    if (h->use_tc && (cudaMemsetAsync(h->Mt, 0, h->n_state * 2, stream) != cudaSuccess ||
+                      cudaMemsetAsync(h->St, 0, h->n_state * 2, stream) != cudaSuccess))
+        return ARL2_ERR_CUDA;
+    return ARL2_OK;
+}
+
+arl2_status arl2_state_get(arl2_handle* h, float* dst, cudaStream_t stream) {
+    if (!h || !dst) return ARL2_ERR_INVALID_ARG;
+    arl2_status s = check_device(h);
+    if (s != ARL2_OK) return s;
+    if (cudaMemcpyAsync(dst, h->S, h->n_state * sizeof(float), cudaMemcpyDeviceToDevice, stream) !=
+        cudaSuccess)
+        return ARL2_ERR_CUDA;
+    return ARL2_OK;
+}
+
+arl2_status arl2_state_set(arl2_handle* h, const float* src, cudaStream_t stream) {
+    if (!h || !src) return ARL2_ERR_INVALID_ARG;
+    arl2_status s = check_device(h);
+    if (s != ARL2_OK) return s;
+    if (cudaMemcpyAsync(h->S, src, h->n_state * sizeof(float), cudaMemcpyDeviceToDevice, stream) !=
+        cudaSuccess)
+        return ARL2_ERR_CUDA;
+    return refresh_derived(h, stream);
+}
+
+arl2_status arl2_phi_apply(arl2_handle* h, int which, const void* x, void* out,
+                           cudaStream_t stream) {
+    if (!h || !x || !out || which < 0 || which > 2) return ARL2_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(out)) return ARL2_ERR_ALIGN;
+    arl2_status s = check_device(h);
+    if (s != ARL2_OK) return s;
+    const bool bf16 = h->dtype == ARL2_BF16;
+    if (arl2::launch_phi_simt(bf16, x, h->w[which], which == 1, nullptr, out, h->dm, stream) !=
+        cudaSuccess)
+        return ARL2_ERR_CUDA;
+    return ARL2_OK;
+}
+
+arl2_status arl2_device_status(arl2_handle* h, cudaStream_t stream) {
+    if (!h) return ARL2_ERR_INVALID_ARG;
+    arl2_status s = check_device(h);
+    if (s != ARL2_OK) return s;
+    int word = 0;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return ARL2_ERR_CUDA;
+    if (cudaMemcpy(&word, h->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return ARL2_ERR_CUDA;
+    if (word != 0) {
+        if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess) return ARL2_ERR_CUDA;
+        return ARL2_ERR_TIMEOUT;
+    }
+    return ARL2_OK;
+}
+
+size_t arl2_device_bytes(const arl2_handle* h) { return h ? h->bytes : 0; }
+
+void arl2_destroy(arl2_handle* h) {
+    if (!h) return;
+    const int dev = h->device;
+    int prev = -1;
+    cudaGetDevice(&prev);
+    if (prev != dev) cudaSetDevice(dev);
+    cudaDeviceSynchronize();
+    release(h);
+    if (prev >= 0 && prev != dev) cudaSetDevice(prev);
+}
+
+}  // extern "C"

@@ -1,0 +1,22 @@
+// Tensor-core (tcgen05) kernel for the per-pass read of the ARL2 layer:
+//   out = softmax(Q K^T scale) V + Q (W_q S_{N-1})
+// bf16 in, fp32 accumulate in TMEM, bf16 out; head_dim 128.
+#pragma once
+
+#include "internal.h"
+
+namespace arl2 {
+
+struct AttnTc;
+
+// Resolve the driver's tensor-map encoder and configure the kernel for the
+// given dimensions.  Returns nullptr on failure (no driver, bad dims).
+AttnTc* attn_tc_create(Dims dm);
+void attn_tc_destroy(AttnTc* t);
+
+// q, k, v, out: [B][L][H][128] bf16.  Mt: [B][H][128][128] bf16 holding
+// (W_q S)^T.  err: device error word (bit kErrTimeoutAttn on a timeout).
+cudaError_t attn_tc_launch(AttnTc* t, const void* q, const void* k, const void* v,
+                           const void* Mt, void* out, float scale, int* err, cudaStream_t st);
+
+}  // namespace arl2

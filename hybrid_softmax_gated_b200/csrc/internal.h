@@ -1,0 +1,54 @@
+// Internal declarations shared by the host library and the kernel files of
+// libarl2.so.  Nothing here is part of the C ABI (see include/arl2.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace arl2 {
+
+// Problem dimensions of one handle: B streams, H heads, head width d,
+// L tokens per frame.  Token tensors are [B][L][H][d].
+struct Dims {
+    int B, H, d, L;
+};
+
+// Error word bits set by kernels whose bounded waits ran out.
+enum : int {
+    kErrTimeoutAttn = 1 << 0,
+    kErrTimeoutUpdate = 1 << 1,
+};
+
+// ---- SIMT kernels (fp32 arithmetic; T = float or __nv_bfloat16) ----------
+
+// One-time kernel attribute setup (dynamic shared memory limits); called by
+// arl2_create so that no launch path changes attributes (graph capture).
+cudaError_t simt_init();
+
+// out = x W[h] per head, optionally with L2-normalised rows.  Exactly one of
+// out_f (fp32) and out_t (element type of x) is non-null.
+cudaError_t launch_phi_simt(bool bf16, const void* x, const void* w, bool l2norm,
+                            float* out_f, void* out_t, Dims dm, cudaStream_t st);
+
+// out = softmax(Q K^T scale) V + qp S   (qp = Q W_q, fp32 [B][L][H][d])
+cudaError_t launch_attn_simt(bool bf16, const void* q, const void* k, const void* v,
+                             const float* qp, const float* S, void* out, float scale,
+                             Dims dm, cudaStream_t st);
+
+// r = vp - kp S, written over vp (fp32 [B][L][H][d]); S is the pre-update state.
+cudaError_t launch_residual_simt(const float* kp, float* vp_to_r, const float* S, Dims dm,
+                                 cudaStream_t st);
+
+// S = alpha S + kp^T diag(beta) r, in place.
+cudaError_t launch_accum_simt(const float* kp, const float* r, const float* alpha,
+                              const float* beta, float* S, Dims dm, cudaStream_t st);
+
+// Derived bf16 copies of the state used by the tensor-core kernels:
+// Mt[b][h][n][a] = sum_c Wq[h][a][c] S[b][h][c][n]   ((W_q S)^T)
+// St[b][h][n][c] = S[b][h][c][n]                      (S^T)
+cudaError_t launch_fold_state(const void* wq_bf16, const float* S, void* Mt, void* St, Dims dm,
+                              cudaStream_t st);
+
+}  // namespace arl2

@@ -1,0 +1,339 @@
+// SIMT kernels of the ARL2 layer, fp32 arithmetic on fp32 or bf16 storage.
+//
+// These carry the fp32 workloads (whose 1e-4 tolerance no bf16/tf32 tensor
+// core operand can meet) and serve as an independent GPU cross-check of the
+// tensor-core kernels.  Steps ("Attend Locally, Remember Linearly",
+// technical summary §2.1 and §2.2):
+//   phi      x' = x W[h] (+ row L2 norm for k')          §2.1 Adaptation
+//   attn     softmax(Q K^T s) V + (Q W_q) S_{N-1}          §2.1 items 1-2, Output
+//   residual r = v' - k' S_{N-1}                           §2.1 State Update
+//   accum    S = alpha S + k'^T diag(beta) r               §2.1 State Update
+//   fold     (W_q S)^T and S^T in bf16 for the tensor-core read and update
+#include "internal.h"
+
+#include <cmath>
+
+namespace arl2 {
+namespace {
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ size_t tok(int b, int t, int h, int c, const Dims& dm) {
+    return (((size_t)b * dm.L + t) * dm.H + h) * dm.d + c;
+}
+
+// ---------------------------------------------------------------- phi ----
+constexpr int kPhiRows = 32;
+
+template <typename T>
+__global__ void __launch_bounds__(128) phi_simt_kernel(const T* __restrict__ x,
+                                                       const T* __restrict__ w, int l2norm,
+                                                       float* __restrict__ out_f,
+                                                       T* __restrict__ out_t, Dims dm) {
+    extern __shared__ float sm[];
+    const int d = dm.d;
+    float* Ws = sm;                 // [d][d]
+    float* Xs = Ws + d * d;         // [kPhiRows][d]
+    float* Ys = Xs + kPhiRows * d;  // [kPhiRows][d]
+    __shared__ float inv[kPhiRows];
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int t0 = blockIdx.x * kPhiRows;
+    const int nt = min(kPhiRows, dm.L - t0);
+    for (int i = threadIdx.x; i < d * d; i += blockDim.x) Ws[i] = to_f(w[(size_t)h * d * d + i]);
+    for (int i = threadIdx.x; i < nt * d; i += blockDim.x) {
+        const int r = i / d, c = i - r * d;
+        Xs[i] = to_f(x[tok(b, t0 + r, h, c, dm)]);
+    }
+    __syncthreads();
+    const int c = threadIdx.x;
+    if (c < d) {
+        for (int r = 0; r < nt; ++r) {
+            float acc = 0.f;
+            for (int a = 0; a < d; ++a) acc = fmaf(Xs[r * d + a], Ws[a * d + c], acc);
+            Ys[r * d + c] = acc;
+        }
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int r = warp; r < nt; r += blockDim.x >> 5) {
+        float ss = 0.f;
+        if (l2norm)
+            for (int cc = lane; cc < d; cc += 32) ss = fmaf(Ys[r * d + cc], Ys[r * d + cc], ss);
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane == 0) inv[r] = l2norm ? 1.f / fmaxf(sqrtf(ss), 1e-6f) : 1.f;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < nt * d; i += blockDim.x) {
+        const int r = i / d, cc = i - r * d;
+        const float y = Ys[i] * inv[r];
+        const size_t o = tok(b, t0 + r, h, cc, dm);
+        if (out_f) out_f[o] = y;
+        else out_t[o] = from_f<T>(y);
+    }
+}
+
+// --------------------------------------------------------------- attn ----
+// One block: 32 query rows of one (b, h); 256 threads, thread (r, g) with
+// r = tid / 8 owns output columns g, g+8, g+16, ... of row r.  Keys stream
+// through shared memory 32 at a time with an online softmax.
+constexpr int kAQ = 32, kAK = 32, kAThreads = 256, kAColsPerThread = 16;
+
+template <typename T>
+__global__ void __launch_bounds__(kAThreads) attn_simt_kernel(
+    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+    const float* __restrict__ qp, const float* __restrict__ S, T* __restrict__ out,
+    float scale_log2, Dims dm) {
+    extern __shared__ float sm[];
+    const int d = dm.d;
+    float* Qs = sm;                    // [kAQ][d]
+    float* Ks = Qs + kAQ * d;          // [kAK][d + 1]
+    float* Vs = Ks + kAK * (d + 1);    // [kAK][d]
+    float* Ps = Vs + kAK * d;          // [kAQ][kAK + 1]
+    float* Ss = Ps + kAQ * (kAK + 1);  // [d][d]
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int q0 = blockIdx.x * kAQ;
+    const int nq = min(kAQ, dm.L - q0);
+    const int tid = threadIdx.x, r = tid >> 3, g = tid & 7;
+
+    for (int i = tid; i < kAQ * d; i += kAThreads) {
+        const int rr = i / d, c = i - rr * d;
+        Qs[i] = rr < nq ? to_f(q[tok(b, q0 + rr, h, c, dm)]) : 0.f;
+    }
+    float o[kAColsPerThread];
+#pragma unroll
+    for (int i = 0; i < kAColsPerThread; ++i) o[i] = 0.f;
+    float m = -INFINITY, l = 0.f;
+
+    for (int k0 = 0; k0 < dm.L; k0 += kAK) {
+        const int nk = min(kAK, dm.L - k0);
+        __syncthreads();  // previous tile fully consumed (and Qs written)
+        for (int i = tid; i < kAK * d; i += kAThreads) {
+            const int j = i / d, c = i - j * d;
+            const bool ok = j < nk;
+            Ks[j * (d + 1) + c] = ok ? to_f(k[tok(b, k0 + j, h, c, dm)]) : 0.f;
+            Vs[j * d + c] = ok ? to_f(v[tok(b, k0 + j, h, c, dm)]) : 0.f;
+        }
+        __syncthreads();
+        float s[4];
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const int j = g * 4 + jj;
+            float dot = 0.f;
+            for (int a = 0; a < d; ++a) dot = fmaf(Qs[r * d + a], Ks[j * (d + 1) + a], dot);
+            s[jj] = j < nk ? dot * scale_log2 : -INFINITY;
+            tmax = fmaxf(tmax, s[jj]);
+        }
+        for (int off = 1; off < 8; off <<= 1)
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
+        const float m_new = fmaxf(m, tmax);
+        const float corr = exp2f(m - m_new);
+        float psum = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const float p = exp2f(s[jj] - m_new);
+            Ps[r * (kAK + 1) + g * 4 + jj] = p;
+            psum += p;
+        }
+        for (int off = 1; off < 8; off <<= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
+        l = l * corr + psum;
+        m = m_new;
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < kAColsPerThread; ++i) o[i] *= corr;
+        for (int j = 0; j < nk; ++j) {
+            const float p = Ps[r * (kAK + 1) + j];
+#pragma unroll
+            for (int i = 0; i < kAColsPerThread; ++i) {
+                const int c = g + 8 * i;
+                if (c < d) o[i] = fmaf(p, Vs[j * d + c], o[i]);
+            }
+        }
+    }
+    const float inv_l = 1.f / l;
+    __syncthreads();
+    // inter-frame read: (q W_q) S with the pre-update state
+    const float* Sbh = S + ((size_t)b * dm.H + h) * d * d;
+    for (int i = tid; i < d * d; i += kAThreads) Ss[i] = Sbh[i];
+    for (int i = tid; i < kAQ * d; i += kAThreads) {
+        const int rr = i / d, c = i - rr * d;
+        Qs[i] = rr < nq ? qp[tok(b, q0 + rr, h, c, dm)] : 0.f;
+    }
+    __syncthreads();
+    if (r < nq) {
+#pragma unroll
+        for (int i = 0; i < kAColsPerThread; ++i) {
+            const int c = g + 8 * i;
+            if (c >= d) continue;
+            float acc = 0.f;
+            for (int a = 0; a < d; ++a) acc = fmaf(Qs[r * d + a], Ss[a * d + c], acc);
+            out[tok(b, q0 + r, h, c, dm)] = from_f<T>(o[i] * inv_l + acc);
+        }
+    }
+}
+
+// ----------------------------------------------------------- residual ----
+constexpr int kRRows = 32;
+
+__global__ void __launch_bounds__(128) residual_simt_kernel(const float* __restrict__ kp,
+                                                            float* __restrict__ vr,
+                                                            const float* __restrict__ S, Dims dm) {
+    extern __shared__ float sm[];
+    const int d = dm.d;
+    float* Ss = sm;          // [d][d]
+    float* Kt = Ss + d * d;  // [kRRows][d]
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int t0 = blockIdx.x * kRRows;
+    const int nt = min(kRRows, dm.L - t0);
+    const float* Sbh = S + ((size_t)b * dm.H + h) * d * d;
+    for (int i = threadIdx.x; i < d * d; i += blockDim.x) Ss[i] = Sbh[i];
+    for (int i = threadIdx.x; i < nt * d; i += blockDim.x) {
+        const int rr = i / d, c = i - rr * d;
+        Kt[i] = kp[tok(b, t0 + rr, h, c, dm)];
+    }
+    __syncthreads();
+    const int n = threadIdx.x;
+    if (n >= d) return;
+    for (int rr = 0; rr < nt; ++rr) {
+        float acc = 0.f;
+        for (int c = 0; c < d; ++c) acc = fmaf(Kt[rr * d + c], Ss[c * d + n], acc);
+        const size_t o = tok(b, t0 + rr, h, n, dm);
+        vr[o] = vr[o] - acc;
+    }
+}
+
+// -------------------------------------------------------------- accum ----
+constexpr int kCRows = 8;
+
+__global__ void __launch_bounds__(128) accum_simt_kernel(const float* __restrict__ kp,
+                                                         const float* __restrict__ r,
+                                                         const float* __restrict__ alpha,
+                                                         const float* __restrict__ beta,
+                                                         float* __restrict__ S, Dims dm) {
+    const int d = dm.d;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int c0 = blockIdx.x * kCRows;
+    const int n = threadIdx.x;
+    if (n >= d) return;
+    float acc[kCRows];
+#pragma unroll
+    for (int i = 0; i < kCRows; ++i) acc[i] = 0.f;
+    const float* bt = beta + ((size_t)b * dm.H + h) * dm.L;
+    for (int t = 0; t < dm.L; ++t) {
+        const float rb = bt[t] * r[tok(b, t, h, n, dm)];
+        const float* krow = kp + tok(b, t, h, 0, dm);
+#pragma unroll
+        for (int i = 0; i < kCRows; ++i)
+            if (c0 + i < d) acc[i] = fmaf(krow[c0 + i], rb, acc[i]);
+    }
+    const float a = alpha[(size_t)b * dm.H + h];
+    float* Sbh = S + ((size_t)b * dm.H + h) * d * d;
+#pragma unroll
+    for (int i = 0; i < kCRows; ++i) {
+        const int c = c0 + i;
+        if (c < d) Sbh[c * d + n] = fmaf(a, Sbh[c * d + n], acc[i]);
+    }
+}
+
+// --------------------------------------------------------------- fold ----
+__global__ void __launch_bounds__(128) fold_state_kernel(const __nv_bfloat16* __restrict__ wq,
+                                                         const float* __restrict__ S,
+                                                         __nv_bfloat16* __restrict__ Mt,
+                                                         __nv_bfloat16* __restrict__ St, Dims dm) {
+    const int d = dm.d;
+    const int a = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int n = threadIdx.x;
+    if (n >= d) return;
+    const size_t base = ((size_t)b * dm.H + h) * d * d;
+    const __nv_bfloat16* W = wq + (size_t)h * d * d;
+    float acc = 0.f;
+    for (int c = 0; c < d; ++c) acc = fmaf(__bfloat162float(W[a * d + c]), S[base + c * d + n], acc);
+    Mt[base + (size_t)n * d + a] = __float2bfloat16_rn(acc);
+    St[base + (size_t)n * d + a] = __float2bfloat16_rn(S[base + (size_t)a * d + n]);
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+// Dynamic shared memory of each kernel at the largest head_dim (128).
+constexpr size_t kPhiSmemMax = sizeof(float) * (128 * 128 + 2 * kPhiRows * 128);
+constexpr size_t kAttnSmemMax =
+    sizeof(float) * (kAQ * 128 + kAK * 129 + kAK * 128 + kAQ * (kAK + 1) + 128 * 128);
+constexpr size_t kResidualSmemMax = sizeof(float) * (128 * 128 + kRRows * 128);
+
+}  // namespace
+
+cudaError_t simt_init() {
+    cudaError_t e;
+    if ((e = set_smem(phi_simt_kernel<float>, kPhiSmemMax)) != cudaSuccess) return e;
+    if ((e = set_smem(phi_simt_kernel<__nv_bfloat16>, kPhiSmemMax)) != cudaSuccess) return e;
+    if ((e = set_smem(attn_simt_kernel<float>, kAttnSmemMax)) != cudaSuccess) return e;
+    if ((e = set_smem(attn_simt_kernel<__nv_bfloat16>, kAttnSmemMax)) != cudaSuccess) return e;
+    return set_smem(residual_simt_kernel, kResidualSmemMax);
+}
+
+cudaError_t launch_phi_simt(bool bf16, const void* x, const void* w, bool l2norm, float* out_f,
+                            void* out_t, Dims dm, cudaStream_t st) {
+    const size_t smem = sizeof(float) * ((size_t)dm.d * dm.d + 2 * kPhiRows * dm.d);
+    const dim3 grid((dm.L + kPhiRows - 1) / kPhiRows, dm.H, dm.B);
+    if (bf16) {
+        phi_simt_kernel<__nv_bfloat16><<<grid, 128, smem, st>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)w, l2norm,
+                                     out_f, (__nv_bfloat16*)out_t, dm);
+    } else {
+        phi_simt_kernel<float><<<grid, 128, smem, st>>>((const float*)x, (const float*)w, l2norm, out_f,
+                                     (float*)out_t, dm);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attn_simt(bool bf16, const void* q, const void* k, const void* v,
+                             const float* qp, const float* S, void* out, float scale, Dims dm,
+                             cudaStream_t st) {
+    const int d = dm.d;
+    const size_t smem = sizeof(float) * ((size_t)kAQ * d + (size_t)kAK * (d + 1) +
+                                         (size_t)kAK * d + (size_t)kAQ * (kAK + 1) + (size_t)d * d);
+    const dim3 grid((dm.L + kAQ - 1) / kAQ, dm.H, dm.B);
+    const float scale_log2 = scale * 1.4426950408889634f;
+    if (bf16) {
+        attn_simt_kernel<__nv_bfloat16><<<grid, kAThreads, smem, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                           (const __nv_bfloat16*)v, qp, S, (__nv_bfloat16*)out,
+                                           scale_log2, dm);
+    } else {
+        attn_simt_kernel<float><<<grid, kAThreads, smem, st>>>((const float*)q, (const float*)k, (const float*)v, qp, S,
+                                           (float*)out, scale_log2, dm);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_residual_simt(const float* kp, float* vp_to_r, const float* S, Dims dm,
+                                 cudaStream_t st) {
+    const size_t smem = sizeof(float) * ((size_t)dm.d * dm.d + (size_t)kRRows * dm.d);
+    const dim3 grid((dm.L + kRRows - 1) / kRRows, dm.H, dm.B);
+    residual_simt_kernel<<<grid, 128, smem, st>>>(kp, vp_to_r, S, dm);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_accum_simt(const float* kp, const float* r, const float* alpha,
+                              const float* beta, float* S, Dims dm, cudaStream_t st) {
+    const dim3 grid((dm.d + kCRows - 1) / kCRows, dm.H, dm.B);
+    accum_simt_kernel<<<grid, 128, 0, st>>>(kp, r, alpha, beta, S, dm);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fold_state(const void* wq_bf16, const float* S, void* Mt, void* St, Dims dm,
+                              cudaStream_t st) {
+    const dim3 grid(dm.d, dm.H, dm.B);
+    fold_state_kernel<<<grid, 128, 0, st>>>((const __nv_bfloat16*)wq_bf16, S,
+                                            (__nv_bfloat16*)Mt, (__nv_bfloat16*)St, dm);
+    return cudaGetLastError();
+}
+
+}  // namespace arl2

@@ -1,0 +1,154 @@
+/*
+ * arl2.h — C ABI of the ARL2 hybrid attention layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer ("Attend Locally, Remember Linearly", technical summary §2.1
+ * Hybrid Attention Decomposition and §2.2 Memory State Management) runs once
+ * per latent frame and denoising pass.  For every stream b and head h:
+ *
+ *   O = softmax(Q K^T * scale) V  +  (Q W_q[h]) S_{N-1}[b,h]
+ *
+ * the first term being the intra-frame bidirectional softmax branch over the
+ * frame's L tokens (§2.1 item 1) and the second the inter-frame read of the
+ * fixed-size state through the per-head feature map phi_q (§2.1 "Adaptation",
+ * "Output"), every token reading the same pre-update state (§2.2 "Frame-Level
+ * Access").  On the clean pass only (§2.2 "Clean-Pass Updates"), after the
+ * read, the state is updated once for the frame (§2.1 "State Update"):
+ *
+ *   K' = rownorm(K W_k[h]),  V' = V W_v[h]
+ *   S_N = alpha S_{N-1} + K'^T diag(beta) (V' - K' S_{N-1})
+ *
+ * Conventions used by every entry point:
+ *   - Token tensors (q, k, v, out, x) are [B][L][H][d], dense, in the
+ *     handle's dtype, device memory, 16-byte aligned.
+ *   - Feature maps W are [H][d][d] with row = input feature (x' = x W).
+ *   - The state S is fp32 [B][H][d][d], row = key feature, column = value
+ *     feature.  It is owned by the handle.
+ *   - alpha is fp32 [B][H] (one forget gate per stream and head for the
+ *     frame), beta is fp32 [B][H][L] (one rate per token).
+ *   - Every call is asynchronous and stream-ordered on the given stream: it
+ *     makes no host synchronisation and allocates nothing after
+ *     arl2_create.  A call that returns anything but ARL2_OK enqueued
+ *     nothing, except ARL2_ERR_CUDA, which reports a failed launch or copy.
+ *   - The caller keeps ownership of every pointer it passes; the handle owns
+ *     the state, its derived copies, the weight copies and all workspaces.
+ *   - The caller's current CUDA device must be the handle's device.
+ *   - A handle is not thread-safe: calls on one handle must be serialised
+ *     by the caller, and calls enqueued on different streams must not
+ *     overlap on the GPU.
+ */
+#ifndef ARL2_H
+#define ARL2_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ARL2_OK = 0,
+    ARL2_ERR_INVALID_ARG = -1,  /* null pointer, bad flag, wrong device     */
+    ARL2_ERR_SHAPE = -2,        /* a dimension out of the supported range   */
+    ARL2_ERR_ALIGN = -3,        /* a tensor pointer not 16-byte aligned     */
+    ARL2_ERR_CUDA = -4,         /* a CUDA runtime or driver call failed     */
+    ARL2_ERR_OOM = -5,          /* device allocation failed in arl2_create  */
+    ARL2_ERR_TIMEOUT = -6,      /* a kernel's bounded wait ran out          */
+    ARL2_ERR_UNSUPPORTED = -7   /* valid, but not built for this dtype/size */
+} arl2_status;
+
+typedef enum { ARL2_BF16 = 0, ARL2_FP32 = 1 } arl2_dtype;
+
+/* Kernel family.  AUTO picks the tensor-core (tcgen05) kernels for bf16 with
+ * head_dim 128 and the fp32 SIMT kernels for fp32.  SIMT forces the SIMT
+ * kernels (fp32 arithmetic) for either dtype; it exists to cross-check the
+ * tensor-core kernels on the GPU and is not a fallback: AUTO never falls
+ * back to it. */
+typedef enum { ARL2_IMPL_AUTO = 0, ARL2_IMPL_SIMT = 1 } arl2_impl;
+
+typedef struct arl2_handle arl2_handle;
+
+typedef struct {
+    int batch;             /* B >= 1: independent streams                     */
+    int heads;             /* H >= 1                                          */
+    int head_dim;          /* d: 128 for bf16 tensor-core kernels; 1..128 SIMT */
+    int tokens_per_frame;  /* L >= 1                                          */
+    arl2_dtype dtype;      /* dtype of q, k, v, out and the feature maps      */
+    const void* w_q;       /* device [H][d][d], dtype; copied at create       */
+    const void* w_k;
+    const void* w_v;
+    float softmax_scale;   /* 0 selects 1/sqrt(d)                             */
+    int host_staging;      /* nonzero: allocate device staging buffers so that
+                              arl2_frame_forward_host can be used             */
+    arl2_impl impl;
+} arl2_config;
+
+/* Create a layer on the current device.  Validates cfg, allocates the zeroed
+ * state S_0 = 0 and every workspace, and copies the three feature maps
+ * (stream-ordered on `stream`).  On success *out receives the handle.
+ * Errors: INVALID_ARG (null cfg/out/weights), SHAPE, ALIGN (weights),
+ * UNSUPPORTED (dtype/head_dim the chosen kernels do not handle), OOM, CUDA. */
+arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle** out);
+
+/* One denoising pass of one latent frame (technical summary §2.1, §2.2).
+ * Writes out = O_intra + O_inter for every token, reading S_{N-1}.  When
+ * clean_pass is nonzero, then also updates the state in place to S_N; alpha
+ * and beta are read only in that case and may be NULL otherwise.
+ * q, k, v, out: device [B][L][H][d] dtype, 16-byte aligned; out must not
+ * alias q, k or v.  alpha: device fp32 [B][H]; beta: device fp32 [B][H][L]. */
+arl2_status arl2_frame_forward(arl2_handle* h, const void* q, const void* k, const void* v,
+                               const float* alpha, const float* beta, int clean_pass,
+                               void* out, cudaStream_t stream);
+
+/* arl2_frame_forward on HOST buffers: copies q, k, v (and alpha, beta on a
+ * clean pass) from host memory into the handle's device staging buffers,
+ * runs the pass, and copies out back to host memory, all stream-ordered on
+ * `stream`.  Host buffers should be pinned for the copies to be
+ * asynchronous; the caller must not touch them until the stream reaches
+ * this point.  Needs a handle created with host_staging != 0
+ * (INVALID_ARG otherwise). */
+arl2_status arl2_frame_forward_host(arl2_handle* h, const void* q, const void* k, const void* v,
+                                    const float* alpha, const float* beta, int clean_pass,
+                                    void* out, cudaStream_t stream);
+
+/* S := 0 for every stream and head (the start of a new video stream). */
+arl2_status arl2_state_reset(arl2_handle* h, cudaStream_t stream);
+
+/* Copy the fp32 state [B][H][d][d] to device memory dst (checkpoint, parity). */
+arl2_status arl2_state_get(arl2_handle* h, float* dst_device, cudaStream_t stream);
+
+/* Replace the state by the fp32 [B][H][d][d] device buffer src (resume). */
+arl2_status arl2_state_set(arl2_handle* h, const float* src_device, cudaStream_t stream);
+
+/* Apply one of the handle's per-head feature maps to a token tensor:
+ * which = 0: out = x W_q;  1: out = rownorm(x W_k);  2: out = x W_v
+ * (technical summary §2.1 "Adaptation").  x, out: device [B][L][H][d] in
+ * the handle's dtype.  This is the stand-alone form of the projection the
+ * forward pass fuses; it exists for step-level checks. */
+arl2_status arl2_phi_apply(arl2_handle* h, int which, const void* x, void* out,
+                           cudaStream_t stream);
+
+/* Synchronise `stream`, then read and clear the handle's device error word.
+ * Returns ARL2_ERR_TIMEOUT if a kernel gave up a bounded wait since the last
+ * check (its outputs are then undefined), ARL2_ERR_CUDA on a CUDA error,
+ * else ARL2_OK.  This is the one call that blocks the host. */
+arl2_status arl2_device_status(arl2_handle* h, cudaStream_t stream);
+
+/* Device bytes the handle holds (state, copies, weights, workspaces). */
+size_t arl2_device_bytes(const arl2_handle* h);
+
+/* Release everything the handle owns.  Synchronises the device first.
+ * NULL is ignored. */
+void arl2_destroy(arl2_handle* h);
+
+/* Static string for a status code. */
+const char* arl2_status_string(arl2_status s);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int arl2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ARL2_H */

@@ -1,0 +1,80 @@
+"""The C-ABI library loads and exports every entry point include/arl2.h declares.
+
+CPU only: no call here reaches the GPU (argument checks return before any
+CUDA call).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import hybrid_softmax_gated_b200 as arl2
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "arl2.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(arl2_[a-z_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary_calls():
+    names = declared_functions()
+    for required in ("arl2_create", "arl2_frame_forward", "arl2_state_reset", "arl2_state_get",
+                     "arl2_state_set", "arl2_destroy", "arl2_status_string"):
+        assert required in names
+
+
+@pytest.mark.parametrize("name", declared_functions())
+def test_library_exports_declared_symbol(name):
+    lib = ctypes.CDLL(arl2.library_path())
+    assert hasattr(lib, name), name
+
+
+def test_binding_covers_every_export():
+    assert sorted(arl2.EXPORTED) == declared_functions()
+
+
+def test_version_and_status_strings():
+    assert arl2.version() == 10000
+    for code in range(0, -8, -1):
+        s = arl2._lib.arl2_status_string(code).decode()
+        assert s and s != "unknown status"
+    assert arl2._lib.arl2_status_string(-99).decode() == "unknown status"
+
+
+def test_null_arguments_are_rejected_before_any_cuda_call():
+    lib = arl2._lib
+    h = ctypes.c_void_p()
+    assert lib.arl2_create(None, None, ctypes.byref(h)) == -1
+    cfg = arl2.Arl2Config(1, 1, 16, 16, 1, None, None, None, 0.0, 0, 0)
+    assert lib.arl2_create(ctypes.byref(cfg), None, None) == -1
+    assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1  # null weights
+    assert lib.arl2_frame_forward(None, None, None, None, None, None, 0, None, None) == -1
+    assert lib.arl2_state_reset(None, None) == -1
+    assert lib.arl2_state_get(None, None, None) == -1
+    assert lib.arl2_state_set(None, None, None) == -1
+    assert lib.arl2_phi_apply(None, 0, None, None, None) == -1
+    assert lib.arl2_device_status(None, None) == -1
+    assert lib.arl2_device_bytes(None) == 0
+    lib.arl2_destroy(None)
+
+
+def test_shape_and_alignment_checks_come_before_cuda():
+    lib = arl2._lib
+    h = ctypes.c_void_p()
+    fake = 0x1000  # never dereferenced: validation fails first
+    for bad in [(0, 1, 16, 16), (1, 0, 16, 16), (1, 1, 0, 16), (1, 1, 129, 16), (1, 1, 16, 0)]:
+        cfg = arl2.Arl2Config(*bad, 1, fake, fake, fake, 0.0, 0, 0)
+        assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -2
+    cfg = arl2.Arl2Config(1, 1, 16, 16, 1, fake + 4, fake, fake, 0.0, 0, 0)
+    assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -3
+    cfg = arl2.Arl2Config(1, 1, 64, 16, 0, fake, fake, fake, 0.0, 0, 0)  # bf16 tensor cores need d=128
+    assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -7
+    cfg = arl2.Arl2Config(1, 1, 16, 16, 7, fake, fake, fake, 0.0, 0, 0)  # bad dtype
+    assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1
+    cfg = arl2.Arl2Config(1, 1, 16, 16, 1, fake, fake, fake, -1.0, 0, 0)  # bad scale
+    assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1

@@ -1,0 +1,121 @@
+"""Full-size workloads on the GPU, in the launch configuration the benchmark
+times, against the CPU oracle on sampled output rows and the full state.
+
+- 480p: 21 frames x 4 passes; every row of the first and the last clean
+  pass, 64 random rows of every other pass, the full state after each
+  frame.
+- 720p: 30 frames x 4 passes; every row of the first pass, 16 random rows
+  elsewhere, the full state after each frame.
+- long stream (240 frames): device memory and per-frame time stay flat,
+  the state stays finite and bounded, and the last frame matches the
+  oracle when the oracle starts from the GPU's own state.
+- 30-layer stack with 4 streams: layers 0 and 29 against the oracle for
+  the first frames; every layer's streams independent of each other.
+"""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from gpu_harness import TOL, err, make_layer, run_and_check
+
+pytestmark = pytest.mark.gpu
+
+W = workloads.WORKLOADS
+
+
+def test_480p_stream_sampled_parity():
+    w = W["480p_bf16"]
+    last = w.frames - 1
+    eo, es = run_and_check(
+        w, full_rows=lambda f, p: (f == 0 and p == 0) or (f == last and p == w.passes - 1),
+        sample_rows=64)
+    print(f"480p worst output err {eo:.3e}, worst state err {es:.3e}")
+
+
+def test_720p_stream_sampled_parity():
+    w = W["720p_bf16"]
+    eo, es = run_and_check(w, full_rows=lambda f, p: f == 0 and p == 0, sample_rows=16)
+    print(f"720p worst output err {eo:.3e}, worst state err {es:.3e}")
+
+
+def test_long_stream_memory_and_time_flat_and_last_frame_parity():
+    w = W["long_stream_bf16"]
+    lay, (wq, wk, wv) = make_layer(w)
+    try:
+        free0, _ = torch.cuda.mem_get_info()
+        alloc0 = torch.cuda.memory_allocated()
+        times, frees = [], []
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        last = w.frames - 1
+        for f in range(w.frames):
+            a, b = (t.cuda() for t in workloads.frame_gates(w, 0, f))
+            ins = [workloads.pass_inputs(w, 0, f, p, device="cuda") for p in range(w.passes)]
+            if f == last:
+                S_prev = lay.state_get().cpu().numpy()
+            start.record()
+            outs = []
+            for p in range(w.passes):
+                q, k, v = ins[p]
+                outs.append(lay.forward(q, k, v, a, b, clean_pass=workloads.is_clean(w, p)))
+            stop.record()
+            stop.synchronize()
+            times.append(start.elapsed_time(stop))
+            frees.append(torch.cuda.mem_get_info()[0])
+            if f == last:
+                S_gpu = lay.state_get().cpu().numpy()
+            del outs
+        assert lay.device_status() == 0
+        # memory: nothing grows with the frame index
+        assert max(frees) - min(frees) <= 64 << 20
+        assert torch.cuda.memory_allocated() - alloc0 <= 64 << 20
+        # time: the second half is not slower than the first
+        t = np.array(times[5:])
+        assert np.median(t[len(t) // 2:]) <= 1.25 * np.median(t[: len(t) // 2])
+        assert np.all(np.isfinite(S_gpu)) and np.max(np.abs(S_gpu)) < 10.0
+        # last frame: oracle from the GPU's own pre-frame state
+        q, k, v = (x.cpu() for x in ins[w.passes - 1])
+        a, b = workloads.frame_gates(w, 0, last)
+        rng = np.random.default_rng(7)
+        rt = rng.choice(w.tokens, size=64, replace=False)
+        rb = np.zeros_like(rt)
+        ref = oracle.rows(q, k, v, wq, S_prev, rb, rt)
+        # replay the last clean pass from the state the stream had before it
+        lay.state_set(torch.from_numpy(S_prev).cuda())
+        o = lay.forward(ins[-1][0], ins[-1][1], ins[-1][2], a.cuda(), b.cuda(), clean_pass=True)
+        assert err(o.float().cpu().numpy()[rb, rt], ref) <= TOL["bf16"]
+        S_ref = oracle.state_update(k, v, wk, wv, a, b, S_prev)
+        assert err(lay.state_get().cpu().numpy(), S_ref) <= TOL["bf16"]
+        print(f"long stream: median frame {np.median(t):.3f} ms, free-mem spread "
+              f"{(max(frees) - min(frees)) / 2**20:.1f} MiB")
+    finally:
+        lay.close()
+
+
+def test_stack30_layers_against_oracle_and_streams_independent():
+    w = W["stack30_bf16"]
+    for layer in (0, w.layers - 1):
+        run_and_check(w, layer=layer, frames=2, full_rows=lambda f, p: False, sample_rows=32)
+    # all 30 layers: 4-stream runs equal single-stream runs of the same inputs
+    import dataclasses
+    w1 = dataclasses.replace(w, batch=1)
+    for layer in range(w.layers):
+        lay4, _ = make_layer(w, layer)
+        lay1, _ = make_layer(w1, layer)
+        try:
+            for f in range(2):
+                a, b = (t.cuda() for t in workloads.frame_gates(w, layer, f))
+                q, k, v = (t.cuda() for t in workloads.pass_inputs(w, layer, f, w.passes - 1))
+                o4 = lay4.forward(q, k, v, a, b, clean_pass=True)
+                s = 3
+                o1 = lay1.forward(q[s:s + 1].contiguous(), k[s:s + 1].contiguous(),
+                                  v[s:s + 1].contiguous(), a[s:s + 1].contiguous(),
+                                  b[s:s + 1].contiguous(), clean_pass=True)
+                assert torch.equal(o1[0], o4[s])
+            assert torch.equal(lay1.state_get()[0], lay4.state_get()[s])
+        finally:
+            lay4.close()
+            lay1.close()

@@ -84,8 +84,8 @@ def stream_base(layer: int, stream: int) -> int:
 _TAG_QKV, _TAG_GATES, _TAG_W = 1, 2, 3
 
 
-def _gen(*parts: int) -> torch.Generator:
-    return torch.Generator().manual_seed(subseed(*parts))
+def _gen(*parts: int, device: str = "cpu") -> torch.Generator:
+    return torch.Generator(device=device).manual_seed(subseed(*parts))
 
 
 def phi_weights(w: Workload, layer: int = 0):
@@ -104,17 +104,21 @@ def phi_weights(w: Workload, layer: int = 0):
     return tuple(out)
 
 
-def pass_inputs(w: Workload, layer: int, frame: int, pass_idx: int):
-    """q, k, v for one (frame, pass): [B, L, H, d] each, in w's dtype."""
+def pass_inputs(w: Workload, layer: int, frame: int, pass_idx: int, device: str = "cpu"):
+    """q, k, v for one (frame, pass): [B, L, H, d] each, in w's dtype.
+
+    device="cuda" draws with the device generator (same seeds and
+    distribution, different random stream; much faster for long streams).
+    """
     B, L, H, d = w.batch, w.tokens, w.heads, w.head_dim
-    q = torch.empty(B, L, H, d, dtype=torch.float32)
+    q = torch.empty(B, L, H, d, dtype=torch.float32, device=device)
     k = torch.empty_like(q)
     v = torch.empty_like(q)
     for b in range(B):
-        g = _gen(stream_base(layer, b), _TAG_QKV, frame, pass_idx)
-        q[b] = torch.randn(L, H, d, generator=g)
-        k[b] = torch.randn(L, H, d, generator=g)
-        v[b] = torch.randn(L, H, d, generator=g)
+        g = _gen(stream_base(layer, b), _TAG_QKV, frame, pass_idx, device=device)
+        q[b] = torch.randn(L, H, d, generator=g, device=device)
+        k[b] = torch.randn(L, H, d, generator=g, device=device)
+        v[b] = torch.randn(L, H, d, generator=g, device=device)
     t = w.torch_dtype
     return q.to(t).contiguous(), k.to(t).contiguous(), v.to(t).contiguous()
 
