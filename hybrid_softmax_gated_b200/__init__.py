@@ -31,7 +31,8 @@ ARL2_IMPL_AUTO, ARL2_IMPL_SIMT = 0, 1
 EXPORTED = (
     "arl2_create", "arl2_frame_forward", "arl2_frame_forward_host", "arl2_state_reset",
     "arl2_state_get", "arl2_state_set", "arl2_phi_apply", "arl2_device_status",
-    "arl2_device_bytes", "arl2_destroy", "arl2_status_string", "arl2_version",
+    "arl2_device_bytes", "arl2_kernel_launches", "arl2_destroy", "arl2_status_string",
+    "arl2_version",
 )
 
 
@@ -47,7 +48,7 @@ class Arl2Config(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m hybrid_softmax_gated_b200.build`")
+                          "`python hybrid_softmax_gated_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     H = ctypes.c_void_p
@@ -61,6 +62,7 @@ def _load() -> ctypes.CDLL:
         "arl2_phi_apply": ([H, I, P, P, P], I),
         "arl2_device_status": ([H, P], I),
         "arl2_device_bytes": ([H], S),
+        "arl2_kernel_launches": ([H], ctypes.c_ulonglong),
         "arl2_destroy": ([H], None),
         "arl2_status_string": ([I], ctypes.c_char_p),
         "arl2_version": ([], I),
@@ -222,6 +224,10 @@ class Arl2Layer:
 
     def device_bytes(self) -> int:
         return int(_lib.arl2_device_bytes(self.handle))
+
+    def kernel_launches(self) -> int:
+        """Kernels this layer has enqueued (or recorded into a graph) so far."""
+        return int(_lib.arl2_kernel_launches(self.handle))
 
     def close(self) -> None:
         if getattr(self, "_h", None) is not None:

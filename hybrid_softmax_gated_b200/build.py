@@ -1,6 +1,9 @@
 """Build libarl2.so in place with nvcc for sm_100a.
 
-    python -m hybrid_softmax_gated_b200.build [--verbose-ptxas]
+    python hybrid_softmax_gated_b200/build.py [--verbose-ptxas]
+
+Run it by path: importing the package loads the library, which must not be
+needed to build it.
 
 The CUDA runtime is linked statically and the driver API is reached through
 cudaGetDriverEntryPoint, so the library loads on machines without a GPU

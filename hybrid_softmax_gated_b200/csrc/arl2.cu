@@ -41,6 +41,7 @@ struct arl2_handle {
     float* stage_beta = nullptr;
     int* err = nullptr;       // device error word
     arl2::AttnTc* tc = nullptr;
+    unsigned long long launches = 0;  // kernels enqueued by this handle
 };
 
 namespace {
@@ -84,6 +85,7 @@ void release(arl2_handle* h) {
 // Recompute the tensor-core copies of the state after it changed.
 arl2_status refresh_derived(arl2_handle* h, cudaStream_t st) {
     if (!h->use_tc) return ARL2_OK;
+    ++h->launches;
     if (arl2::launch_fold_state(h->w[0], h->S, h->Mt, h->St, h->dm, st) != cudaSuccess)
         return ARL2_ERR_CUDA;
     return ARL2_OK;
@@ -92,6 +94,7 @@ arl2_status refresh_derived(arl2_handle* h, cudaStream_t st) {
 arl2_status clean_update(arl2_handle* h, const void* k, const void* v, const float* alpha,
                          const float* beta, cudaStream_t st) {
     const bool bf16 = h->dtype == ARL2_BF16;
+    h->launches += 4;
     if (arl2::launch_phi_simt(bf16, k, h->w[1], true, h->kp, nullptr, h->dm, st) != cudaSuccess)
         return ARL2_ERR_CUDA;
     if (arl2::launch_phi_simt(bf16, v, h->w[2], false, h->vp, nullptr, h->dm, st) != cudaSuccess)
@@ -209,6 +212,7 @@ arl2_status arl2_frame_forward(arl2_handle* h, const void* q, const void* k, con
     arl2_status s = check_device(h);
     if (s != ARL2_OK) return s;
     const bool bf16 = h->dtype == ARL2_BF16;
+    h->launches += h->use_tc ? 1 : 2;
     if (h->use_tc) {
         if (arl2::attn_tc_launch(h->tc, q, k, v, h->Mt, out, h->scale, h->err, stream) != cudaSuccess)
             return ARL2_ERR_CUDA;
@@ -295,6 +299,7 @@ arl2_status arl2_phi_apply(arl2_handle* h, int which, const void* x, void* out,
     arl2_status s = check_device(h);
     if (s != ARL2_OK) return s;
     const bool bf16 = h->dtype == ARL2_BF16;
+    ++h->launches;
     if (arl2::launch_phi_simt(bf16, x, h->w[which], which == 1, nullptr, out, h->dm, stream) !=
         cudaSuccess)
         return ARL2_ERR_CUDA;
@@ -317,6 +322,8 @@ arl2_status arl2_device_status(arl2_handle* h, cudaStream_t stream) {
 }
 
 size_t arl2_device_bytes(const arl2_handle* h) { return h ? h->bytes : 0; }
+
+unsigned long long arl2_kernel_launches(const arl2_handle* h) { return h ? h->launches : 0; }
 
 void arl2_destroy(arl2_handle* h) {
     if (!h) return;

@@ -137,6 +137,10 @@ arl2_status arl2_device_status(arl2_handle* h, cudaStream_t stream);
 /* Device bytes the handle holds (state, copies, weights, workspaces). */
 size_t arl2_device_bytes(const arl2_handle* h);
 
+/* Number of kernels this handle has enqueued (or recorded into a CUDA graph
+ * capture) since creation; memsets and copies are not counted.  0 for NULL. */
+unsigned long long arl2_kernel_launches(const arl2_handle* h);
+
 /* Release everything the handle owns.  Synchronises the device first.
  * NULL is ignored. */
 void arl2_destroy(arl2_handle* h);
