@@ -31,9 +31,10 @@ ARL2_IMPL_AUTO, ARL2_IMPL_SIMT = 0, 1
 EXPORTED = (
     "arl2_create", "arl2_frame_forward", "arl2_frame_forward_host", "arl2_state_reset",
     "arl2_state_get", "arl2_state_set", "arl2_phi_apply", "arl2_device_status",
-    "arl2_device_bytes", "arl2_kernel_launches", "arl2_destroy", "arl2_status_string",
-    "arl2_version",
+    "arl2_device_bytes", "arl2_kernel_launches", "arl2_state_update_noalloc", "arl2_destroy",
+    "arl2_status_string", "arl2_version",
 )
+NOALLOC_MAX_ELEMENTS = 1 << 22
 
 
 class Arl2Config(ctypes.Structure):
@@ -63,6 +64,7 @@ def _load() -> ctypes.CDLL:
         "arl2_device_status": ([H, P], I),
         "arl2_device_bytes": ([H], S),
         "arl2_kernel_launches": ([H], ctypes.c_ulonglong),
+        "arl2_state_update_noalloc": ([I, I, I, I, I, P, P, P, P, P, P, P, P], I),
         "arl2_destroy": ([H], None),
         "arl2_status_string": ([I], ctypes.c_char_p),
         "arl2_version": ([], I),
@@ -96,6 +98,16 @@ def _stream(stream) -> int:
 
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def state_update_noalloc(k, v, w_k, w_v, alpha, beta, state, stream=None) -> None:
+    """arl2_state_update_noalloc: the clean-pass update in place on a
+    caller-owned fp32 state [B, H, d, d], allocating no device memory."""
+    B, L, H, d = k.shape
+    dt = ARL2_BF16 if k.dtype == torch.bfloat16 else ARL2_FP32
+    _check(_lib.arl2_state_update_noalloc(B, H, d, L, dt, _ptr(k), _ptr(v), _ptr(w_k), _ptr(w_v),
+                                          _ptr(alpha), _ptr(beta), _ptr(state), _stream(stream)),
+           "arl2_state_update_noalloc")
 
 
 def library_path() -> str:

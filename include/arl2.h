@@ -141,6 +141,40 @@ size_t arl2_device_bytes(const arl2_handle* h);
  * capture) since creation; memsets and copies are not counted.  0 for NULL. */
 unsigned long long arl2_kernel_launches(const arl2_handle* h);
 
+/* Largest batch * tokens * heads * head_dim that arl2_state_update_noalloc
+ * accepts: 4,194,304 elements (a 1560-token, 12-head, 128-wide frame of one
+ * stream is 2,396,160). */
+#define ARL2_NOALLOC_MAX_ELEMENTS (1u << 22)
+
+/* The clean-pass state update, for callers that cannot allocate device
+ * memory.  The ARL2 pages have no counterpart to this call: it exists for
+ * deployment.  Some callers cannot call cudaMalloc where they run this step
+ * (a plugin that only gets fixed buffers from its host framework, or a
+ * process whose caching allocator has already reserved the device memory),
+ * and arl2_create allocates.  This call allocates nothing: the caller owns
+ * the state, and the two fp32 scratch arrays the update needs live in a
+ * static device array inside the library (2 x ARL2_NOALLOC_MAX_ELEMENTS
+ * floats = 32 MiB, held on every GPU that loads the library until exit).
+ *
+ * Computes, in place on `state` (fp32 [B][H][d][d], row = key feature):
+ *   S = alpha S + K'^T diag(beta) (V' - K' S),  K' = rownorm(K W_k), V' = V W_v
+ * k, v: device [B][L][H][d] in dtype; w_k, w_v: device [H][d][d] in dtype;
+ * alpha: device fp32 [B][H]; beta: device fp32 [B][H][L].  All pointers
+ * 16-byte aligned.  Uses the fp32 SIMT kernels for either dtype.
+ *
+ * The first call on each device looks up the scratch array's device address
+ * (cudaGetSymbolAddress, with that device current) and sets kernel
+ * attributes; make that first call before any stream capture.  Every call
+ * shares the one scratch array and leaves its contents behind, so calls
+ * whose work overlaps on the GPU (other streams, other threads) race: keep
+ * them ordered.  Errors: INVALID_ARG (null pointer, bad dtype), SHAPE (a
+ * dimension out of range, or B*L*H*d > ARL2_NOALLOC_MAX_ELEMENTS), ALIGN,
+ * CUDA; nothing is enqueued on an error other than CUDA. */
+arl2_status arl2_state_update_noalloc(int batch, int heads, int head_dim, int tokens,
+                                      arl2_dtype dtype, const void* k, const void* v,
+                                      const void* w_k, const void* w_v, const float* alpha,
+                                      const float* beta, float* state, cudaStream_t stream);
+
 /* Release everything the handle owns.  Synchronises the device first.
  * NULL is ignored. */
 void arl2_destroy(arl2_handle* h);
