@@ -1,14 +1,24 @@
 // Host side of libarl2.so: the C ABI declared in include/arl2.h.
 //
-// The handle owns the fp32 state S[B][H][d][d], its bf16 derived copies
-// for the tensor-core kernels, copies of the three feature maps, and every
-// workspace.  All of it is allocated in arl2_create; no later call
-// allocates, which keeps device memory flat over arbitrarily long streams
-// (the constant-memory property the ARL2 pages claim for the fixed-size
-// state, technical summary §1 and §4 "Memory").
+// The handle owns the fp32 state S[B][H][d][d], its derived copies, one
+// copy of the three feature maps, and every workspace.  All of it is
+// allocated in arl2_create; no later call allocates, which keeps device
+// memory flat over arbitrarily long streams (the constant-memory property
+// the ARL2 pages claim for the fixed-size state, technical summary §1 and
+// §4 "Memory").
+//
+// Kernels per call (tensor-core path, bf16, head_dim 128):
+//   read-only pass : attn_tc_kernel                         (1 launch)
+//   clean pass     : attn_tc_kernel, update_chunk_kernel,
+//                    update_finalize_kernel, fold_state      (4 launches)
+// SIMT path (fp32, or impl = ARL2_IMPL_SIMT):
+//   read-only pass : phi (q'), attn_simt                     (2 launches)
+//   clean pass     : + phi (k'), phi (v'), residual, accum   (6 launches)
 #include "arl2.h"
 #include "internal.h"
 #include "attn_tc.h"
+#include "tma.h"
+#include "update_tc.h"
 
 #include <cmath>
 #include <cstdint>
@@ -29,18 +39,25 @@ struct arl2_handle {
     size_t n_tok = 0;         // B*L*H*d
     size_t n_state = 0;       // B*H*d*d
     size_t bytes = 0;         // device bytes held
-    void* w[3] = {nullptr, nullptr, nullptr};  // feature-map copies [H][d][d] dtype
+    void* w_all = nullptr;    // feature maps [3][H][d][d] in dtype: W_q, W_k, W_v
+    void* w[3] = {nullptr, nullptr, nullptr};
     float* S = nullptr;       // fp32 master state
-    void* Mt = nullptr;       // bf16 (W_q S)^T, tensor-core read
-    void* St = nullptr;       // bf16 S^T, tensor-core update
+    // tensor-core path (both copies are functions of S alone)
+    void* Mt = nullptr;       // bf16 (W_q S)^T, read by the attention kernel
+    void* Sb = nullptr;       // bf16 S, read by the update kernel
+    float* part_s = nullptr;  // fp32 update partials [B][H][chunks][d][d]
+    arl2::TokenMapCache* maps = nullptr;
+    arl2::AttnTc* tc = nullptr;
+    arl2::UpdateTc* up = nullptr;
+    // SIMT path
     float* qp = nullptr;      // fp32 workspaces [B][L][H][d]
     float* kp = nullptr;
     float* vp = nullptr;
+    // host staging
     void* stage_tok[4] = {nullptr, nullptr, nullptr, nullptr};  // q, k, v, out
     float* stage_alpha = nullptr;
     float* stage_beta = nullptr;
     int* err = nullptr;       // device error word
-    arl2::AttnTc* tc = nullptr;
     unsigned long long launches = 0;  // kernels enqueued by this handle
 };
 
@@ -74,43 +91,56 @@ arl2_status dalloc(arl2_handle* h, T** p, size_t bytes) {
 void release(arl2_handle* h) {
     if (!h) return;
     if (h->tc) arl2::attn_tc_destroy(h->tc);
-    void* ptrs[] = {h->w[0], h->w[1], h->w[2], h->S, h->Mt, h->St, h->qp, h->kp, h->vp,
-                    h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], h->stage_tok[3],
+    if (h->up) arl2::update_tc_destroy(h->up);
+    delete h->maps;
+    void* ptrs[] = {h->w_all, h->S, h->Mt, h->Sb, h->part_s, h->qp, h->kp,
+                    h->vp, h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], h->stage_tok[3],
                     h->stage_alpha, h->stage_beta, h->err};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     delete h;
 }
 
-// Recompute the tensor-core copies of the state after it changed.
+arl2_status zero_state(arl2_handle* h, cudaStream_t st) {
+    if (cudaMemsetAsync(h->S, 0, h->n_state * sizeof(float), st) != cudaSuccess) return ARL2_ERR_CUDA;
+    if (h->use_tc && (cudaMemsetAsync(h->Mt, 0, h->n_state * 2, st) != cudaSuccess ||
+                      cudaMemsetAsync(h->Sb, 0, h->n_state * 2, st) != cudaSuccess))
+        return ARL2_ERR_CUDA;
+    return ARL2_OK;
+}
+
+// Recompute the tensor-core copies of the state after arl2_state_set.
 arl2_status refresh_derived(arl2_handle* h, cudaStream_t st) {
     if (!h->use_tc) return ARL2_OK;
     ++h->launches;
-    if (arl2::launch_fold_state(h->w[0], h->S, h->Mt, h->St, h->dm, st) != cudaSuccess)
+    if (arl2::launch_fold_state(h->w[0], h->S, h->Mt, h->Sb, h->dm, st) != cudaSuccess)
         return ARL2_ERR_CUDA;
     return ARL2_OK;
 }
 
 arl2_status clean_update(arl2_handle* h, const void* k, const void* v, const float* alpha,
                          const float* beta, cudaStream_t st) {
+    if (h->use_tc) {
+        h->launches += 3;
+        return arl2::update_tc_launch(h->up, *h->maps, k, v, alpha, beta, h->err, st) == cudaSuccess
+                   ? ARL2_OK
+                   : ARL2_ERR_CUDA;
+    }
     const bool bf16 = h->dtype == ARL2_BF16;
     h->launches += 4;
-    if (arl2::launch_phi_simt(bf16, k, h->w[1], true, h->kp, nullptr, h->dm, st) != cudaSuccess)
+    if (arl2::launch_phi_simt(bf16, k, h->w[1], true, h->kp, nullptr, h->dm, st) != cudaSuccess ||
+        arl2::launch_phi_simt(bf16, v, h->w[2], false, h->vp, nullptr, h->dm, st) != cudaSuccess ||
+        arl2::launch_residual_simt(h->kp, h->vp, h->S, h->dm, st) != cudaSuccess ||
+        arl2::launch_accum_simt(h->kp, h->vp, alpha, beta, h->S, h->dm, st) != cudaSuccess)
         return ARL2_ERR_CUDA;
-    if (arl2::launch_phi_simt(bf16, v, h->w[2], false, h->vp, nullptr, h->dm, st) != cudaSuccess)
-        return ARL2_ERR_CUDA;
-    if (arl2::launch_residual_simt(h->kp, h->vp, h->S, h->dm, st) != cudaSuccess)
-        return ARL2_ERR_CUDA;
-    if (arl2::launch_accum_simt(h->kp, h->vp, alpha, beta, h->S, h->dm, st) != cudaSuccess)
-        return ARL2_ERR_CUDA;
-    return refresh_derived(h, st);
+    return ARL2_OK;
 }
 
 }  // namespace
 
 extern "C" {
 
-int arl2_version(void) { return 10000; }
+int arl2_version(void) { return 10100; }
 
 const char* arl2_status_string(arl2_status s) {
     switch (s) {
@@ -158,15 +188,22 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
     h->n_state = (size_t)dm.B * dm.H * dm.d * dm.d;
     const size_t wbytes = (size_t)dm.H * dm.d * dm.d * h->esz;
 
-    arl2_status s = ARL2_OK;
-    for (int i = 0; i < 3 && s == ARL2_OK; ++i) s = dalloc(h, &h->w[i], wbytes);
-    if (s == ARL2_OK) s = dalloc(h, &h->S, h->n_state * sizeof(float));
-    if (s == ARL2_OK && use_tc) s = dalloc(h, &h->Mt, h->n_state * 2);
-    if (s == ARL2_OK && use_tc) s = dalloc(h, &h->St, h->n_state * 2);
-    if (s == ARL2_OK && !use_tc) s = dalloc(h, &h->qp, h->n_tok * sizeof(float));
-    if (s == ARL2_OK) s = dalloc(h, &h->kp, h->n_tok * sizeof(float));
-    if (s == ARL2_OK) s = dalloc(h, &h->vp, h->n_tok * sizeof(float));
+    arl2_status s = dalloc(h, &h->w_all, 3 * wbytes);
+    if (s == ARL2_OK) {
+        for (int i = 0; i < 3; ++i) h->w[i] = static_cast<char*>(h->w_all) + i * wbytes;
+        s = dalloc(h, &h->S, h->n_state * sizeof(float));
+    }
     if (s == ARL2_OK) s = dalloc(h, &h->err, sizeof(int));
+    if (use_tc) {
+        const size_t parts = (size_t)dm.B * dm.H * arl2::update_tc_chunks(dm) * dm.d * dm.d;
+        if (s == ARL2_OK) s = dalloc(h, &h->Mt, h->n_state * 2);
+        if (s == ARL2_OK) s = dalloc(h, &h->Sb, h->n_state * 2);
+        if (s == ARL2_OK) s = dalloc(h, &h->part_s, parts * sizeof(float));
+    } else {
+        if (s == ARL2_OK) s = dalloc(h, &h->qp, h->n_tok * sizeof(float));
+        if (s == ARL2_OK) s = dalloc(h, &h->kp, h->n_tok * sizeof(float));
+        if (s == ARL2_OK) s = dalloc(h, &h->vp, h->n_tok * sizeof(float));
+    }
     if (s == ARL2_OK && cfg->host_staging) {
         for (int i = 0; i < 4 && s == ARL2_OK; ++i) s = dalloc(h, &h->stage_tok[i], h->n_tok * h->esz);
         if (s == ARL2_OK) s = dalloc(h, &h->stage_alpha, (size_t)dm.B * dm.H * sizeof(float));
@@ -174,8 +211,11 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
     }
     if (s == ARL2_OK && arl2::simt_init() != cudaSuccess) s = ARL2_ERR_CUDA;
     if (s == ARL2_OK && use_tc) {
+        h->maps = new (std::nothrow) arl2::TokenMapCache(dm);
         h->tc = arl2::attn_tc_create(dm);
-        if (!h->tc) s = ARL2_ERR_CUDA;
+        const arl2::UpdateBuffers ub{h->w_all, h->S, h->Sb, h->Mt, h->part_s};
+        h->up = arl2::update_tc_create(dm, ub);
+        if (!h->maps || !h->maps->ok() || !h->tc || !h->up) s = ARL2_ERR_CUDA;
     }
     if (s != ARL2_OK) {
         release(h);
@@ -185,12 +225,7 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
     for (int i = 0; i < 3; ++i)
         if (cudaMemcpyAsync(h->w[i], src[i], wbytes, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
             s = ARL2_ERR_CUDA;
-    if (s == ARL2_OK && cudaMemsetAsync(h->S, 0, h->n_state * sizeof(float), stream) != cudaSuccess)
-        s = ARL2_ERR_CUDA;
-    if (s == ARL2_OK && use_tc &&
-        (cudaMemsetAsync(h->Mt, 0, h->n_state * 2, stream) != cudaSuccess ||
-         cudaMemsetAsync(h->St, 0, h->n_state * 2, stream) != cudaSuccess))
-        s = ARL2_ERR_CUDA;
+    if (s == ARL2_OK) s = zero_state(h, stream);
     if (s == ARL2_OK && cudaMemsetAsync(h->err, 0, sizeof(int), stream) != cudaSuccess)
         s = ARL2_ERR_CUDA;
     if (s != ARL2_OK) {
@@ -212,15 +247,16 @@ arl2_status arl2_frame_forward(arl2_handle* h, const void* q, const void* k, con
     arl2_status s = check_device(h);
     if (s != ARL2_OK) return s;
     const bool bf16 = h->dtype == ARL2_BF16;
-    h->launches += h->use_tc ? 1 : 2;
     if (h->use_tc) {
-        if (arl2::attn_tc_launch(h->tc, q, k, v, h->Mt, out, h->scale, h->err, stream) != cudaSuccess)
+        ++h->launches;
+        if (arl2::attn_tc_launch(h->tc, *h->maps, q, k, v, h->Mt, out, h->scale, h->err, stream) !=
+            cudaSuccess)
             return ARL2_ERR_CUDA;
     } else {
-        if (arl2::launch_phi_simt(bf16, q, h->w[0], false, h->qp, nullptr, h->dm, stream) != cudaSuccess)
-            return ARL2_ERR_CUDA;
-        if (arl2::launch_attn_simt(bf16, q, k, v, h->qp, h->S, out, h->scale, h->dm, stream) !=
-            cudaSuccess)
+        h->launches += 2;
+        if (arl2::launch_phi_simt(bf16, q, h->w[0], false, h->qp, nullptr, h->dm, stream) != cudaSuccess ||
+            arl2::launch_attn_simt(bf16, q, k, v, h->qp, h->S, out, h->scale, h->dm, stream) !=
+                cudaSuccess)
             return ARL2_ERR_CUDA;
     }
     if (clean_pass) return clean_update(h, k, v, alpha, beta, stream);
@@ -264,12 +300,7 @@ arl2_status arl2_state_reset(arl2_handle* h, cudaStream_t stream) {
     if (!h) return ARL2_ERR_INVALID_ARG;
     arl2_status s = check_device(h);
     if (s != ARL2_OK) return s;
-    if (cudaMemsetAsync(h->S, 0, h->n_state * sizeof(float), stream) != cudaSuccess)
-        return ARL2_ERR_CUDA;
-    if (h->use_tc && (cudaMemsetAsync(h->Mt, 0, h->n_state * 2, stream) != cudaSuccess ||
-                      cudaMemsetAsync(h->St, 0, h->n_state * 2, stream) != cudaSuccess))
-        return ARL2_ERR_CUDA;
-    return ARL2_OK;
+    return zero_state(h, stream);
 }
 
 arl2_status arl2_state_get(arl2_handle* h, float* dst, cudaStream_t stream) {

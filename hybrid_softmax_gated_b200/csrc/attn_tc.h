@@ -4,19 +4,21 @@
 #pragma once
 
 #include "internal.h"
+#include "tma.h"
 
 namespace arl2 {
 
 struct AttnTc;
 
-// Resolve the driver's tensor-map encoder and configure the kernel for the
-// given dimensions.  Returns nullptr on failure (no driver, bad dims).
+// Configure the kernel for the given dimensions.  Returns nullptr on
+// failure (no tensor-map encoder, bad dims).
 AttnTc* attn_tc_create(Dims dm);
 void attn_tc_destroy(AttnTc* t);
 
 // q, k, v, out: [B][L][H][128] bf16.  Mt: [B][H][128][128] bf16 holding
 // (W_q S)^T.  err: device error word (bit kErrTimeoutAttn on a timeout).
-cudaError_t attn_tc_launch(AttnTc* t, const void* q, const void* k, const void* v,
-                           const void* Mt, void* out, float scale, int* err, cudaStream_t st);
+cudaError_t attn_tc_launch(AttnTc* t, TokenMapCache& maps, const void* q, const void* k,
+                           const void* v, const void* Mt, void* out, float scale, int* err,
+                           cudaStream_t st);
 
 }  // namespace arl2

@@ -45,10 +45,10 @@ cudaError_t launch_residual_simt(const float* kp, float* vp_to_r, const float* S
 cudaError_t launch_accum_simt(const float* kp, const float* r, const float* alpha,
                               const float* beta, float* S, Dims dm, cudaStream_t st);
 
-// Derived bf16 copies of the state used by the tensor-core kernels:
-// Mt[b][h][n][a] = sum_c Wq[h][a][c] S[b][h][c][n]   ((W_q S)^T)
-// St[b][h][n][c] = S[b][h][c][n]                      (S^T)
-cudaError_t launch_fold_state(const void* wq_bf16, const float* S, void* Mt, void* St, Dims dm,
+// Copies of the state derived from S alone, used by the tensor-core kernels:
+// Mt[b][h][n][a] = bf16(sum_c Wq[h][a][c] S[b][h][c][n])   ((W_q S)^T)
+// Sb[b][h][c][n] = bf16(S[b][h][c][n])
+cudaError_t launch_fold_state(const void* wq_bf16, const float* S, void* Mt, void* Sb, Dims dm,
                               cudaStream_t st);
 
 }  // namespace arl2

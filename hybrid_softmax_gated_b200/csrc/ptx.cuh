@@ -203,5 +203,43 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
            | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
 
+// Operand tiles of 128 rows x 128 bf16, stored as two 128-row x 64-column
+// halves of 16 KB with the 128-byte swizzle (the layout TMA writes for a
+// {64, ..., 128} box).
+constexpr uint32_t kTileBytes = 128 * 128 * 2;
+constexpr uint32_t kHalfBytes = kTileBytes / 2;
+
+// K-major operand (row = M or N index, 128 K values along the row): the
+// descriptor of k-step kk (16 K values) starts kk*32 bytes into its half.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
+    return sdesc_sw128(tile + (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32u, 16u,
+                       1024u);
+}
+// MN-major operand (row = K index, 128 M/N values along the row in two
+// 64-wide halves 16 KB apart): k-step kk starts 16 rows = 2048 bytes on.
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk) {
+    return sdesc_sw128(tile + (uint32_t)kk * 2048u, kHalfBytes, 1024u);
+}
+
+// Byte offset of the 16-byte chunk c16 (0..15 along a 128-element bf16
+// row) of row r inside such a tile.
+__device__ __forceinline__ uint32_t tile_chunk_offset(int r, int c16) {
+    return (uint32_t)(c16 >> 3) * kHalfBytes + (uint32_t)r * 128u +
+           (uint32_t)(((c16 & 7) ^ (r & 7)) << 4);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 }  // namespace ptx
 }  // namespace arl2

@@ -8,7 +8,7 @@
 //   attn     softmax(Q K^T s) V + (Q W_q) S_{N-1}          §2.1 items 1-2, Output
 //   residual r = v' - k' S_{N-1}                           §2.1 State Update
 //   accum    S = alpha S + k'^T diag(beta) r               §2.1 State Update
-//   fold     (W_q S)^T and S^T in bf16 for the tensor-core read and update
+//   fold     (W_q S)^T and S in bf16 for the tensor-core path
 #include "internal.h"
 
 #include <cmath>
@@ -242,20 +242,42 @@ __global__ void __launch_bounds__(128) accum_simt_kernel(const float* __restrict
 }
 
 // --------------------------------------------------------------- fold ----
+// Copies of the state derived from S alone, for the tensor-core path:
+//   Mt[b][h][n][a] = bf16(sum_c Wq[h][a][c] S[b][h][c][n])   ((W_q S)^T)
+//   Sb[b][h][c][n] = bf16(S[b][h][c][n])
+// One CTA: 16 rows a of W_q S (and rows c = a of Sb); thread n owns column n.
+constexpr int kFoldRows = 16;
+
 __global__ void __launch_bounds__(128) fold_state_kernel(const __nv_bfloat16* __restrict__ wq,
                                                          const float* __restrict__ S,
                                                          __nv_bfloat16* __restrict__ Mt,
-                                                         __nv_bfloat16* __restrict__ St, Dims dm) {
+                                                         __nv_bfloat16* __restrict__ Sb, Dims dm) {
+    __shared__ float Ws[kFoldRows][128];
     const int d = dm.d;
-    const int a = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int a0 = blockIdx.x * kFoldRows, h = blockIdx.y, b = blockIdx.z;
     const int n = threadIdx.x;
-    if (n >= d) return;
     const size_t base = ((size_t)b * dm.H + h) * d * d;
     const __nv_bfloat16* W = wq + (size_t)h * d * d;
-    float acc = 0.f;
-    for (int c = 0; c < d; ++c) acc = fmaf(__bfloat162float(W[a * d + c]), S[base + c * d + n], acc);
-    Mt[base + (size_t)n * d + a] = __float2bfloat16_rn(acc);
-    St[base + (size_t)n * d + a] = __float2bfloat16_rn(S[base + (size_t)a * d + n]);
+    for (int i = threadIdx.x; i < kFoldRows * d; i += blockDim.x) {
+        const int r = i / d, c = i - r * d;
+        Ws[r][c] = a0 + r < d ? __bfloat162float(W[(size_t)(a0 + r) * d + c]) : 0.f;
+    }
+    __syncthreads();
+    if (n >= d) return;
+    float acc[kFoldRows];
+#pragma unroll
+    for (int i = 0; i < kFoldRows; ++i) acc[i] = 0.f;
+    for (int c = 0; c < d; ++c) {
+        const float s = S[base + (size_t)c * d + n];
+#pragma unroll
+        for (int i = 0; i < kFoldRows; ++i) acc[i] = fmaf(Ws[i][c], s, acc[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < kFoldRows; ++i) {
+        if (a0 + i >= d) break;
+        Mt[base + (size_t)n * d + a0 + i] = __float2bfloat16_rn(acc[i]);
+        Sb[base + (size_t)(a0 + i) * d + n] = __float2bfloat16_rn(S[base + (size_t)(a0 + i) * d + n]);
+    }
 }
 
 template <typename K>
@@ -328,11 +350,11 @@ cudaError_t launch_accum_simt(const float* kp, const float* r, const float* alph
     return cudaGetLastError();
 }
 
-cudaError_t launch_fold_state(const void* wq_bf16, const float* S, void* Mt, void* St, Dims dm,
+cudaError_t launch_fold_state(const void* wq_bf16, const float* S, void* Mt, void* Sb, Dims dm,
                               cudaStream_t st) {
-    const dim3 grid(dm.d, dm.H, dm.B);
-    fold_state_kernel<<<grid, 128, 0, st>>>((const __nv_bfloat16*)wq_bf16, S,
-                                            (__nv_bfloat16*)Mt, (__nv_bfloat16*)St, dm);
+    const dim3 grid((dm.d + kFoldRows - 1) / kFoldRows, dm.H, dm.B);
+    fold_state_kernel<<<grid, 128, 0, st>>>((const __nv_bfloat16*)wq_bf16, S, (__nv_bfloat16*)Mt,
+                                            (__nv_bfloat16*)Sb, dm);
     return cudaGetLastError();
 }
 

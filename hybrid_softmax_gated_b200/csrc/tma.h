@@ -1,0 +1,44 @@
+// Host-side TMA tensor-map encoding shared by the tensor-core kernels.
+//
+// All operand tiles are 128 rows x 128 bf16, loaded as two boxes of
+// 128 rows x 64 columns (128 bytes, the 128-byte swizzle span).
+#pragma once
+
+#include <cuda.h>
+#include <cstdint>
+
+#include "internal.h"
+
+namespace arl2 {
+
+// Resolve cuTensorMapEncodeTiled through the runtime (no libcuda link).
+bool tma_available();
+
+// Token tensor [B][L][H][128] bf16: dims {128, H, L, B}; box {64, 1, 128, 1}.
+bool tma_encode_tokens(CUtensorMap* m, const void* p, const Dims& dm);
+
+// Square bf16 tiles [outer][128][128] (outer = H or B*H flattened, the
+// innermost dimension contiguous): dims {128, 128, outer}; box {64, 128, 1}.
+bool tma_encode_tiles(CUtensorMap* m, const void* p, int outer);
+
+// Direct-mapped cache of token-tensor maps keyed by pointer (one per
+// handle; its dimensions never change).
+class TokenMapCache {
+public:
+    explicit TokenMapCache(const Dims& dm);
+    ~TokenMapCache();
+    bool ok() const { return entries_ != nullptr; }
+    // Returns a copy of the map for p (false if encoding failed).
+    bool get(const void* p, CUtensorMap* out);
+
+private:
+    static constexpr int kSlots = 1024;
+    struct Entry {
+        const void* p;
+        CUtensorMap m;
+    };
+    Dims dm_;
+    Entry* entries_;
+};
+
+}  // namespace arl2

@@ -1,0 +1,329 @@
+// Clean-pass state update on sm_100a tensor cores.
+//
+// "Attend Locally, Remember Linearly", technical summary §2.1 "Adaptation"
+// (phi_k, phi_v) and "State Update", §2.2 "Frame-Level Access" (every token
+// of the frame is measured against the same pre-update state) and
+// "Clean-Pass Updates" (one state write per frame):
+//
+//   S_N = alpha S_{N-1} + K'^T diag(beta) (V' - K' S_{N-1}),
+//   K' = rownorm(K W_k),  V' = V W_v.
+//
+// The sum over the frame's tokens splits into 128-token chunks that are
+// independent given S_{N-1}.  update_chunk_kernel (one CTA per chunk, head
+// and stream) computes, on tcgen05 with fp32 accumulators in TMEM:
+//   Kp = K W_k, Vp = V W_v                     (bf16 x bf16)
+//   K' = Kp / max(|Kp|, 1e-6)  -> bf16 tile    (epilogue)
+//   KS = K' S_{N-1}                            (S_{N-1} as bf16)
+//   beta R = beta (Vp - KS)    -> bf16 tile    (epilogue)
+//   dS = K'^T (beta R)                         (the same K' tile read MN-major)
+// and writes dS as an fp32 partial.  update_finalize_kernel sums the
+// partials in chunk order (deterministic) and applies the forget gate,
+//   S_N = alpha S_{N-1} + sum dS,
+// and the fold kernel then derives from S_N alone the bf16 copy of S and
+// Mt = (W_q S_N)^T, the matrix the attention kernel reads (so that the
+// inter-frame read Q' S = Q (W_q S) needs no per-token phi_q product, and a
+// restored checkpoint reproduces Mt exactly).
+#include "update_tc.h"
+#include "ptx.cuh"
+
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <new>
+
+namespace arl2 {
+namespace {
+
+using ptx::kHalfBytes;
+using ptx::kTileBytes;
+using ptx::kmajor_desc;
+using ptx::mnmajor_desc;
+
+constexpr int kD = 128;
+constexpr int kChunk = 128;
+constexpr int kThreads = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColKp = 0, kColVp = 128, kColKS = 256, kColDS = 384;
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+
+struct __align__(1024) Smem {
+    uint8_t xk[kTileBytes];  // K chunk -> K' (bf16)
+    uint8_t xv[kTileBytes];  // V chunk -> beta R (bf16)
+    uint8_t wk[kTileBytes];  // W_k[h], rows = input feature
+    uint8_t wv[kTileBytes];  // W_v[h]
+    uint8_t sb[kTileBytes];  // S_{N-1} bf16, rows = key feature
+    uint64_t ld_k, ld_v, proj, kp_ready, ks, r_ready, ds;
+    uint32_t tmem_base;
+    int abort;
+};
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+
+__global__ void __launch_bounds__(kThreads, 1)
+    update_chunk_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sb,
+                        const float* __restrict__ beta, float* __restrict__ part_s, int L, int H,
+                        int* err) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                        ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int n_chunks = gridDim.x;
+    const int bh = b * H + h;
+    volatile int* abort = &sm.abort;
+    const int no_abort = 0;
+
+    if (threadIdx.x == 0) {
+        uint64_t* bars[] = {&sm.ld_k, &sm.ld_v, &sm.proj, &sm.ks, &sm.ds};
+        for (uint64_t* p : bars) ptx::mbar_init(ptx::smem_u32(p), 1);
+        ptx::mbar_init(ptx::smem_u32(&sm.kp_ready), 128);
+        ptx::mbar_init(ptx::smem_u32(&sm.r_ready), 128);
+        sm.abort = 0;
+        ptx::fence_mbar_init();
+        ptx::fence_proxy_async_smem();
+    }
+    if (warp == 2) {
+        ptx::tmem_alloc(ptx::smem_u32(&sm.tmem_base), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    auto fail = [&]() {
+        atomicOr(err, kErrTimeoutUpdate);
+        *abort = 1;
+    };
+    auto wait = [&](uint64_t* bar) {
+        return ptx::mbar_wait_bounded(ptx::smem_u32(bar), 0, abort, kWaitLimitNs);
+    };
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ TMA producer --
+        const int t0 = chunk * kChunk;
+        const uint32_t bk = ptx::smem_u32(&sm.ld_k), bv = ptx::smem_u32(&sm.ld_v);
+        ptx::mbar_arrive_expect_tx(bk, 2 * kTileBytes);
+        ptx::tma_load_4d(ptx::smem_u32(sm.xk), &tm_k, 0, h, t0, b, bk);
+        ptx::tma_load_4d(ptx::smem_u32(sm.xk) + kHalfBytes, &tm_k, 64, h, t0, b, bk);
+        ptx::tma_load_4d(ptx::smem_u32(sm.wk), &tm_w, 0, 0, H + h, 0, bk);
+        ptx::tma_load_4d(ptx::smem_u32(sm.wk) + kHalfBytes, &tm_w, 64, 0, H + h, 0, bk);
+        ptx::mbar_arrive_expect_tx(bv, 3 * kTileBytes);
+        ptx::tma_load_4d(ptx::smem_u32(sm.xv), &tm_v, 0, h, t0, b, bv);
+        ptx::tma_load_4d(ptx::smem_u32(sm.xv) + kHalfBytes, &tm_v, 64, h, t0, b, bv);
+        ptx::tma_load_4d(ptx::smem_u32(sm.wv), &tm_w, 0, 0, 2 * H + h, 0, bv);
+        ptx::tma_load_4d(ptx::smem_u32(sm.wv) + kHalfBytes, &tm_w, 64, 0, 2 * H + h, 0, bv);
+        ptx::tma_load_4d(ptx::smem_u32(sm.sb), &tm_sb, 0, 0, bh, 0, bv);
+        ptx::tma_load_4d(ptx::smem_u32(sm.sb) + kHalfBytes, &tm_sb, 64, 0, bh, 0, bv);
+        // The loads have landed before the CTA may exit.
+        ptx::mbar_wait_bounded(bk, 0, &no_abort, kWaitLimitNs);
+        ptx::mbar_wait_bounded(bv, 0, &no_abort, kWaitLimitNs);
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------- UMMA issuer --
+        constexpr uint32_t id_k_mn = ptx::idesc_bf16_f32(128, 128, false, true);
+        constexpr uint32_t id_mn_mn = ptx::idesc_bf16_f32(128, 128, true, true);
+        const uint32_t xk = ptx::smem_u32(sm.xk), xv = ptx::smem_u32(sm.xv);
+        const uint32_t wk = ptx::smem_u32(sm.wk), wv = ptx::smem_u32(sm.wv);
+        const uint32_t sb = ptx::smem_u32(sm.sb);
+        bool ok = wait(&sm.ld_k);
+        if (ok) {
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // Kp = K W_k
+                ptx::umma_f16_ss(tmem + kColKp, kmajor_desc(xk, kk), mnmajor_desc(wk, kk), id_k_mn, kk > 0);
+            ok = wait(&sm.ld_v);
+        }
+        if (ok) {
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // Vp = V W_v
+                ptx::umma_f16_ss(tmem + kColVp, kmajor_desc(xv, kk), mnmajor_desc(wv, kk), id_k_mn, kk > 0);
+            ptx::umma_commit(ptx::smem_u32(&sm.proj));
+            ok = wait(&sm.kp_ready);
+        }
+        if (ok) {
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // KS = K' S_{N-1}
+                ptx::umma_f16_ss(tmem + kColKS, kmajor_desc(xk, kk), mnmajor_desc(sb, kk), id_k_mn, kk > 0);
+            ptx::umma_commit(ptx::smem_u32(&sm.ks));
+            ok = wait(&sm.r_ready);
+        }
+        if (ok) {
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // dS = K'^T (beta R): sum over the chunk's tokens
+                ptx::umma_f16_ss(tmem + kColDS, mnmajor_desc(xk, kk), mnmajor_desc(xv, kk), id_mn_mn, kk > 0);
+            ptx::umma_commit(ptx::smem_u32(&sm.ds));
+        } else {
+            fail();
+            // no UMMA may still run when TMEM is released
+            ptx::umma_commit(ptx::smem_u32(&sm.ds));
+            ptx::mbar_wait_bounded(ptx::smem_u32(&sm.ds), 0, &no_abort, kWaitLimitNs);
+        }
+    } else if (warp >= 4) {
+        // --------------------------------------------------- epilogue --
+        const int r = threadIdx.x - 128;  // TMEM lane = tile row
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const int t = chunk * kChunk + r;
+        const float beta_t = t < L ? beta[(size_t)bh * L + t] : 0.f;
+        const uint32_t xk = ptx::smem_u32(sm.xk), xv = ptx::smem_u32(sm.xv);
+        const size_t part_row = (((size_t)bh * n_chunks + chunk) * kD + r) * kD;
+        bool ok = __all_sync(0xffffffffu, wait(&sm.proj));
+        if (ok) {
+            // K' = Kp / max(|Kp|, 1e-6) -> bf16 into xk (the K tile is consumed)
+            ptx::tc_fence_after();
+            uint32_t raw[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tmem + lane_base + kColKp + c * 32, raw[c]);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) ptx::reg_fence(raw[c]);
+            float ss = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(raw[c][i]), __uint_as_float(raw[c][i]), ss);
+            const float inv = 1.f / fmaxf(sqrtf(ss), 1e-6f);
+#pragma unroll
+            for (int c16 = 0; c16 < 16; ++c16) {
+                const uint32_t* s = &raw[c16 >> 2][(c16 & 3) * 8];
+                ptx::st_shared_v4(xk + ptx::tile_chunk_offset(r, c16),
+                                  ptx::pack_bf16x2(__uint_as_float(s[0]) * inv, __uint_as_float(s[1]) * inv),
+                                  ptx::pack_bf16x2(__uint_as_float(s[2]) * inv, __uint_as_float(s[3]) * inv),
+                                  ptx::pack_bf16x2(__uint_as_float(s[4]) * inv, __uint_as_float(s[5]) * inv),
+                                  ptx::pack_bf16x2(__uint_as_float(s[6]) * inv, __uint_as_float(s[7]) * inv));
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(ptx::smem_u32(&sm.kp_ready));
+            ok = __all_sync(0xffffffffu, wait(&sm.ks));
+        }
+        if (ok) {
+            // beta R = beta (Vp - K' S) -> bf16 into xv (the V tile is consumed)
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t vp[32], ks[32];
+                ptx::tmem_ld32(tmem + lane_base + kColVp + c * 32, vp);
+                ptx::tmem_ld32(tmem + lane_base + kColKS + c * 32, ks);
+                ptx::tmem_wait_ld();
+                ptx::reg_fence(vp);
+                ptx::reg_fence(ks);
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    float rr[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        rr[e] = beta_t * (__uint_as_float(vp[g * 8 + e]) - __uint_as_float(ks[g * 8 + e]));
+                    ptx::st_shared_v4(xv + ptx::tile_chunk_offset(r, c * 4 + g), ptx::pack_bf16x2(rr[0], rr[1]),
+                                      ptx::pack_bf16x2(rr[2], rr[3]), ptx::pack_bf16x2(rr[4], rr[5]),
+                                      ptx::pack_bf16x2(rr[6], rr[7]));
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(ptx::smem_u32(&sm.r_ready));
+            ok = __all_sync(0xffffffffu, wait(&sm.ds));
+        }
+        if (ok) {
+            // dS row r (key feature r): fp32 partial out
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t ds[32];
+                ptx::tmem_ld32(tmem + lane_base + kColDS + c * 32, ds);
+                ptx::tmem_wait_ld();
+                ptx::reg_fence(ds);
+                float4* dst = reinterpret_cast<float4*>(part_s + part_row + c * 32);
+#pragma unroll
+                for (int g = 0; g < 8; ++g)
+                    dst[g] = make_float4(__uint_as_float(ds[4 * g]), __uint_as_float(ds[4 * g + 1]),
+                                         __uint_as_float(ds[4 * g + 2]), __uint_as_float(ds[4 * g + 3]));
+            }
+        } else {
+            fail();
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Deterministic reduction of the chunk partials and the forget gate:
+// S_N = alpha S_{N-1} + sum over chunks (in chunk order) of dS.
+// One CTA: 8 rows of S of one (stream, head); one float4 per thread.
+__global__ void __launch_bounds__(256) update_finalize_kernel(const float* __restrict__ part_s,
+                                                              const float* __restrict__ alpha,
+                                                              float* __restrict__ S, int n_chunks,
+                                                              int H) {
+    const int h = blockIdx.y, b = blockIdx.z, bh = b * H + h;
+    const int e = blockIdx.x * 1024 + threadIdx.x * 4;  // element of the 128x128 matrix
+    const float a = alpha[bh];
+    const size_t base = (size_t)bh * kD * kD + e;
+    const size_t pbase = (size_t)bh * n_chunks * kD * kD + e;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < n_chunks; ++c) {
+        const float4 p = __ldcg(reinterpret_cast<const float4*>(part_s + pbase + (size_t)c * kD * kD));
+        acc.x += p.x;
+        acc.y += p.y;
+        acc.z += p.z;
+        acc.w += p.w;
+    }
+    float4 s = *reinterpret_cast<const float4*>(S + base);
+    s = make_float4(fmaf(a, s.x, acc.x), fmaf(a, s.y, acc.y), fmaf(a, s.z, acc.z), fmaf(a, s.w, acc.w));
+    *reinterpret_cast<float4*>(S + base) = s;
+}
+
+}  // namespace
+
+struct UpdateTc {
+    Dims dm{};
+    UpdateBuffers buf{};
+    int n_chunks = 0;
+    CUtensorMap tm_w{}, tm_sb{};
+};
+
+int update_tc_chunks(const Dims& dm) { return (dm.L + kChunk - 1) / kChunk; }
+
+UpdateTc* update_tc_create(const Dims& dm, const UpdateBuffers& buf) {
+    if (dm.d != kD || !tma_available()) return nullptr;
+    if (cudaFuncSetAttribute(update_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    UpdateTc* u = new (std::nothrow) UpdateTc();
+    if (!u) return nullptr;
+    u->dm = dm;
+    u->buf = buf;
+    u->n_chunks = update_tc_chunks(dm);
+    if (!tma_encode_tiles(&u->tm_w, buf.w_all, 3 * dm.H) ||
+        !tma_encode_tiles(&u->tm_sb, buf.Sb, dm.B * dm.H)) {
+        delete u;
+        return nullptr;
+    }
+    return u;
+}
+
+void update_tc_destroy(UpdateTc* u) { delete u; }
+
+cudaError_t update_tc_launch(UpdateTc* u, TokenMapCache& maps, const void* k, const void* v,
+                             const float* alpha, const float* beta, int* err, cudaStream_t st) {
+    const Dims& dm = u->dm;
+    CUtensorMap ck, cv;
+    if (!maps.get(k, &ck) || !maps.get(v, &cv)) return cudaErrorInvalidValue;
+    update_chunk_kernel<<<dim3(u->n_chunks, dm.H, dm.B), kThreads, kSmemBytes, st>>>(
+        ck, cv, u->tm_w, u->tm_sb, beta, u->buf.part_s, dm.L, dm.H, err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    update_finalize_kernel<<<dim3(kD * kD / 1024, dm.H, dm.B), 256, 0, st>>>(
+        u->buf.part_s, alpha, u->buf.S, u->n_chunks, dm.H);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return launch_fold_state(u->buf.w_all, u->buf.S, u->buf.Mt, u->buf.Sb, dm, st);
+}
+
+}  // namespace arl2

@@ -39,7 +39,7 @@ def test_binding_covers_every_export():
 
 
 def test_version_and_status_strings():
-    assert arl2.version() == 10000
+    assert arl2.version() == 10100
     for code in range(0, -8, -1):
         s = arl2._lib.arl2_status_string(code).decode()
         assert s and s != "unknown status"
