@@ -43,6 +43,7 @@ class Arl2Config(ctypes.Structure):
         ("tokens_per_frame", ctypes.c_int), ("dtype", ctypes.c_int),
         ("w_q", ctypes.c_void_p), ("w_k", ctypes.c_void_p), ("w_v", ctypes.c_void_p),
         ("softmax_scale", ctypes.c_float), ("host_staging", ctypes.c_int), ("impl", ctypes.c_int),
+        ("max_ctas", ctypes.c_int),
     ]
 
 
@@ -128,7 +129,7 @@ class Arl2Layer:
 
     def __init__(self, batch: int, heads: int, head_dim: int, tokens: int, w_q, w_k, w_v, *,
                  dtype: torch.dtype = torch.bfloat16, softmax_scale: float = 0.0,
-                 host_staging: bool = False, impl: str = "auto", stream=None):
+                 host_staging: bool = False, impl: str = "auto", max_ctas: int = 0, stream=None):
         if dtype not in (torch.bfloat16, torch.float32):
             raise ValueError("dtype must be torch.bfloat16 or torch.float32")
         for w in (w_q, w_k, w_v):
@@ -143,7 +144,7 @@ class Arl2Layer:
                          ARL2_BF16 if dtype == torch.bfloat16 else ARL2_FP32,
                          w_q.data_ptr(), w_k.data_ptr(), w_v.data_ptr(), float(softmax_scale),
                          1 if host_staging else 0,
-                         {"auto": ARL2_IMPL_AUTO, "simt": ARL2_IMPL_SIMT}[impl])
+                         {"auto": ARL2_IMPL_AUTO, "simt": ARL2_IMPL_SIMT}[impl], int(max_ctas))
         h = ctypes.c_void_p()
         with torch.cuda.device(self.device):
             _check(_lib.arl2_create(ctypes.byref(cfg), _stream(stream), ctypes.byref(h)), "arl2_create")

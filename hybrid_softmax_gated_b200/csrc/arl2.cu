@@ -46,6 +46,7 @@ struct arl2_handle {
     void* Mt = nullptr;       // bf16 (W_q S)^T, read by the attention kernel
     void* Sb = nullptr;       // bf16 S, read by the update kernel
     float* part_s = nullptr;  // fp32 update partials [B][H][chunks][d][d]
+    void* attn_ws = nullptr;  // attention split-tile partials and flags
     arl2::TokenMapCache* maps = nullptr;
     arl2::AttnTc* tc = nullptr;
     arl2::UpdateTc* up = nullptr;
@@ -93,7 +94,7 @@ void release(arl2_handle* h) {
     if (h->tc) arl2::attn_tc_destroy(h->tc);
     if (h->up) arl2::update_tc_destroy(h->up);
     delete h->maps;
-    void* ptrs[] = {h->w_all, h->S, h->Mt, h->Sb, h->part_s, h->qp, h->kp,
+    void* ptrs[] = {h->w_all, h->S, h->Mt, h->Sb, h->part_s, h->attn_ws, h->qp, h->kp,
                     h->vp, h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], h->stage_tok[3],
                     h->stage_alpha, h->stage_beta, h->err};
     for (void* p : ptrs)
@@ -167,6 +168,7 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
         cfg->head_dim > kMaxHeadDim)
         return ARL2_ERR_SHAPE;
     if (!(cfg->softmax_scale >= 0.f) || std::isinf(cfg->softmax_scale)) return ARL2_ERR_INVALID_ARG;
+    if (cfg->max_ctas < 0) return ARL2_ERR_INVALID_ARG;
     if (!aligned16(cfg->w_q) || !aligned16(cfg->w_k) || !aligned16(cfg->w_v)) return ARL2_ERR_ALIGN;
     const bool use_tc = cfg->impl == ARL2_IMPL_AUTO && cfg->dtype == ARL2_BF16;
     if (use_tc && cfg->head_dim != 128) return ARL2_ERR_UNSUPPORTED;
@@ -199,6 +201,7 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
         if (s == ARL2_OK) s = dalloc(h, &h->Mt, h->n_state * 2);
         if (s == ARL2_OK) s = dalloc(h, &h->Sb, h->n_state * 2);
         if (s == ARL2_OK) s = dalloc(h, &h->part_s, parts * sizeof(float));
+        if (s == ARL2_OK) s = dalloc(h, &h->attn_ws, arl2::attn_tc_workspace_bytes(dm));
     } else {
         if (s == ARL2_OK) s = dalloc(h, &h->qp, h->n_tok * sizeof(float));
         if (s == ARL2_OK) s = dalloc(h, &h->kp, h->n_tok * sizeof(float));
@@ -212,7 +215,7 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
     if (s == ARL2_OK && arl2::simt_init() != cudaSuccess) s = ARL2_ERR_CUDA;
     if (s == ARL2_OK && use_tc) {
         h->maps = new (std::nothrow) arl2::TokenMapCache(dm);
-        h->tc = arl2::attn_tc_create(dm);
+        h->tc = arl2::attn_tc_create(dm, h->attn_ws, cfg->max_ctas);
         const arl2::UpdateBuffers ub{h->w_all, h->S, h->Sb, h->Mt, h->part_s};
         h->up = arl2::update_tc_create(dm, ub);
         if (!h->maps || !h->maps->ok() || !h->tc || !h->up) s = ARL2_ERR_CUDA;
@@ -227,6 +230,9 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
             s = ARL2_ERR_CUDA;
     if (s == ARL2_OK) s = zero_state(h, stream);
     if (s == ARL2_OK && cudaMemsetAsync(h->err, 0, sizeof(int), stream) != cudaSuccess)
+        s = ARL2_ERR_CUDA;
+    if (s == ARL2_OK && use_tc &&
+        cudaMemsetAsync(h->attn_ws, 0, arl2::attn_tc_workspace_bytes(dm), stream) != cudaSuccess)
         s = ARL2_ERR_CUDA;
     if (s != ARL2_OK) {
         cudaStreamSynchronize(stream);
@@ -346,7 +352,14 @@ arl2_status arl2_device_status(arl2_handle* h, cudaStream_t stream) {
     if (cudaMemcpy(&word, h->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
         return ARL2_ERR_CUDA;
     if (word != 0) {
+        // a kernel gave up: clear the error word and any split-tile flags it
+        // may have left set, so that the next launch starts clean
         if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess) return ARL2_ERR_CUDA;
+        if (h->use_tc) {
+            size_t nflags = 0;
+            int* flags = arl2::attn_tc_flags(h->tc, &nflags);
+            if (cudaMemset(flags, 0, nflags * sizeof(int)) != cudaSuccess) return ARL2_ERR_CUDA;
+        }
         return ARL2_ERR_TIMEOUT;
     }
     return ARL2_OK;

@@ -8,19 +8,34 @@
 //
 // Since phi_q is a plain linear map, Q' S = Q (W_q S): the product
 // M = W_q S is formed once per frame when the state changes, and the read
-// becomes one extra 128x128x128 tensor-core product of the Q tile this CTA
-// already holds in shared memory.  O = O_intra + O_inter leaves the kernel
-// once, in bf16.
+// becomes one extra 128x128x128 tensor-core product of a Q tile that is in
+// shared memory anyway.  O = O_intra + O_inter leaves the kernel once, bf16.
 //
-// One CTA owns 128 query rows of one (stream, head):
-//   warp 0      TMA producer: Q, then K/V blocks of 128 keys through a
-//               2-stage ring, then the (W_q S)^T tile in the K ring
-//   warp 1      UMMA issuer (one thread): S_j = Q K_j^T into TMEM
-//               (double-buffered), O += P_j V_j, O_inter = Q M
-//   warp 2      TMEM allocator
-//   warps 4-7   softmax + epilogue: thread i owns query row i (TMEM lane i)
-// TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256,384) O,
-// [384,512) O_inter, all fp32.
+// Work decomposition.  A tile is 128 query rows of one (stream, head); a
+// unit is one tile against one block of 128 keys.  When there are more
+// tiles than SMs the grid is persistent (one CTA per SM, cooperative launch
+// so that all CTAs are resident) and CTA c takes the contiguous unit range
+// [c U / G, (c+1) U / G).  A tile cut by a range boundary has a head piece
+// (its first key blocks, at the end of CTA c's range) and a tail piece (the
+// rest, at the start of CTA c+1's range).  Each CTA runs its head piece
+// FIRST and writes it as an fp32 partial (unnormalised O, running max, row
+// sum) with a release flag; it runs its tail piece LAST, then acquires the
+// flag of the partial the previous CTA wrote at its start and merges the
+// two.  Waits are bounded.  With no more tiles than SMs, one CTA per tile.
+//
+// One CTA, 384 threads:
+//   warp 0       TMA producer: Q tiles (2 slots), K and V blocks (2-stage
+//                rings), the (W_q S)^T tile through the K ring
+//   warp 1       UMMA issuer (one thread): S = Q K^T into TMEM (two
+//                buffers), O += P V with P read from TMEM, O_inter = Q M
+//   warp 2       TMEM allocator
+//   warps 4-7    softmax warpgroup 0: keys 0-63 of each block, O cols 0-63
+//   warps 8-11   softmax warpgroup 1: keys 64-127, O cols 64-127
+// Row r of a tile is TMEM lane r; both warpgroups own row r (lane quadrant
+// = warp % 4) and exchange row maxima and sums through shared memory,
+// synchronised by mbarriers (bounded waits, unlike bar.sync).
+// TMEM columns: [0,128) S/P buffer 0, [128,256) S/P buffer 1, [256,384) O,
+// [384,512) O_inter, fp32 (P: bf16 pairs packed over its S buffer).
 // Online softmax with lazy rescaling: the running row max only moves when
 // it grows by more than 2^8; the final 1/l uses the same max as the
 // numerator, so the result is exact up to rounding.
@@ -36,64 +51,132 @@
 namespace arl2 {
 namespace {
 
-constexpr int kBM = 128;                       // query rows per CTA
-constexpr int kBN = 128;                       // keys per block
-constexpr int kD = 128;                        // head dim
 using ptx::kHalfBytes;
 using ptx::kTileBytes;
 using ptx::kmajor_desc;
 using ptx::mnmajor_desc;
-constexpr int kStages = 2;
-constexpr int kThreads = 256;
+
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // keys per block
+constexpr int kD = 128;   // head dim
+constexpr int kThreads = 384;
+constexpr int kSoftmaxThreads = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256, kColOi = 384;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
 
+enum SegKind : int { kFull = 0, kHead = 1, kTail = 2 };
+
+struct Seg {
+    int tile, kv0, kv1, kind;
+};
+
+// Unit schedule shared by every role of every CTA.
+struct Sched {
+    int n_q, n_kv, T;  // tiles per (stream, head), key blocks, tiles in total
+    int G;             // CTAs
+    int split;         // 1: persistent unit ranges, 0: one tile per CTA
+    long long U;       // units
+};
+
+struct CtaRange {
+    int n_segs;
+    int has_head, has_tail;
+    int t_first, t_last, e0, e1;  // e0: first key block of t_first; e1: end block of t_last
+    int full_lo, full_hi;         // full tiles [full_lo, full_hi)
+};
+
+__device__ __forceinline__ CtaRange cta_range(const Sched& s, int c) {
+    CtaRange r{};
+    if (!s.split) {
+        r.n_segs = 1;
+        r.full_lo = c;
+        r.full_hi = c + 1;
+        return r;
+    }
+    const long long u0 = (long long)c * s.U / s.G, u1 = (long long)(c + 1) * s.U / s.G;
+    r.t_first = (int)(u0 / s.n_kv);
+    r.e0 = (int)(u0 - (long long)r.t_first * s.n_kv);
+    r.t_last = (int)((u1 - 1) / s.n_kv);
+    r.e1 = (int)(u1 - (long long)r.t_last * s.n_kv);
+    r.has_tail = r.e0 > 0;
+    r.has_head = r.e1 < s.n_kv;  // (t_last > t_first whenever units per CTA >= n_kv)
+    r.full_lo = r.t_first + (r.has_tail ? 1 : 0);
+    r.full_hi = r.t_last + (r.has_head ? 0 : 1);
+    if (r.full_hi < r.full_lo) r.full_hi = r.full_lo;
+    r.n_segs = r.has_head + (r.full_hi - r.full_lo) + r.has_tail;
+    return r;
+}
+
+// Segment i of the CTA: head piece first, full tiles, tail piece last.
+__device__ __forceinline__ Seg seg_at(const Sched& s, const CtaRange& r, int i) {
+    if (r.has_head) {
+        if (i == 0) return Seg{r.t_last, 0, r.e1, kHead};
+        --i;
+    }
+    const int nf = r.full_hi - r.full_lo;
+    if (i < nf) return Seg{r.full_lo + i, 0, s.n_kv, kFull};
+    return Seg{r.t_first, r.e0, s.n_kv, kTail};
+}
+
 struct __align__(1024) Smem {
-    uint8_t q[kTileBytes];
-    uint8_t k[kStages][kTileBytes];
-    uint8_t v[kStages][kTileBytes];
-    uint8_t p[kTileBytes];
-    uint64_t q_full;
-    uint64_t k_full[kStages], k_empty[kStages];
-    uint64_t v_full[kStages], v_empty[kStages];
-    uint64_t s_full[2], s_empty[2];
-    uint64_t p_full, o_ready, done;
+    uint8_t q[2][kTileBytes];
+    uint8_t k[2][kTileBytes];
+    uint8_t v[2][kTileBytes];
+    uint64_t q_full[2], q_empty[2];
+    uint64_t k_full[2], k_empty[2];
+    uint64_t v_full[2], v_empty[2];
+    uint64_t s_full[2];
+    uint64_t p_full;    // 256 arrivals per key block: P written (and O rescaled)
+    uint64_t o_ready;   // one commit per key block: that block's P V is done
+    uint64_t seg_done;  // one commit per segment: its last UMMA is done
+    uint64_t o_free;    // 256 arrivals per segment: O and O_inter read out
+    uint64_t xch[2];    // 256 arrivals: row maxima of a key block exchanged
+    uint64_t ebar;      // 256 arrivals: epilogue exchanges
+    float red_max[2][2][kBM];  // [block parity][warpgroup][row]
+    float red_sum[2][kBM];     // [warpgroup][row]
     uint32_t tmem_base;
     int abort;
 };
-
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+
+__device__ __forceinline__ int valid_keys(int L, int kv) {
+    const int v = L - kv * kBN;
+    return v < kBN ? v : kBN;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_m,
-                   __nv_bfloat16* __restrict__ out, int L, int H, float scale_log2, int* err) {
+                   __nv_bfloat16* __restrict__ out, float* __restrict__ part_o,
+                   float* __restrict__ part_ml, int* __restrict__ flags, int L, int H, Sched sch,
+                   float scale_log2, int* err) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                         ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int n_kv = (L + kBN - 1) / kBN;
     volatile int* abort = &sm.abort;
     const int no_abort = 0;
+    const CtaRange rng = cta_range(sch, blockIdx.x);
 
     if (threadIdx.x == 0) {
-        ptx::mbar_init(ptx::smem_u32(&sm.q_full), 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(ptx::smem_u32(&sm.q_full[s]), 1);
+            ptx::mbar_init(ptx::smem_u32(&sm.q_empty[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sm.k_full[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sm.k_empty[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sm.v_full[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sm.v_empty[s]), 1);
-        }
-        for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(ptx::smem_u32(&sm.s_full[s]), 1);
-            ptx::mbar_init(ptx::smem_u32(&sm.s_empty[s]), kBM);
         }
-        ptx::mbar_init(ptx::smem_u32(&sm.p_full), kBM);
+        ptx::mbar_init(ptx::smem_u32(&sm.p_full), kSoftmaxThreads);
         ptx::mbar_init(ptx::smem_u32(&sm.o_ready), 1);
-        ptx::mbar_init(ptx::smem_u32(&sm.done), 1);
+        ptx::mbar_init(ptx::smem_u32(&sm.seg_done), 1);
+        ptx::mbar_init(ptx::smem_u32(&sm.o_free), kSoftmaxThreads);
+        ptx::mbar_init(ptx::smem_u32(&sm.xch[0]), kSoftmaxThreads);
+        ptx::mbar_init(ptx::smem_u32(&sm.xch[1]), kSoftmaxThreads);
+        ptx::mbar_init(ptx::smem_u32(&sm.ebar), kSoftmaxThreads);
         sm.abort = 0;
         ptx::fence_mbar_init();
         ptx::fence_proxy_async_smem();
@@ -111,6 +194,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicOr(err, kErrTimeoutAttn);
         *abort = 1;
     };
+    auto bwait = [&](uint64_t* bar, uint32_t parity) {
+        return ptx::mbar_wait_bounded(ptx::smem_u32(bar), parity, abort, kWaitLimitNs);
+    };
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------ TMA producer --
@@ -118,193 +204,225 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tma_prefetch_desc(&tm_k);
         ptx::tma_prefetch_desc(&tm_v);
         ptx::tma_prefetch_desc(&tm_m);
-        const uint32_t q_s = ptx::smem_u32(sm.q);
-        const int t0 = qt * kBM;
-        ptx::mbar_arrive_expect_tx(ptx::smem_u32(&sm.q_full), kTileBytes);
-        ptx::tma_load_4d(q_s, &tm_q, 0, h, t0, b, ptx::smem_u32(&sm.q_full));
-        ptx::tma_load_4d(q_s + kHalfBytes, &tm_q, 64, h, t0, b, ptx::smem_u32(&sm.q_full));
-        // Block i of the K ring is keys [128 i, 128 i + 128); block n_kv is
-        // the (W_q S)^T tile.  Loads follow the order the UMMA warp
-        // consumes them: K0, then (K_{j+1}, V_j) for j = 0 .. n_kv-1.
-        auto load_k = [&](int i) -> bool {
-            const int s = i & 1;
-            if (i >= 2 &&
-                !ptx::mbar_wait_bounded(ptx::smem_u32(&sm.k_empty[s]), ((i >> 1) - 1) & 1, abort,
-                                        kWaitLimitNs))
-                return false;
-            const uint32_t bar = ptx::smem_u32(&sm.k_full[s]);
-            const uint32_t dst = ptx::smem_u32(sm.k[s]);
+        int kc = 0, vc = 0;  // ring counters (same sequence as the UMMA issuer)
+        bool ok = true;
+        auto load_k = [&](int b, int h, int kv) -> bool {  // kv < 0: the (W_q S)^T tile
+            const int s = kc & 1;
+            if (kc >= 2 && !bwait(&sm.k_empty[s], ((kc >> 1) - 1) & 1)) return false;
+            const uint32_t bar = ptx::smem_u32(&sm.k_full[s]), dst = ptx::smem_u32(sm.k[s]);
             ptx::mbar_arrive_expect_tx(bar, kTileBytes);
-            if (i < n_kv) {
-                ptx::tma_load_4d(dst, &tm_k, 0, h, i * kBN, b, bar);
-                ptx::tma_load_4d(dst + kHalfBytes, &tm_k, 64, h, i * kBN, b, bar);
+            if (kv >= 0) {
+                ptx::tma_load_4d(dst, &tm_k, 0, h, kv * kBN, b, bar);
+                ptx::tma_load_4d(dst + kHalfBytes, &tm_k, 64, h, kv * kBN, b, bar);
             } else {
                 ptx::tma_load_4d(dst, &tm_m, 0, 0, b * H + h, 0, bar);
                 ptx::tma_load_4d(dst + kHalfBytes, &tm_m, 64, 0, b * H + h, 0, bar);
             }
+            ++kc;
             return true;
         };
-        auto load_v = [&](int j) -> bool {
-            const int s = j & 1;
-            if (j >= 2 &&
-                !ptx::mbar_wait_bounded(ptx::smem_u32(&sm.v_empty[s]), ((j >> 1) - 1) & 1, abort,
-                                        kWaitLimitNs))
-                return false;
-            const uint32_t bar = ptx::smem_u32(&sm.v_full[s]);
-            const uint32_t dst = ptx::smem_u32(sm.v[s]);
+        auto load_v = [&](int b, int h, int kv) -> bool {
+            const int s = vc & 1;
+            if (vc >= 2 && !bwait(&sm.v_empty[s], ((vc >> 1) - 1) & 1)) return false;
+            const uint32_t bar = ptx::smem_u32(&sm.v_full[s]), dst = ptx::smem_u32(sm.v[s]);
             ptx::mbar_arrive_expect_tx(bar, kTileBytes);
-            ptx::tma_load_4d(dst, &tm_v, 0, h, j * kBN, b, bar);
-            ptx::tma_load_4d(dst + kHalfBytes, &tm_v, 64, h, j * kBN, b, bar);
+            ptx::tma_load_4d(dst, &tm_v, 0, h, kv * kBN, b, bar);
+            ptx::tma_load_4d(dst + kHalfBytes, &tm_v, 64, h, kv * kBN, b, bar);
+            ++vc;
             return true;
         };
-        bool ok = load_k(0);
-        int k_issued = ok ? 1 : 0, v_issued = 0;
-        for (int j = 0; ok && j < n_kv; ++j) {
-            ok = load_k(j + 1);
-            if (ok) k_issued = j + 2;
-            if (ok) ok = load_v(j);
-            if (ok) v_issued = j + 1;
+        int si = 0;
+        for (; ok && si < rng.n_segs; ++si) {
+            const Seg sg = seg_at(sch, rng, si);
+            const int bh = sg.tile / sch.n_q, qt = sg.tile - bh * sch.n_q;
+            const int b = bh / H, h = bh - b * H;
+            const int qs = si & 1;
+            if (si >= 2 && !bwait(&sm.q_empty[qs], ((si >> 1) - 1) & 1)) {
+                ok = false;
+                break;
+            }
+            const uint32_t qbar = ptx::smem_u32(&sm.q_full[qs]), qdst = ptx::smem_u32(sm.q[qs]);
+            ptx::mbar_arrive_expect_tx(qbar, kTileBytes);
+            ptx::tma_load_4d(qdst, &tm_q, 0, h, qt * kBM, b, qbar);
+            ptx::tma_load_4d(qdst + kHalfBytes, &tm_q, 64, h, qt * kBM, b, qbar);
+            // K and V in the order the issuer consumes them:
+            // K0 K1 V0 K2 V1 ... V_{n-1} [M]
+            const int n = sg.kv1 - sg.kv0;
+            ok = load_k(b, h, sg.kv0) && (n < 2 || load_k(b, h, sg.kv0 + 1));
+            for (int j = 0; ok && j < n; ++j) {
+                ok = load_v(b, h, sg.kv0 + j);
+                if (ok && j + 2 < n) ok = load_k(b, h, sg.kv0 + j + 2);
+            }
+            if (ok && sg.kind != kHead) ok = load_k(b, h, -1);
         }
         if (!ok) fail();
-        // Drain: every load this thread issued has landed before the CTA
-        // may exit (consumed phases return at once).
-        ptx::mbar_wait_bounded(ptx::smem_u32(&sm.q_full), 0, &no_abort, kWaitLimitNs);
-        for (int i = k_issued - 2; i < k_issued; ++i)
-            if (i >= 0)
-                ptx::mbar_wait_bounded(ptx::smem_u32(&sm.k_full[i & 1]), (i >> 1) & 1, &no_abort,
-                                       kWaitLimitNs);
-        for (int j = v_issued - 2; j < v_issued; ++j)
-            if (j >= 0)
-                ptx::mbar_wait_bounded(ptx::smem_u32(&sm.v_full[j & 1]), (j >> 1) & 1, &no_abort,
-                                       kWaitLimitNs);
+        // Drain: the last loads of each ring have landed before exit.
+        for (int i = kc - 2; i < kc; ++i)
+            if (i >= 0) ptx::mbar_wait_bounded(ptx::smem_u32(&sm.k_full[i & 1]), (i >> 1) & 1, &no_abort, kWaitLimitNs);
+        for (int i = vc - 2; i < vc; ++i)
+            if (i >= 0) ptx::mbar_wait_bounded(ptx::smem_u32(&sm.v_full[i & 1]), (i >> 1) & 1, &no_abort, kWaitLimitNs);
+        for (int i = si - 2; i < si; ++i)
+            if (i >= 0) ptx::mbar_wait_bounded(ptx::smem_u32(&sm.q_full[i & 1]), (i >> 1) & 1, &no_abort, kWaitLimitNs);
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------- UMMA issuer --
-        constexpr uint32_t idesc_kk = ptx::idesc_bf16_f32(kBM, kBN, false, false);
         constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBM, kD, false, true);
-        const uint32_t q_s = ptx::smem_u32(sm.q);
-        const uint32_t p_s = ptx::smem_u32(sm.p);
-        bool ok = ptx::mbar_wait_bounded(ptx::smem_u32(&sm.q_full), 0, abort, kWaitLimitNs);
-        auto issue_qk = [&](int i) -> bool {  // S_i = Q K_i^T into buffer i & 1
-            const int s = i & 1;
-            if (!ptx::mbar_wait_bounded(ptx::smem_u32(&sm.k_full[s]), (i >> 1) & 1, abort,
-                                        kWaitLimitNs))
-                return false;
-            if (i >= 2 && !ptx::mbar_wait_bounded(ptx::smem_u32(&sm.s_empty[s]), ((i >> 1) - 1) & 1,
-                                                  abort, kWaitLimitNs))
-                return false;
+        constexpr uint32_t idesc_qm = ptx::idesc_bf16_f32(kBM, kD, false, false);
+        int kc = 0, vc = 0, g = 0;
+        bool ok = true;
+        auto issue_qk = [&](uint32_t q_s, int blk, int kv) -> bool {  // S_blk = Q K^T
+            const int s = kc & 1;
+            if (!bwait(&sm.k_full[s], (kc >> 1) & 1)) return false;
             ptx::tc_fence_after();
+            const int valid = valid_keys(L, kv);
+            const uint32_t idesc = ptx::idesc_bf16_f32(kBM, (valid + 15) & ~15, false, false);
             const uint32_t k_s = ptx::smem_u32(sm.k[s]);
-            const uint32_t d = tmem + kColS + (uint32_t)s * kBN;
+            const uint32_t d = tmem + kColS + (uint32_t)(blk & 1) * kBN;
 #pragma unroll
             for (int kk = 0; kk < kD / 16; ++kk)
-                ptx::umma_f16_ss(d, kmajor_desc(q_s, kk), kmajor_desc(k_s, kk), idesc_kk, kk > 0);
-            ptx::umma_commit(ptx::smem_u32(&sm.s_full[s]));
+                ptx::umma_f16_ss(d, kmajor_desc(q_s, kk), kmajor_desc(k_s, kk), idesc, kk > 0);
+            ptx::umma_commit(ptx::smem_u32(&sm.s_full[blk & 1]));
             ptx::umma_commit(ptx::smem_u32(&sm.k_empty[s]));
+            ++kc;
             return true;
         };
-        if (ok) ok = issue_qk(0);
-        for (int j = 0; ok && j < n_kv; ++j) {
-            if (j + 1 < n_kv) ok = issue_qk(j + 1);
-            if (!ok) break;
-            // O += P_j V_j
-            const int s = j & 1;
-            ok = ptx::mbar_wait_bounded(ptx::smem_u32(&sm.p_full), j & 1, abort, kWaitLimitNs) &&
-                 ptx::mbar_wait_bounded(ptx::smem_u32(&sm.v_full[s]), (j >> 1) & 1, abort,
-                                        kWaitLimitNs);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            const uint32_t v_s = ptx::smem_u32(sm.v[s]);
-#pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk)
-                ptx::umma_f16_ss(tmem + kColO, kmajor_desc(p_s, kk), mnmajor_desc(v_s, kk), idesc_pv,
-                                 (j > 0 || kk > 0) ? 1u : 0u);
-            ptx::umma_commit(ptx::smem_u32(&sm.v_empty[s]));
-            ptx::umma_commit(ptx::smem_u32(&sm.o_ready));
-        }
-        if (ok) {
-            // O_inter = Q (W_q S)^T^T, the folded state tile sits in K slot n_kv
-            const int s = n_kv & 1;
-            ok = ptx::mbar_wait_bounded(ptx::smem_u32(&sm.k_full[s]), (n_kv >> 1) & 1, abort,
-                                        kWaitLimitNs);
-            if (ok) {
-                ptx::tc_fence_after();
-                const uint32_t m_s = ptx::smem_u32(sm.k[s]);
-#pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)
-                    ptx::umma_f16_ss(tmem + kColOi, kmajor_desc(q_s, kk), kmajor_desc(m_s, kk),
-                                     idesc_kk, kk > 0);
+        int si = 0;
+        for (; ok && si < rng.n_segs; ++si) {
+            const Seg sg = seg_at(sch, rng, si);
+            const int qs = si & 1;
+            const int n = sg.kv1 - sg.kv0;
+            if (!bwait(&sm.q_full[qs], (si >> 1) & 1)) {
+                ok = false;
+                break;
             }
-        }
-        if (!ok) fail();
-        // Completion of everything issued above (also on the failure path,
-        // so that no UMMA is in flight when TMEM is released).
-        ptx::umma_commit(ptx::smem_u32(&sm.done));
-        if (!ok)
-            ptx::mbar_wait_bounded(ptx::smem_u32(&sm.done), 0, &no_abort, kWaitLimitNs);
-    } else if (warp >= 4) {
-        // ---------------------------------------- softmax + epilogue --
-        const int row = threadIdx.x - 128;                 // query row in tile = TMEM lane
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t p_row = ptx::smem_u32(sm.p) + (uint32_t)row * 128u;
-        float m_run = -INFINITY, l_run = 0.f;
-        bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
-            const int s = j & 1;
-            // The decision to stop is made warp-wide, so that every lane
-            // reaches (or skips) the warp-collective tcgen05 ops together.
-            ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(ptx::smem_u32(&sm.s_full[s]),
-                                                                (j >> 1) & 1, abort, kWaitLimitNs));
-            if (!ok) break;
-            ptx::tc_fence_after();
-            uint32_t raw[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                ptx::tmem_ld32(tmem + lane_base + kColS + (uint32_t)s * kBN + (uint32_t)c * 32, raw[c]);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) ptx::reg_fence(raw[c]);
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(ptx::smem_u32(&sm.s_empty[s]));
-
-            float x[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(raw[c][i]) * scale_log2;
-            const int valid = L - j * kBN;  // keys of this block inside the frame
-            if (valid < kBN) {
-#pragma unroll
-                for (int i = 0; i < 128; ++i)
-                    if (i >= valid) x[i] = -INFINITY;
-            }
-            float mx = x[0];
-#pragma unroll
-            for (int i = 1; i < 128; ++i) mx = fmaxf(mx, x[i]);
-            const float m_new = fmaxf(m_run, mx);
-            const bool need = m_new > m_run + kRescaleLog2;
-            const float m_use = need ? m_new : m_run;
-            const float corr = need ? ptx::ex2(m_run - m_new) : 1.f;
-            float sum = 0.f;
-#pragma unroll
-            for (int i = 0; i < 128; ++i) {
-                x[i] = ptx::ex2(x[i] - m_use);
-                sum += x[i];
-            }
-            l_run = l_run * corr + sum;
-            m_run = m_use;
-
-            if (j >= 1) {
-                // PV_{j-1} done: O is stable and the P buffer is free.
-                ok = __all_sync(0xffffffffu,
-                                ptx::mbar_wait_bounded(ptx::smem_u32(&sm.o_ready), (j - 1) & 1,
-                                                       abort, kWaitLimitNs));
+            const uint32_t q_s = ptx::smem_u32(sm.q[qs]);
+            // S buffers are free: the P V that last read each was issued before.
+            ok = issue_qk(q_s, g, sg.kv0) && (n < 2 || issue_qk(q_s, g + 1, sg.kv0 + 1));
+            // O and O_inter of the previous segment have been read out.
+            if (ok && si >= 1) ok = bwait(&sm.o_free, (si - 1) & 1);
+            for (int j = 0; ok && j < n; ++j) {
+                const int blk = g + j;
+                const int vs = vc & 1;
+                ok = bwait(&sm.p_full, blk & 1) && bwait(&sm.v_full[vs], (vc >> 1) & 1);
                 if (!ok) break;
                 ptx::tc_fence_after();
-                if (__any_sync(0xffffffffu, need)) {
+                const int ksteps = (valid_keys(L, sg.kv0 + j) + 15) >> 4;
+                const uint32_t p_t = tmem + kColS + (uint32_t)(blk & 1) * kBN;
+                const uint32_t v_s = ptx::smem_u32(sm.v[vs]);
+                for (int kk = 0; kk < ksteps; ++kk)  // O += P V, P from TMEM
+                    ptx::umma_f16_ts(tmem + kColO, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv,
+                                     (j > 0 || kk > 0) ? 1u : 0u);
+                ptx::umma_commit(ptx::smem_u32(&sm.v_empty[vs]));
+                ptx::umma_commit(ptx::smem_u32(&sm.o_ready));
+                ++vc;
+                // The next QK into this S/P buffer follows the P V that reads it.
+                if (j + 2 < n) ok = issue_qk(q_s, blk + 2, sg.kv0 + j + 2);
+            }
+            if (ok && sg.kind != kHead) {
+                const int s = kc & 1;
+                ok = bwait(&sm.k_full[s], (kc >> 1) & 1);
+                if (ok) {
+                    ptx::tc_fence_after();
+                    const uint32_t m_s = ptx::smem_u32(sm.k[s]);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
+                    for (int kk = 0; kk < kD / 16; ++kk)  // O_inter = Q (W_q S)
+                        ptx::umma_f16_ss(tmem + kColOi, kmajor_desc(q_s, kk), kmajor_desc(m_s, kk), idesc_qm,
+                                         kk > 0);
+                    ptx::umma_commit(ptx::smem_u32(&sm.k_empty[s]));
+                    ++kc;
+                }
+            }
+            if (!ok) break;
+            ptx::umma_commit(ptx::smem_u32(&sm.q_empty[qs]));
+            ptx::umma_commit(ptx::smem_u32(&sm.seg_done));
+            g += n;
+        }
+        if (!ok) {
+            fail();
+            // nothing may still run on the tensor cores when TMEM is released
+            ptx::umma_commit(ptx::smem_u32(&sm.seg_done));
+            ptx::mbar_wait_bounded(ptx::smem_u32(&sm.seg_done), si & 1, &no_abort, kWaitLimitNs);
+        }
+    } else if (warp >= 4) {
+        // ---------------------------------------- softmax + epilogue --
+        const int wg = (warp - 4) >> 2;               // 0: keys/cols 0-63, 1: 64-127
+        const int row = ((warp & 3) << 5) + lane;     // tile row = TMEM lane
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t col0 = (uint32_t)wg * 64;
+        int g = 0;
+        uint32_t e_uses = 0;  // completed uses of ebar
+        bool ok = true;
+        // all 256 softmax threads meet at bar (arrive, then a bounded wait)
+        auto meet = [&](uint64_t* bar, uint32_t parity) -> bool {
+            ptx::mbar_arrive(ptx::smem_u32(bar));
+            return __all_sync(0xffffffffu, bwait(bar, parity));
+        };
+        auto meet_e = [&]() -> bool { return meet(&sm.ebar, (e_uses++) & 1); };
+        for (int si = 0; ok && si < rng.n_segs; ++si) {
+            const Seg sg = seg_at(sch, rng, si);
+            const int n = sg.kv1 - sg.kv0;
+            float m_run = -INFINITY, l_part = 0.f;
+            for (int j = 0; j < n; ++j) {
+                const int blk = g + j;
+                const uint32_t sbuf = tmem + lane_base + kColS + (uint32_t)(blk & 1) * kBN;
+                ok = __all_sync(0xffffffffu, bwait(&sm.s_full[blk & 1], (blk >> 1) & 1));
+                if (!ok) break;
+                ptx::tc_fence_after();
+                uint32_t raw[2][32];
+                ptx::tmem_ld32(sbuf + col0, raw[0]);
+                ptx::tmem_ld32(sbuf + col0 + 32, raw[1]);
+                ptx::tmem_wait_ld();
+                ptx::reg_fence(raw[0]);
+                ptx::reg_fence(raw[1]);
+                float x[64];
+#pragma unroll
+                for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(raw[i >> 5][i & 31]);
+                const int valid = valid_keys(L, sg.kv0 + j) - (int)col0;  // valid keys in my 64
+                if (valid < 64) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        if (i >= valid) x[i] = -INFINITY;
+                }
+                // row max of my 64 columns: 3-input max tree
+                float m8[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    m8[i] = ptx::max3(ptx::max3(x[8 * i], x[8 * i + 1], x[8 * i + 2]),
+                                      ptx::max3(x[8 * i + 3], x[8 * i + 4], x[8 * i + 5]),
+                                      fmaxf(x[8 * i + 6], x[8 * i + 7]));
+                float mx = ptx::max3(ptx::max3(m8[0], m8[1], m8[2]), ptx::max3(m8[3], m8[4], m8[5]),
+                                     fmaxf(m8[6], m8[7]));
+                sm.red_max[blk & 1][wg][row] = mx;
+                ok = meet(&sm.xch[blk & 1], (blk >> 1) & 1);
+                if (!ok) break;
+                mx = fmaxf(mx, sm.red_max[blk & 1][wg ^ 1][row]);
+                const float m_new = fmaxf(m_run, mx * scale_log2);
+                const bool need = m_new > m_run + kRescaleLog2;
+                const float m_use = need ? m_new : m_run;
+                const float corr = need ? ptx::ex2(m_run - m_new) : 1.f;
+                const float neg_m = -m_use;
+                float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float p0 = ptx::ex2(fmaf(x[2 * i], scale_log2, neg_m));
+                    const float p1 = ptx::ex2(fmaf(x[2 * i + 1], scale_log2, neg_m));
+                    sum4[i & 3] += p0 + p1;
+                    pk[i] = ptx::pack_bf16x2(p0, p1);
+                }
+                l_part = l_part * corr + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+                m_run = m_use;
+                // P over my half of the S columns (both warpgroups finished
+                // reading S at the barrier above)
+                ptx::tmem_st32_u(sbuf + (uint32_t)wg * 32, pk);
+                if (j >= 1 && __any_sync(0xffffffffu, need)) {
+                    // rescale my half of O once the previous P V is done
+                    ok = __all_sync(0xffffffffu, bwait(&sm.o_ready, (blk - 1) & 1));
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
                         uint32_t o[32];
-                        const uint32_t ta = tmem + lane_base + kColO + (uint32_t)c * 32;
+                        const uint32_t ta = tmem + lane_base + kColO + col0 + (uint32_t)c * 32;
                         ptx::tmem_ld32(ta, o);
                         ptx::tmem_wait_ld();
                         ptx::reg_fence(o);
@@ -312,68 +430,117 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
                         ptx::tmem_st32(ta, o);
                     }
-                    ptx::tmem_wait_st();
                 }
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(ptx::smem_u32(&sm.p_full));
             }
-            // P row -> shared memory, bf16, 128-byte swizzled K-major layout
-#pragma unroll
-            for (int ch = 0; ch < 16; ++ch) {
-                const int half = ch >> 3, c16 = ch & 7;
-                const __nv_bfloat162 p0 = __floats2bfloat162_rn(x[ch * 8 + 0], x[ch * 8 + 1]);
-                const __nv_bfloat162 p1 = __floats2bfloat162_rn(x[ch * 8 + 2], x[ch * 8 + 3]);
-                const __nv_bfloat162 p2 = __floats2bfloat162_rn(x[ch * 8 + 4], x[ch * 8 + 5]);
-                const __nv_bfloat162 p3 = __floats2bfloat162_rn(x[ch * 8 + 6], x[ch * 8 + 7]);
-                const uint32_t addr =
-                    p_row + (uint32_t)half * kHalfBytes + (uint32_t)((c16 ^ (row & 7)) << 4);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                             "r"(*reinterpret_cast<const uint32_t*>(&p0)),
-                             "r"(*reinterpret_cast<const uint32_t*>(&p1)),
-                             "r"(*reinterpret_cast<const uint32_t*>(&p2)),
-                             "r"(*reinterpret_cast<const uint32_t*>(&p3))
-                             : "memory");
-            }
-            ptx::fence_proxy_async_smem();
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(ptx::smem_u32(&sm.p_full));
-        }
-        if (ok)
-            ok = ptx::mbar_wait_bounded(ptx::smem_u32(&sm.o_ready), (n_kv - 1) & 1, abort,
-                                        kWaitLimitNs) &&
-                 ptx::mbar_wait_bounded(ptx::smem_u32(&sm.done), 0, abort, kWaitLimitNs);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) {
-            fail();
-        } else {
+            if (!ok) break;
+            // ------------------------------------------------ epilogue --
+            sm.red_sum[wg][row] = l_part;
+            ok = meet_e();
+            if (!ok) break;
+            const float l_row = l_part + sm.red_sum[wg ^ 1][row];
+            ok = __all_sync(0xffffffffu, bwait(&sm.seg_done, si & 1));
+            if (!ok) break;
             ptx::tc_fence_after();
-            const float inv_l = 1.f / l_run;
+            const int bh = sg.tile / sch.n_q, qt = sg.tile - bh * sch.n_q;
+            const int b = bh / H, h = bh - b * H;
             const int t = qt * kBM + row;
-            __nv_bfloat16* orow = out + (((size_t)b * L + t) * H + h) * kD;
+            float* prow = part_o + ((size_t)sg.tile * kBM + row) * kD + col0;
+            if (sg.kind == kHead) {
+                // unnormalised O, running max and row sum -> partial, then the flag
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t o[32], oi[32];
-                ptx::tmem_ld32(tmem + lane_base + kColO + (uint32_t)c * 32, o);
-                ptx::tmem_ld32(tmem + lane_base + kColOi + (uint32_t)c * 32, oi);
-                ptx::tmem_wait_ld();
-                ptx::reg_fence(o);
-                ptx::reg_fence(oi);
-                if (t < L) {
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t o[32];
+                    ptx::tmem_ld32(tmem + lane_base + kColO + col0 + (uint32_t)c * 32, o);
+                    ptx::tmem_wait_ld();
+                    ptx::reg_fence(o);
+                    float4* dst = reinterpret_cast<float4*>(prow + c * 32);
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i = g * 8 + e * 2;
-                            const float a0 = fmaf(__uint_as_float(o[i]), inv_l, __uint_as_float(oi[i]));
-                            const float a1 =
-                                fmaf(__uint_as_float(o[i + 1]), inv_l, __uint_as_float(oi[i + 1]));
-                            const __nv_bfloat162 pr = __floats2bfloat162_rn(a0, a1);
-                            w[e] = *reinterpret_cast<const uint32_t*>(&pr);
+                    for (int i = 0; i < 8; ++i)
+                        dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                             __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+                }
+                if (wg == 0)
+                    *reinterpret_cast<float2*>(part_ml + ((size_t)sg.tile * kBM + row) * 2) =
+                        make_float2(m_run, l_row);
+                __threadfence();
+                ok = meet_e();
+                if (!ok) break;
+                if (threadIdx.x == 128) ptx::st_release_gpu(flags + sg.tile, 1);
+            } else {
+                float a_t = 1.f, a_h = 0.f, inv_l = 1.f / l_row;
+                if (sg.kind == kTail) {
+                    // the head piece of this tile was written by the previous CTA
+                    // at its start
+                    if (threadIdx.x == 128) {
+                        const uint64_t t0 = ptx::globaltimer_ns();
+                        while (ptx::ld_acquire_gpu(flags + sg.tile) == 0) {
+                            if (*abort || ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+                                fail();
+                                break;
+                            }
                         }
-                        *reinterpret_cast<uint4*>(orow + c * 32 + g * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                    ok = meet_e();
+                    if (!ok) break;
+                    const float2 ml = __ldcg(reinterpret_cast<const float2*>(
+                        part_ml + ((size_t)sg.tile * kBM + row) * 2));
+                    const float mm = fmaxf(ml.x, m_run);
+                    a_h = ptx::ex2(ml.x - mm);
+                    a_t = ptx::ex2(m_run - mm);
+                    inv_l = 1.f / (a_h * ml.y + a_t * l_row);
+                }
+                __nv_bfloat16* orow = out + (((size_t)b * L + t) * H + h) * kD + col0;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t o[32], oi[32];
+                    ptx::tmem_ld32(tmem + lane_base + kColO + col0 + (uint32_t)c * 32, o);
+                    ptx::tmem_ld32(tmem + lane_base + kColOi + col0 + (uint32_t)c * 32, oi);
+                    ptx::tmem_wait_ld();
+                    ptx::reg_fence(o);
+                    ptx::reg_fence(oi);
+                    float acc[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[i] = a_t * __uint_as_float(o[i]);
+                    if (sg.kind == kTail) {
+                        const float4* src = reinterpret_cast<const float4*>(prow + c * 32);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 ph = __ldcg(src + i);
+                            acc[4 * i] = fmaf(a_h, ph.x, acc[4 * i]);
+                            acc[4 * i + 1] = fmaf(a_h, ph.y, acc[4 * i + 1]);
+                            acc[4 * i + 2] = fmaf(a_h, ph.z, acc[4 * i + 2]);
+                            acc[4 * i + 3] = fmaf(a_h, ph.w, acc[4 * i + 3]);
+                        }
+                    }
+                    if (t < L) {
+#pragma unroll
+                        for (int gq = 0; gq < 4; ++gq) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int i = gq * 8 + e * 2;
+                                w[e] = ptx::pack_bf16x2(fmaf(acc[i], inv_l, __uint_as_float(oi[i])),
+                                                        fmaf(acc[i + 1], inv_l, __uint_as_float(oi[i + 1])));
+                            }
+                            *reinterpret_cast<uint4*>(orow + c * 32 + gq * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
                     }
                 }
+                if (sg.kind == kTail) {
+                    // every thread has read the partial: clear the flag for the next launch
+                    ok = meet_e();
+                    if (!ok) break;
+                    if (threadIdx.x == 128) flags[sg.tile] = 0;
+                }
             }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(ptx::smem_u32(&sm.o_free));
+            g += n;
         }
+        if (!ok) fail();
     }
 
     ptx::tc_fence_before();
@@ -392,18 +559,52 @@ struct AttnTc {
     Dims dm{};
     const void* m_ptr = nullptr;
     CUtensorMap tm_m{};
+    Sched sch{};
+    float* part_o = nullptr;
+    float* part_ml = nullptr;
+    int* flags = nullptr;
 };
 
-AttnTc* attn_tc_create(Dims dm) {
-    if (dm.d != kD || dm.L < 1 || dm.H < 1 || dm.B < 1 || !tma_available()) return nullptr;
+size_t attn_tc_workspace_bytes(const Dims& dm) {
+    const size_t tiles = (size_t)dm.B * dm.H * ((dm.L + kBM - 1) / kBM);
+    return tiles * ((size_t)kBM * kD * 4 + (size_t)kBM * 2 * 4 + 4);
+}
+
+AttnTc* attn_tc_create(Dims dm, void* workspace, int max_ctas) {
+    if (dm.d != kD || dm.L < 1 || dm.H < 1 || dm.B < 1 || !tma_available() || !workspace) return nullptr;
     if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes) != cudaSuccess) {
         cudaGetLastError();
         return nullptr;
     }
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
+        cudaGetLastError();
+        return nullptr;
+    }
     AttnTc* t = new (std::nothrow) AttnTc();
-    if (t) t->dm = dm;
+    if (!t) return nullptr;
+    t->dm = dm;
+    Sched& s = t->sch;
+    s.n_q = (dm.L + kBM - 1) / kBM;
+    s.n_kv = (dm.L + kBN - 1) / kBN;
+    s.T = dm.B * dm.H * s.n_q;
+    s.U = (long long)s.T * s.n_kv;
+    const int G = max_ctas > 0 && max_ctas < sms ? max_ctas : sms;
+    s.split = s.T > G ? 1 : 0;
+    s.G = s.split ? G : s.T;
+    const size_t tiles = (size_t)s.T;
+    char* w = static_cast<char*>(workspace);
+    t->part_o = reinterpret_cast<float*>(w);
+    t->part_ml = reinterpret_cast<float*>(w + tiles * kBM * kD * 4);
+    t->flags = reinterpret_cast<int*>(w + tiles * kBM * kD * 4 + tiles * kBM * 2 * 4);
     return t;
+}
+
+int* attn_tc_flags(AttnTc* t, size_t* count) {
+    *count = (size_t)t->sch.T;
+    return t->flags;
 }
 
 void attn_tc_destroy(AttnTc* t) { delete t; }
@@ -418,11 +619,20 @@ cudaError_t attn_tc_launch(AttnTc* t, TokenMapCache& maps, const void* q, const 
     }
     CUtensorMap cq, ck, cv;
     if (!maps.get(q, &cq) || !maps.get(k, &ck) || !maps.get(v, &cv)) return cudaErrorInvalidValue;
-    const dim3 grid((dm.L + kBM - 1) / kBM, dm.H, dm.B);
-    attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(cq, ck, cv, t->tm_m,
-                                                       static_cast<__nv_bfloat16*>(out), dm.L, dm.H,
-                                                       scale * 1.4426950408889634f, err);
-    return cudaGetLastError();
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+    const float sl2 = scale * 1.4426950408889634f;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(t->sch.G, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = t->sch.split ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, attn_tc_kernel, cq, ck, cv, t->tm_m, o, t->part_o, t->part_ml,
+                              t->flags, dm.L, dm.H, t->sch, sl2, err);
 }
 
 }  // namespace arl2

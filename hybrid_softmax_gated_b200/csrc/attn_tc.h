@@ -10,10 +10,19 @@ namespace arl2 {
 
 struct AttnTc;
 
-// Configure the kernel for the given dimensions.  Returns nullptr on
-// failure (no tensor-map encoder, bad dims).
-AttnTc* attn_tc_create(Dims dm);
+// Device workspace the kernel needs (split-tile partials and flags).
+size_t attn_tc_workspace_bytes(const Dims& dm);
+
+// Configure the kernel for the given dimensions.  workspace: device buffer
+// of attn_tc_workspace_bytes(dm) bytes, its flag words zeroed (see
+// attn_tc_flags).  max_ctas > 0 caps the persistent grid (else one CTA per
+// SM).  Returns nullptr on failure (no tensor-map encoder, bad dims).
+AttnTc* attn_tc_create(Dims dm, void* workspace, int max_ctas);
 void attn_tc_destroy(AttnTc* t);
+
+// The split-tile flag words inside the workspace (count of them in *count);
+// they must be zero between launches.
+int* attn_tc_flags(AttnTc* t, size_t* count);
 
 // q, k, v, out: [B][L][H][128] bf16.  Mt: [B][H][128][128] bf16 holding
 // (W_q S)^T.  err: device error word (bit kErrTimeoutAttn on a timeout).

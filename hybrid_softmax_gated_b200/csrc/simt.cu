@@ -262,7 +262,16 @@ __global__ void __launch_bounds__(128) fold_state_kernel(const __nv_bfloat16* __
     const int n = threadIdx.x;
     const size_t base = ((size_t)b * dm.H + h) * d * d;
     const __nv_bfloat16* W = wq + (size_t)h * d * d;
-    for (int i = threadIdx.x; i < d * d; i += blockDim.x) Ss[i] = S[base + i];
+    if ((d & 3) == 0) {
+        // float4 copies, unrolled so that many loads are in flight at once
+        const float4* src = reinterpret_cast<const float4*>(S + base);
+        float4* dst = reinterpret_cast<float4*>(Ss);
+        const int n4 = d * d / 4;
+#pragma unroll 8
+        for (int i = threadIdx.x; i < n4; i += blockDim.x) dst[i] = src[i];
+    } else {
+        for (int i = threadIdx.x; i < d * d; i += blockDim.x) Ss[i] = S[base + i];
+    }
     for (int i = threadIdx.x; i < kFoldRows * d; i += blockDim.x) {
         const int r = i / d, c = i - r * d;
         Ws[i] = a0 + r < d ? __bfloat162float(W[(size_t)(a0 + r) * d + c]) : 0.f;

@@ -266,12 +266,22 @@ __global__ void __launch_bounds__(256) update_finalize_kernel(const float* __res
     const size_t base = (size_t)bh * kD * kD + e;
     const size_t pbase = (size_t)bh * n_chunks * kD * kD + e;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = 0; c < n_chunks; ++c) {
-        const float4 p = __ldcg(reinterpret_cast<const float4*>(part_s + pbase + (size_t)c * kD * kD));
-        acc.x += p.x;
-        acc.y += p.y;
-        acc.z += p.z;
-        acc.w += p.w;
+    // Loads in groups of 8 so that they are in flight together; the sum
+    // itself stays in chunk order.
+    for (int c0 = 0; c0 < n_chunks; c0 += 8) {
+        float4 p[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (c0 + i < n_chunks)
+                p[i] = __ldcg(reinterpret_cast<const float4*>(part_s + pbase + (size_t)(c0 + i) * kD * kD));
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (c0 + i < n_chunks) {
+                acc.x += p[i].x;
+                acc.y += p[i].y;
+                acc.z += p[i].z;
+                acc.w += p[i].w;
+            }
     }
     float4 s = *reinterpret_cast<const float4*>(S + base);
     s = make_float4(fmaf(a, s.x, acc.x), fmaf(a, s.y, acc.y), fmaf(a, s.z, acc.z), fmaf(a, s.w, acc.w));

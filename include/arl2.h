@@ -81,6 +81,9 @@ typedef struct {
     int host_staging;      /* nonzero: allocate device staging buffers so that
                               arl2_frame_forward_host can be used             */
     arl2_impl impl;
+    int max_ctas;          /* 0: the tensor-core attention kernel may use every
+                              SM; > 0 caps its persistent grid (co-scheduling
+                              with other work, tests of the split schedule)   */
 } arl2_config;
 
 /* Create a layer on the current device.  Validates cfg, allocates the zeroed

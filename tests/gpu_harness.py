@@ -29,7 +29,7 @@ def err(x, ref) -> float:
 
 def run_and_check(w: workloads.Workload, *, impl: str = "auto", layer: int = 0, frames=None,
                   full_rows=lambda f, p: True, sample_rows: int = 64, seed: int = 0,
-                  device_inputs: bool = False):
+                  device_inputs: bool = False, layer_kw=None):
     """Run frames of workload w on the GPU and on the oracle.
 
     full_rows(frame, pass) selects passes whose every output row is
@@ -38,7 +38,7 @@ def run_and_check(w: workloads.Workload, *, impl: str = "auto", layer: int = 0, 
     the worst output and state errors.
     """
     tol = TOL[w.dtype]
-    lay, (wq, wk, wv) = make_layer(w, layer, impl)
+    lay, (wq, wk, wv) = make_layer(w, layer, impl, **(layer_kw or {}))
     rng = np.random.default_rng(seed)
     S_ref = oracle.zero_state(w.batch, w.heads, w.head_dim)
     worst_o = worst_s = 0.0

@@ -50,7 +50,7 @@ def test_null_arguments_are_rejected_before_any_cuda_call():
     lib = arl2._lib
     h = ctypes.c_void_p()
     assert lib.arl2_create(None, None, ctypes.byref(h)) == -1
-    cfg = arl2.Arl2Config(1, 1, 16, 16, 1, None, None, None, 0.0, 0, 0)
+    cfg = arl2.Arl2Config(1, 1, 16, 16, 1, None, None, None, 0.0, 0, 0, 0)
     assert lib.arl2_create(ctypes.byref(cfg), None, None) == -1
     assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1  # null weights
     assert lib.arl2_frame_forward(None, None, None, None, None, None, 0, None, None) == -1
@@ -69,13 +69,13 @@ def test_shape_and_alignment_checks_come_before_cuda():
     h = ctypes.c_void_p()
     fake = 0x1000  # never dereferenced: validation fails first
     for bad in [(0, 1, 16, 16), (1, 0, 16, 16), (1, 1, 0, 16), (1, 1, 129, 16), (1, 1, 16, 0)]:
-        cfg = arl2.Arl2Config(*bad, 1, fake, fake, fake, 0.0, 0, 0)
+        cfg = arl2.Arl2Config(*bad, 1, fake, fake, fake, 0.0, 0, 0, 0)
         assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -2
-    cfg = arl2.Arl2Config(1, 1, 16, 16, 1, fake + 4, fake, fake, 0.0, 0, 0)
+    cfg = arl2.Arl2Config(1, 1, 16, 16, 1, fake + 4, fake, fake, 0.0, 0, 0, 0)
     assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -3
-    cfg = arl2.Arl2Config(1, 1, 64, 16, 0, fake, fake, fake, 0.0, 0, 0)  # bf16 tensor cores need d=128
+    cfg = arl2.Arl2Config(1, 1, 64, 16, 0, fake, fake, fake, 0.0, 0, 0, 0)  # bf16 tensor cores need d=128
     assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -7
-    cfg = arl2.Arl2Config(1, 1, 16, 16, 7, fake, fake, fake, 0.0, 0, 0)  # bad dtype
+    cfg = arl2.Arl2Config(1, 1, 16, 16, 7, fake, fake, fake, 0.0, 0, 0, 0)  # bad dtype
     assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1
     cfg = arl2.Arl2Config(1, 1, 16, 16, 1, fake, fake, fake, -1.0, 0, 0)  # bad scale
     assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1

@@ -31,6 +31,26 @@ def test_tc_stream_matches_oracle_everywhere(L):
     run_and_check(small(L))
 
 
+@pytest.mark.parametrize("L,max_ctas", [(129, 3), (129, 7), (515, 3), (515, 7), (515, 19), (700, 5)])
+def test_split_tile_schedule_matches_oracle(L, max_ctas):
+    # More tiles than CTAs: the persistent schedule cuts tiles into a head
+    # and a tail piece on different CTAs and merges them.
+    run_and_check(small(L, B=2, H=2, frames=2), layer_kw={"max_ctas": max_ctas})
+
+
+def test_split_schedule_repeats_bit_exactly():
+    w = small(515, B=2, H=2)
+    lay, _ = make_layer(w, max_ctas=7)
+    try:
+        q, k, v, a, b = _inputs(w)
+        o1 = lay.forward(q, k, v).clone()
+        for _ in range(3):
+            assert torch.equal(lay.forward(q, k, v), o1)
+        assert lay.device_status() == 0
+    finally:
+        lay.close()
+
+
 def _inputs(w, f=0, p=0):
     q, k, v = workloads.pass_inputs(w, 0, f, p)
     a, b = workloads.frame_gates(w, 0, f)

