@@ -60,7 +60,7 @@ constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per block
 constexpr int kD = 128;   // head dim
 constexpr int kThreads = 384;
-constexpr int kSoftmaxThreads = 256;
+constexpr int kSoftmaxWarps = 8;  // arrivals on the softmax barriers: one per warp
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256, kColOi = 384;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
@@ -128,12 +128,12 @@ struct __align__(1024) Smem {
     uint64_t k_full[2], k_empty[2];
     uint64_t v_full[2], v_empty[2];
     uint64_t s_full[2];
-    uint64_t p_full;    // 256 arrivals per key block: P written (and O rescaled)
+    uint64_t p_full;    // 8 warp arrivals per key block: P written (and O rescaled)
     uint64_t o_ready;   // one commit per key block: that block's P V is done
     uint64_t seg_done;  // one commit per segment: its last UMMA is done
-    uint64_t o_free;    // 256 arrivals per segment: O and O_inter read out
-    uint64_t xch[2];    // 256 arrivals: row maxima of a key block exchanged
-    uint64_t ebar;      // 256 arrivals: epilogue exchanges
+    uint64_t o_free;    // 8 warp arrivals per segment: O and O_inter read out
+    uint64_t xch[2];    // 8 warp arrivals: row maxima of a key block exchanged
+    uint64_t ebar;      // 8 warp arrivals: epilogue exchanges
     float red_max[2][2][kBM];  // [block parity][warpgroup][row]
     float red_sum[2][kBM];     // [warpgroup][row]
     uint32_t tmem_base;
@@ -170,13 +170,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(ptx::smem_u32(&sm.v_empty[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sm.s_full[s]), 1);
         }
-        ptx::mbar_init(ptx::smem_u32(&sm.p_full), kSoftmaxThreads);
+        ptx::mbar_init(ptx::smem_u32(&sm.p_full), kSoftmaxWarps);
         ptx::mbar_init(ptx::smem_u32(&sm.o_ready), 1);
         ptx::mbar_init(ptx::smem_u32(&sm.seg_done), 1);
-        ptx::mbar_init(ptx::smem_u32(&sm.o_free), kSoftmaxThreads);
-        ptx::mbar_init(ptx::smem_u32(&sm.xch[0]), kSoftmaxThreads);
-        ptx::mbar_init(ptx::smem_u32(&sm.xch[1]), kSoftmaxThreads);
-        ptx::mbar_init(ptx::smem_u32(&sm.ebar), kSoftmaxThreads);
+        ptx::mbar_init(ptx::smem_u32(&sm.o_free), kSoftmaxWarps);
+        ptx::mbar_init(ptx::smem_u32(&sm.xch[0]), kSoftmaxWarps);
+        ptx::mbar_init(ptx::smem_u32(&sm.xch[1]), kSoftmaxWarps);
+        ptx::mbar_init(ptx::smem_u32(&sm.ebar), kSoftmaxWarps);
         sm.abort = 0;
         ptx::fence_mbar_init();
         ptx::fence_proxy_async_smem();
@@ -351,9 +351,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         int g = 0;
         uint32_t e_uses = 0;  // completed uses of ebar
         bool ok = true;
-        // all 256 softmax threads meet at bar (arrive, then a bounded wait)
+        // One arrival per warp on the softmax barriers: the warp's lanes
+        // are synchronised (and their shared-memory writes ordered) by
+        // __syncwarp, then lane 0 arrives.
+        auto warp_arrive = [&](uint64_t* bar) {
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(bar));
+        };
+        // all 8 softmax warps meet at bar (arrive, then a bounded wait)
         auto meet = [&](uint64_t* bar, uint32_t parity) -> bool {
-            ptx::mbar_arrive(ptx::smem_u32(bar));
+            warp_arrive(bar);
             return __all_sync(0xffffffffu, bwait(bar, parity));
         };
         auto meet_e = [&]() -> bool { return meet(&sm.ebar, (e_uses++) & 1); };
@@ -433,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(ptx::smem_u32(&sm.p_full));
+                warp_arrive(&sm.p_full);
             }
             if (!ok) break;
             // ------------------------------------------------ epilogue --
@@ -537,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             ptx::tc_fence_before();
-            ptx::mbar_arrive(ptx::smem_u32(&sm.o_free));
+            warp_arrive(&sm.o_free);
             g += n;
         }
         if (!ok) fail();
