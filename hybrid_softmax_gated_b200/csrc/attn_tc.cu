@@ -38,7 +38,10 @@
 // [384,512) O_inter, fp32 (P: bf16 pairs packed over its S buffer).
 // Online softmax with lazy rescaling: the running row max only moves when
 // it grows by more than 2^8; the final 1/l uses the same max as the
-// numerator, so the result is exact up to rounding.
+// numerator, so the result is exact up to rounding.  One exponential in
+// three runs on the FMA pipe (exp2_fma) to balance it against the SFU.
+// Outputs leave through a TMA store staged in the segment's Q slot; split
+// partials are stored so that a warp's lanes write consecutive 16 bytes.
 #include "attn_tc.h"
 #include "ptx.cuh"
 
@@ -134,6 +137,7 @@ struct __align__(1024) Smem {
     uint64_t o_free;    // 8 warp arrivals per segment: O and O_inter read out
     uint64_t xch[2];    // 8 warp arrivals: row maxima of a key block exchanged
     uint64_t ebar;      // 8 warp arrivals: epilogue exchanges
+    uint64_t stage_free[2];  // 1 arrival per segment: the Q slot used as output staging is free
     float red_max[2][2][kBM];  // [block parity][warpgroup][row]
     float red_sum[2][kBM];     // [warpgroup][row]
     uint32_t tmem_base;
@@ -149,7 +153,7 @@ __device__ __forceinline__ int valid_keys(int L, int kv) {
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_m,
-                   __nv_bfloat16* __restrict__ out, float* __restrict__ part_o,
+                   const __grid_constant__ CUtensorMap tm_o, float* __restrict__ part_o,
                    float* __restrict__ part_ml, int* __restrict__ flags, int L, int H, Sched sch,
                    float scale_log2, int* err) {
     extern __shared__ uint8_t smem_raw[];
@@ -177,6 +181,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_init(ptx::smem_u32(&sm.xch[0]), kSoftmaxWarps);
         ptx::mbar_init(ptx::smem_u32(&sm.xch[1]), kSoftmaxWarps);
         ptx::mbar_init(ptx::smem_u32(&sm.ebar), kSoftmaxWarps);
+        ptx::mbar_init(ptx::smem_u32(&sm.stage_free[0]), 1);
+        ptx::mbar_init(ptx::smem_u32(&sm.stage_free[1]), 1);
         sm.abort = 0;
         ptx::fence_mbar_init();
         ptx::fence_proxy_async_smem();
@@ -237,7 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int bh = sg.tile / sch.n_q, qt = sg.tile - bh * sch.n_q;
             const int b = bh / H, h = bh - b * H;
             const int qs = si & 1;
-            if (si >= 2 && !bwait(&sm.q_empty[qs], ((si >> 1) - 1) & 1)) {
+            // the slot's previous Q is consumed and its output staging stored
+            if (si >= 2 && !(bwait(&sm.q_empty[qs], ((si >> 1) - 1) & 1) &&
+                             bwait(&sm.stage_free[qs], ((si >> 1) - 1) & 1))) {
                 ok = false;
                 break;
             }
@@ -411,8 +419,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t pk[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const float p0 = ptx::ex2(fmaf(x[2 * i], scale_log2, neg_m));
-                    const float p1 = ptx::ex2(fmaf(x[2 * i + 1], scale_log2, neg_m));
+                    // every third exponential on the FMA pipe, the rest on the SFU
+                    const float a0 = fmaf(x[2 * i], scale_log2, neg_m);
+                    const float a1 = fmaf(x[2 * i + 1], scale_log2, neg_m);
+                    const float p0 = ((2 * i) % 3 == 2) ? ptx::exp2_fma(a0) : ptx::ex2(a0);
+                    const float p1 = ((2 * i + 1) % 3 == 2) ? ptx::exp2_fma(a1) : ptx::ex2(a1);
                     sum4[i & 3] += p0 + p1;
                     pk[i] = ptx::pack_bf16x2(p0, p1);
                 }
@@ -453,8 +464,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_after();
             const int bh = sg.tile / sch.n_q, qt = sg.tile - bh * sch.n_q;
             const int b = bh / H, h = bh - b * H;
-            const int t = qt * kBM + row;
-            float* prow = part_o + ((size_t)sg.tile * kBM + row) * kD + col0;
+            // partial of (tile, warpgroup): float4 chunk i of row r at [i][r], so
+            // that the 32 lanes of a warp touch 512 consecutive bytes
+            float4* pbase = reinterpret_cast<float4*>(part_o) + ((size_t)sg.tile * 2 + wg) * 16 * kBM + row;
             if (sg.kind == kHead) {
                 // unnormalised O, running max and row sum -> partial, then the flag
 #pragma unroll
@@ -463,11 +475,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tmem_ld32(tmem + lane_base + kColO + col0 + (uint32_t)c * 32, o);
                     ptx::tmem_wait_ld();
                     ptx::reg_fence(o);
-                    float4* dst = reinterpret_cast<float4*>(prow + c * 32);
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
-                        dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                             __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+                        pbase[(size_t)(c * 8 + i) * kBM] =
+                            make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                        __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
                 }
                 if (wg == 0)
                     *reinterpret_cast<float2*>(part_ml + ((size_t)sg.tile * kBM + row) * 2) =
@@ -475,7 +487,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __threadfence();
                 ok = meet_e();
                 if (!ok) break;
-                if (threadIdx.x == 128) ptx::st_release_gpu(flags + sg.tile, 1);
+                if (threadIdx.x == 128) {
+                    ptx::st_release_gpu(flags + sg.tile, 1);
+                    ptx::mbar_arrive(ptx::smem_u32(&sm.stage_free[si & 1]));  // staging unused
+                }
             } else {
                 float a_t = 1.f, a_h = 0.f, inv_l = 1.f / l_row;
                 if (sg.kind == kTail) {
@@ -499,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     a_t = ptx::ex2(m_run - mm);
                     inv_l = 1.f / (a_h * ml.y + a_t * l_row);
                 }
-                __nv_bfloat16* orow = out + (((size_t)b * L + t) * H + h) * kD + col0;
+                const uint32_t stage = ptx::smem_u32(sm.q[si & 1]);  // the segment's Q slot
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     uint32_t o[32], oi[32];
@@ -512,35 +527,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 32; ++i) acc[i] = a_t * __uint_as_float(o[i]);
                     if (sg.kind == kTail) {
-                        const float4* src = reinterpret_cast<const float4*>(prow + c * 32);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            const float4 ph = __ldcg(src + i);
+                            const float4 ph = __ldcg(pbase + (size_t)(c * 8 + i) * kBM);
                             acc[4 * i] = fmaf(a_h, ph.x, acc[4 * i]);
                             acc[4 * i + 1] = fmaf(a_h, ph.y, acc[4 * i + 1]);
                             acc[4 * i + 2] = fmaf(a_h, ph.z, acc[4 * i + 2]);
                             acc[4 * i + 3] = fmaf(a_h, ph.w, acc[4 * i + 3]);
                         }
                     }
-                    if (t < L) {
+                    // bf16 output row chunk -> the staging tile (128-byte swizzle)
 #pragma unroll
-                        for (int gq = 0; gq < 4; ++gq) {
-                            uint32_t w[4];
+                    for (int gq = 0; gq < 4; ++gq) {
+                        uint32_t w[4];
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int i = gq * 8 + e * 2;
-                                w[e] = ptx::pack_bf16x2(fmaf(acc[i], inv_l, __uint_as_float(oi[i])),
-                                                        fmaf(acc[i + 1], inv_l, __uint_as_float(oi[i + 1])));
-                            }
-                            *reinterpret_cast<uint4*>(orow + c * 32 + gq * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+                        for (int e = 0; e < 4; ++e) {
+                            const int i = gq * 8 + e * 2;
+                            w[e] = ptx::pack_bf16x2(fmaf(acc[i], inv_l, __uint_as_float(oi[i])),
+                                                    fmaf(acc[i + 1], inv_l, __uint_as_float(oi[i + 1])));
                         }
+                        ptx::st_shared_v4(stage + ptx::tile_chunk_offset(row, wg * 8 + c * 4 + gq), w[0], w[1],
+                                          w[2], w[3]);
                     }
                 }
-                if (sg.kind == kTail) {
-                    // every thread has read the partial: clear the flag for the next launch
-                    ok = meet_e();
-                    if (!ok) break;
-                    if (threadIdx.x == 128) flags[sg.tile] = 0;
+                ptx::fence_proxy_async_smem();
+                // every thread has staged its row (and read the partial)
+                ok = meet_e();
+                if (!ok) break;
+                if (threadIdx.x == 128) {
+                    if (sg.kind == kTail) flags[sg.tile] = 0;  // clear for the next launch
+                    ptx::tma_store_4d(&tm_o, stage, 0, h, qt * kBM, b);
+                    ptx::tma_store_4d(&tm_o, stage + kHalfBytes, 64, h, qt * kBM, b);
+                    ptx::bulk_commit_group();
+                    ptx::bulk_wait_group_read0();
+                    ptx::mbar_arrive(ptx::smem_u32(&sm.stage_free[si & 1]));
                 }
             }
             ptx::tc_fence_before();
@@ -624,9 +644,9 @@ cudaError_t attn_tc_launch(AttnTc* t, TokenMapCache& maps, const void* q, const 
         if (!tma_encode_tiles(&t->tm_m, Mt, dm.B * dm.H)) return cudaErrorInvalidValue;
         t->m_ptr = Mt;
     }
-    CUtensorMap cq, ck, cv;
-    if (!maps.get(q, &cq) || !maps.get(k, &ck) || !maps.get(v, &cv)) return cudaErrorInvalidValue;
-    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+    CUtensorMap cq, ck, cv, co;
+    if (!maps.get(q, &cq) || !maps.get(k, &ck) || !maps.get(v, &cv) || !maps.get(out, &co))
+        return cudaErrorInvalidValue;
     const float sl2 = scale * 1.4426950408889634f;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(t->sch.G, 1, 1);
@@ -638,7 +658,7 @@ cudaError_t attn_tc_launch(AttnTc* t, TokenMapCache& maps, const void* q, const 
     attr[0].val.cooperative = t->sch.split ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, attn_tc_kernel, cq, ck, cv, t->tm_m, o, t->part_o, t->part_ml,
+    return cudaLaunchKernelEx(&cfg, attn_tc_kernel, cq, ck, cv, t->tm_m, co, t->part_o, t->part_ml,
                               t->flags, dm.L, dm.H, t->sch, sl2, err);
 }
 

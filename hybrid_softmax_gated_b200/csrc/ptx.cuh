@@ -88,6 +88,24 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* m, 
         : "memory");
 }
 
+// 4-D tiled store from this CTA's shared memory (bulk async-group).  Rows
+// outside the tensor are not written.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* m, uint32_t src, int c0, int c1,
+                                             int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(m)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until every committed bulk store has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // ---- tcgen05: TMEM allocation ---------------------------------------------
 // Whole warp.  Writes the allocated TMEM base address to shared memory.
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
@@ -204,6 +222,23 @@ __device__ __forceinline__ void st_release_gpu(int* p, int v) {
 }
 
 // ---- math -----------------------------------------------------------------
+// 2^x on the FMA and integer pipes instead of the SFU: Cody-Waite style
+// reduction x = n + f, n = rint(x), f in [-1/2, 1/2], and 2^x = 2^n P(f)
+// with P the degree-3 polynomial fitted by fit_exp2_poly.py (relative error
+// below 1e-4).  Inputs are clamped to >= -126 so that 2^n stays a normal
+// scale; results below 2^-126 are not needed by the softmax.
+__device__ __forceinline__ float exp2_fma(float x) {
+    constexpr float kRound = 12582912.f;  // 1.5 * 2^23: x + kRound holds rint(x)
+    x = fmaxf(x, -126.f);
+    const float t = x + kRound;
+    const float f = x - (t - kRound);
+    float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
+    p = fmaf(p, f, 0.6932609677314758f);
+    p = fmaf(p, f, 0.9999280571937561f);
+    const int n = __float_as_int(t) - 0x4B400000;  // rint(x)
+    return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
