@@ -26,16 +26,19 @@
 // One CTA, 384 threads:
 //   warp 0       TMA producer: Q tiles (2 slots), K and V blocks (2-stage
 //                rings), the (W_q S)^T tile through the K ring
-//   warp 1       UMMA issuer (one thread): S = Q K^T into TMEM (two
-//                buffers), O += P V with P read from TMEM, O_inter = Q M
+//   warp 1       UMMA issuer (one thread): S = Q K^T into TMEM (three
+//                buffers, up to three key blocks ahead), O += P V with P
+//                read from TMEM, O_inter = Q M into the next free buffer
 //   warp 2       TMEM allocator
 //   warps 4-7    softmax warpgroup 0: keys 0-63 of each block, O cols 0-63
 //   warps 8-11   softmax warpgroup 1: keys 64-127, O cols 64-127
 // Row r of a tile is TMEM lane r; both warpgroups own row r (lane quadrant
 // = warp % 4) and exchange row maxima and sums through shared memory,
 // synchronised by mbarriers (bounded waits, unlike bar.sync).
-// TMEM columns: [0,128) S/P buffer 0, [128,256) S/P buffer 1, [256,384) O,
-// [384,512) O_inter, fp32 (P: bf16 pairs packed over its S buffer).
+// TMEM columns: [0,384) three S/P buffers, [384,512) O, fp32 (P: bf16
+// pairs packed over its S buffer).  Buffers rotate over "virtual blocks":
+// each key block of a segment, then (for a segment that finishes its tile)
+// one more for O_inter, read by the epilogue.
 // Online softmax with lazy rescaling: the running row max only moves when
 // it grows by more than 2^8; the final 1/l uses the same max as the
 // numerator, so the result is exact up to rounding.  One exponential in
@@ -65,7 +68,8 @@ constexpr int kD = 128;   // head dim
 constexpr int kThreads = 384;
 constexpr int kSoftmaxWarps = 8;  // arrivals on the softmax barriers: one per warp
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256, kColOi = 384;
+constexpr uint32_t kColS = 0, kColO = 384;  // S/P buffers at 0, 128, 256
+constexpr int kSBufs = 3;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -130,7 +134,7 @@ struct __align__(1024) Smem {
     uint64_t q_full[2], q_empty[2];
     uint64_t k_full[2], k_empty[2];
     uint64_t v_full[2], v_empty[2];
-    uint64_t s_full[2];
+    uint64_t s_full[kSBufs];
     uint64_t p_full;    // 8 warp arrivals per key block: P written (and O rescaled)
     uint64_t o_ready;   // one commit per key block: that block's P V is done
     uint64_t seg_done;  // one commit per segment: its last UMMA is done
@@ -172,8 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(ptx::smem_u32(&sm.k_empty[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sm.v_full[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sm.v_empty[s]), 1);
-            ptx::mbar_init(ptx::smem_u32(&sm.s_full[s]), 1);
         }
+        for (int s = 0; s < kSBufs; ++s) ptx::mbar_init(ptx::smem_u32(&sm.s_full[s]), 1);
         ptx::mbar_init(ptx::smem_u32(&sm.p_full), kSoftmaxWarps);
         ptx::mbar_init(ptx::smem_u32(&sm.o_ready), 1);
         ptx::mbar_init(ptx::smem_u32(&sm.seg_done), 1);
@@ -254,12 +258,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tma_load_4d(qdst, &tm_q, 0, h, qt * kBM, b, qbar);
             ptx::tma_load_4d(qdst + kHalfBytes, &tm_q, 64, h, qt * kBM, b, qbar);
             // K and V in the order the issuer consumes them:
-            // K0 K1 V0 K2 V1 ... V_{n-1} [M]
+            // K0 K1 K2 V0 K3 V1 ... V_{n-1} [M]
             const int n = sg.kv1 - sg.kv0;
-            ok = load_k(b, h, sg.kv0) && (n < 2 || load_k(b, h, sg.kv0 + 1));
+            for (int j = 0; ok && j < 3 && j < n; ++j) ok = load_k(b, h, sg.kv0 + j);
             for (int j = 0; ok && j < n; ++j) {
                 ok = load_v(b, h, sg.kv0 + j);
-                if (ok && j + 2 < n) ok = load_k(b, h, sg.kv0 + j + 2);
+                if (ok && j + 3 < n) ok = load_k(b, h, sg.kv0 + j + 3);
             }
             if (ok && sg.kind != kHead) ok = load_k(b, h, -1);
         }
@@ -275,25 +279,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------- UMMA issuer --
         constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBM, kD, false, true);
         constexpr uint32_t idesc_qm = ptx::idesc_bf16_f32(kBM, kD, false, false);
-        int kc = 0, vc = 0, g = 0;
+        int kc = 0, vc = 0;
+        int rb = 0;  // key blocks issued so far (all segments)
+        int vb = 0;  // virtual blocks so far: buffer of the next one is vb % 3
         bool ok = true;
-        auto issue_qk = [&](uint32_t q_s, int blk, int kv) -> bool {  // S_blk = Q K^T
+        auto issue_qk = [&](uint32_t q_s, int buf, int kv) -> bool {  // S = Q K^T into buffer buf
             const int s = kc & 1;
             if (!bwait(&sm.k_full[s], (kc >> 1) & 1)) return false;
             ptx::tc_fence_after();
             const int valid = valid_keys(L, kv);
             const uint32_t idesc = ptx::idesc_bf16_f32(kBM, (valid + 15) & ~15, false, false);
             const uint32_t k_s = ptx::smem_u32(sm.k[s]);
-            const uint32_t d = tmem + kColS + (uint32_t)(blk & 1) * kBN;
+            const uint32_t d = tmem + kColS + (uint32_t)buf * kBN;
 #pragma unroll
             for (int kk = 0; kk < kD / 16; ++kk)
                 ptx::umma_f16_ss(d, kmajor_desc(q_s, kk), kmajor_desc(k_s, kk), idesc, kk > 0);
-            ptx::umma_commit(ptx::smem_u32(&sm.s_full[blk & 1]));
+            ptx::umma_commit(ptx::smem_u32(&sm.s_full[buf]));
             ptx::umma_commit(ptx::smem_u32(&sm.k_empty[s]));
             ++kc;
             return true;
         };
         int si = 0;
+        int prev_oi_buf = -1;  // buffer holding the previous segment's O_inter
         for (; ok && si < rng.n_segs; ++si) {
             const Seg sg = seg_at(sch, rng, si);
             const int qs = si & 1;
@@ -303,18 +310,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             const uint32_t q_s = ptx::smem_u32(sm.q[qs]);
-            // S buffers are free: the P V that last read each was issued before.
-            ok = issue_qk(q_s, g, sg.kv0) && (n < 2 || issue_qk(q_s, g + 1, sg.kv0 + 1));
-            // O and O_inter of the previous segment have been read out.
-            if (ok && si >= 1) ok = bwait(&sm.o_free, (si - 1) & 1);
+            // Up to three blocks ahead.  A buffer last used by a key block is
+            // free (its P V was issued before); the buffer with the previous
+            // segment's O_inter, and O itself, are free once the epilogue of
+            // that segment has read them (o_free).
+            bool freed = si == 0;
+            for (int j = 0; ok && j < 3 && j < n; ++j) {
+                const int buf = (vb + j) % kSBufs;
+                if (!freed && buf == prev_oi_buf) {
+                    ok = bwait(&sm.o_free, (si - 1) & 1);
+                    freed = true;
+                }
+                if (ok) ok = issue_qk(q_s, buf, sg.kv0 + j);
+            }
+            if (ok && !freed) ok = bwait(&sm.o_free, (si - 1) & 1);
             for (int j = 0; ok && j < n; ++j) {
-                const int blk = g + j;
+                const int buf = (vb + j) % kSBufs;
                 const int vs = vc & 1;
-                ok = bwait(&sm.p_full, blk & 1) && bwait(&sm.v_full[vs], (vc >> 1) & 1);
+                ok = bwait(&sm.p_full, rb & 1) && bwait(&sm.v_full[vs], (vc >> 1) & 1);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 const int ksteps = (valid_keys(L, sg.kv0 + j) + 15) >> 4;
-                const uint32_t p_t = tmem + kColS + (uint32_t)(blk & 1) * kBN;
+                const uint32_t p_t = tmem + kColS + (uint32_t)buf * kBN;
                 const uint32_t v_s = ptx::smem_u32(sm.v[vs]);
                 for (int kk = 0; kk < ksteps; ++kk)  // O += P V, P from TMEM
                     ptx::umma_f16_ts(tmem + kColO, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv,
@@ -322,10 +339,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::umma_commit(ptx::smem_u32(&sm.v_empty[vs]));
                 ptx::umma_commit(ptx::smem_u32(&sm.o_ready));
                 ++vc;
+                ++rb;
                 // The next QK into this S/P buffer follows the P V that reads it.
-                if (j + 2 < n) ok = issue_qk(q_s, blk + 2, sg.kv0 + j + 2);
+                if (j + 3 < n) ok = issue_qk(q_s, buf, sg.kv0 + j + 3);
             }
+            prev_oi_buf = -1;
             if (ok && sg.kind != kHead) {
+                const int buf = (vb + n) % kSBufs;
                 const int s = kc & 1;
                 ok = bwait(&sm.k_full[s], (kc >> 1) & 1);
                 if (ok) {
@@ -333,16 +353,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t m_s = ptx::smem_u32(sm.k[s]);
 #pragma unroll
                     for (int kk = 0; kk < kD / 16; ++kk)  // O_inter = Q (W_q S)
-                        ptx::umma_f16_ss(tmem + kColOi, kmajor_desc(q_s, kk), kmajor_desc(m_s, kk), idesc_qm,
-                                         kk > 0);
+                        ptx::umma_f16_ss(tmem + kColS + (uint32_t)buf * kBN, kmajor_desc(q_s, kk),
+                                         kmajor_desc(m_s, kk), idesc_qm, kk > 0);
                     ptx::umma_commit(ptx::smem_u32(&sm.k_empty[s]));
                     ++kc;
+                    prev_oi_buf = buf;
                 }
             }
             if (!ok) break;
             ptx::umma_commit(ptx::smem_u32(&sm.q_empty[qs]));
             ptx::umma_commit(ptx::smem_u32(&sm.seg_done));
-            g += n;
+            vb += n + (sg.kind != kHead ? 1 : 0);
         }
         if (!ok) {
             fail();
@@ -356,7 +377,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = ((warp & 3) << 5) + lane;     // tile row = TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t col0 = (uint32_t)wg * 64;
-        int g = 0;
+        int rb = 0;                  // key blocks processed so far (all segments)
+        int vb = 0;                  // virtual blocks so far (see the issuer)
+        uint32_t s_par = 0;          // bit b: phase parity of s_full[b] to wait for
         uint32_t e_uses = 0;  // completed uses of ebar
         bool ok = true;
         // One arrival per warp on the softmax barriers: the warp's lanes
@@ -377,9 +400,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n = sg.kv1 - sg.kv0;
             float m_run = -INFINITY, l_part = 0.f;
             for (int j = 0; j < n; ++j) {
-                const int blk = g + j;
-                const uint32_t sbuf = tmem + lane_base + kColS + (uint32_t)(blk & 1) * kBN;
-                ok = __all_sync(0xffffffffu, bwait(&sm.s_full[blk & 1], (blk >> 1) & 1));
+                const int blk = rb + j;
+                const int buf = (vb + j) % kSBufs;
+                const uint32_t sbuf = tmem + lane_base + kColS + (uint32_t)buf * kBN;
+                ok = __all_sync(0xffffffffu, bwait(&sm.s_full[buf], (s_par >> buf) & 1));
+                s_par ^= 1u << buf;
                 if (!ok) break;
                 ptx::tc_fence_after();
                 uint32_t raw[2][32];
@@ -519,7 +544,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < 2; ++c) {
                     uint32_t o[32], oi[32];
                     ptx::tmem_ld32(tmem + lane_base + kColO + col0 + (uint32_t)c * 32, o);
-                    ptx::tmem_ld32(tmem + lane_base + kColOi + col0 + (uint32_t)c * 32, oi);
+                    ptx::tmem_ld32(tmem + lane_base + kColS + (uint32_t)((vb + n) % kSBufs) * kBN + col0 +
+                                       (uint32_t)c * 32,
+                                   oi);
                     ptx::tmem_wait_ld();
                     ptx::reg_fence(o);
                     ptx::reg_fence(oi);
@@ -565,7 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ptx::tc_fence_before();
             warp_arrive(&sm.o_free);
-            g += n;
+            rb += n;
+            vb += n + (sg.kind != kHead ? 1 : 0);
         }
         if (!ok) fail();
     }
