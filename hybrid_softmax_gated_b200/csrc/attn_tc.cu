@@ -135,8 +135,10 @@ struct __align__(1024) Smem {
     uint64_t k_full[2], k_empty[2];
     uint64_t v_full[2], v_empty[2];
     uint64_t s_full[kSBufs];
-    uint64_t p_full;    // 8 warp arrivals per key block: P written (and O rescaled)
-    uint64_t o_ready;   // one commit per key block: that block's P V is done
+    // Per S/P buffer: a buffer's next use needs the P V of its previous
+    // use issued, so these never run more than one phase ahead of a waiter.
+    uint64_t p_full[kSBufs];   // 8 warp arrivals: P of the buffer's block written (and O rescaled)
+    uint64_t o_ready[kSBufs];  // one commit: the P V reading the buffer is done
     uint64_t seg_done;  // one commit per segment: its last UMMA is done
     uint64_t o_free;    // 8 warp arrivals per segment: O and O_inter read out
     uint64_t xch[2];    // 8 warp arrivals: row maxima of a key block exchanged
@@ -177,9 +179,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(ptx::smem_u32(&sm.v_full[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sm.v_empty[s]), 1);
         }
-        for (int s = 0; s < kSBufs; ++s) ptx::mbar_init(ptx::smem_u32(&sm.s_full[s]), 1);
-        ptx::mbar_init(ptx::smem_u32(&sm.p_full), kSoftmaxWarps);
-        ptx::mbar_init(ptx::smem_u32(&sm.o_ready), 1);
+        for (int s = 0; s < kSBufs; ++s) {
+            ptx::mbar_init(ptx::smem_u32(&sm.s_full[s]), 1);
+            ptx::mbar_init(ptx::smem_u32(&sm.p_full[s]), kSoftmaxWarps);
+            ptx::mbar_init(ptx::smem_u32(&sm.o_ready[s]), 1);
+        }
         ptx::mbar_init(ptx::smem_u32(&sm.seg_done), 1);
         ptx::mbar_init(ptx::smem_u32(&sm.o_free), kSoftmaxWarps);
         ptx::mbar_init(ptx::smem_u32(&sm.xch[0]), kSoftmaxWarps);
@@ -280,8 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBM, kD, false, true);
         constexpr uint32_t idesc_qm = ptx::idesc_bf16_f32(kBM, kD, false, false);
         int kc = 0, vc = 0;
-        int rb = 0;  // key blocks issued so far (all segments)
-        int vb = 0;  // virtual blocks so far: buffer of the next one is vb % 3
+        int vb = 0;           // virtual blocks so far: buffer of the next one is vb % 3
+        uint32_t p_par = 0;   // bit b: phase parity of p_full[b] to wait for
         bool ok = true;
         auto issue_qk = [&](uint32_t q_s, int buf, int kv) -> bool {  // S = Q K^T into buffer buf
             const int s = kc & 1;
@@ -327,7 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; ok && j < n; ++j) {
                 const int buf = (vb + j) % kSBufs;
                 const int vs = vc & 1;
-                ok = bwait(&sm.p_full, rb & 1) && bwait(&sm.v_full[vs], (vc >> 1) & 1);
+                ok = bwait(&sm.p_full[buf], (p_par >> buf) & 1) && bwait(&sm.v_full[vs], (vc >> 1) & 1);
+                p_par ^= 1u << buf;
                 if (!ok) break;
                 ptx::tc_fence_after();
                 const int ksteps = (valid_keys(L, sg.kv0 + j) + 15) >> 4;
@@ -337,9 +342,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::umma_f16_ts(tmem + kColO, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv,
                                      (j > 0 || kk > 0) ? 1u : 0u);
                 ptx::umma_commit(ptx::smem_u32(&sm.v_empty[vs]));
-                ptx::umma_commit(ptx::smem_u32(&sm.o_ready));
+                ptx::umma_commit(ptx::smem_u32(&sm.o_ready[buf]));
                 ++vc;
-                ++rb;
                 // The next QK into this S/P buffer follows the P V that reads it.
                 if (j + 3 < n) ok = issue_qk(q_s, buf, sg.kv0 + j + 3);
             }
@@ -380,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int rb = 0;                  // key blocks processed so far (all segments)
         int vb = 0;                  // virtual blocks so far (see the issuer)
         uint32_t s_par = 0;          // bit b: phase parity of s_full[b] to wait for
+        uint32_t o_par = 0;          // bit b: parity of the blocks processed on buffer b
         uint32_t e_uses = 0;  // completed uses of ebar
         bool ok = true;
         // One arrival per warp on the softmax barriers: the warp's lanes
@@ -458,8 +463,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // reading S at the barrier above)
                 ptx::tmem_st32_u(sbuf + (uint32_t)wg * 32, pk);
                 if (j >= 1 && __any_sync(0xffffffffu, need)) {
-                    // rescale my half of O once the previous P V is done
-                    ok = __all_sync(0xffffffffu, bwait(&sm.o_ready, (blk - 1) & 1));
+                    // rescale my half of O once the previous block's P V is done
+                    // (its commit is the latest on that buffer)
+                    const int pb = (vb + j - 1) % kSBufs;
+                    ok = __all_sync(0xffffffffu, bwait(&sm.o_ready[pb], ((o_par >> pb) & 1) ^ 1));
                     if (!ok) break;
                     ptx::tc_fence_after();
 #pragma unroll
@@ -476,7 +483,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                warp_arrive(&sm.p_full);
+                warp_arrive(&sm.p_full[buf]);
+                o_par ^= 1u << buf;
             }
             if (!ok) break;
             // ------------------------------------------------ epilogue --
