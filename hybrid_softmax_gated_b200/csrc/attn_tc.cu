@@ -24,12 +24,16 @@
 // two.  Waits are bounded.  With no more tiles than SMs, one CTA per tile.
 //
 // One CTA, 384 threads:
-//   warp 0       TMA producer: Q tiles (2 slots), K and V blocks (2-stage
+//   warp 0       TMA producer (whole warp, one elected lane issues): Q
+//                tiles (2 slots), K and V blocks (2-stage
 //                rings), the (W_q S)^T tile through the K ring
-//   warp 1       UMMA issuer (one thread): S = Q K^T into TMEM (three
+//   warp 1       UMMA issuer (whole warp, one elected lane issues): S = Q K^T into TMEM (three
 //                buffers, up to three key blocks ahead), O += P V with P
 //                read from TMEM, O_inter = Q M into the next free buffer
 //   warp 2       TMEM allocator
+//   warp 3       epilogue helper: publishes head partials (release flag),
+//                acquires the flag of a tail's head partial, issues the TMA
+//                stores of staged outputs
 //   warps 4-7    softmax warpgroup 0: keys 0-63 of each block, O cols 0-63
 //   warps 8-11   softmax warpgroup 1: keys 64-127, O cols 64-127
 // Row r of a tile is TMEM lane r; both warpgroups own row r (lane quadrant
@@ -144,6 +148,10 @@ struct __align__(1024) Smem {
     uint64_t xch[2];    // 8 warp arrivals: row maxima of a key block exchanged
     uint64_t ebar;      // 8 warp arrivals: epilogue exchanges
     uint64_t stage_free[2];  // 1 arrival per segment: the Q slot used as output staging is free
+    uint64_t staged[2];      // 8 warp arrivals per segment (by si & 1): output staged / head
+                             // partial written; a slot's next use needs stage_free, so warp 3
+                             // can never fall two phases behind on one of them
+    uint64_t head_ready;     // 1 arrival: the head partial of this CTA's tail piece is visible
     float red_max[2][2][kBM];  // [block parity][warpgroup][row]
     float red_sum[2][kBM];     // [warpgroup][row]
     uint32_t tmem_base;
@@ -191,6 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_init(ptx::smem_u32(&sm.ebar), kSoftmaxWarps);
         ptx::mbar_init(ptx::smem_u32(&sm.stage_free[0]), 1);
         ptx::mbar_init(ptx::smem_u32(&sm.stage_free[1]), 1);
+        ptx::mbar_init(ptx::smem_u32(&sm.staged[0]), kSoftmaxWarps);
+        ptx::mbar_init(ptx::smem_u32(&sm.staged[1]), kSoftmaxWarps);
+        ptx::mbar_init(ptx::smem_u32(&sm.head_ready), 1);
         sm.abort = 0;
         ptx::fence_mbar_init();
         ptx::fence_proxy_async_smem();
@@ -211,8 +222,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto bwait = [&](uint64_t* bar, uint32_t parity) {
         return ptx::mbar_wait_bounded(ptx::smem_u32(bar), parity, abort, kWaitLimitNs);
     };
+    // bounded wait with a warp-uniform result (for the full-warp roles)
+    auto wwait = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, bwait(bar, parity));
+    };
 
-    if (warp == 0 && lane == 0) {
+    if (warp == 0) {
+        // (the whole warp runs the producer; one elected lane issues)
         // ------------------------------------------------ TMA producer --
         ptx::tma_prefetch_desc(&tm_q);
         ptx::tma_prefetch_desc(&tm_k);
@@ -222,26 +238,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         auto load_k = [&](int b, int h, int kv) -> bool {  // kv < 0: the (W_q S)^T tile
             const int s = kc & 1;
-            if (kc >= 2 && !bwait(&sm.k_empty[s], ((kc >> 1) - 1) & 1)) return false;
+            if (kc >= 2 && !wwait(&sm.k_empty[s], ((kc >> 1) - 1) & 1)) return false;
             const uint32_t bar = ptx::smem_u32(&sm.k_full[s]), dst = ptx::smem_u32(sm.k[s]);
-            ptx::mbar_arrive_expect_tx(bar, kTileBytes);
+            ptx::mbar_arrive_expect_tx_w(bar, kTileBytes);
             if (kv >= 0) {
-                ptx::tma_load_4d(dst, &tm_k, 0, h, kv * kBN, b, bar);
-                ptx::tma_load_4d(dst + kHalfBytes, &tm_k, 64, h, kv * kBN, b, bar);
+                ptx::tma_load_4d_w(dst, &tm_k, 0, h, kv * kBN, b, bar);
+                ptx::tma_load_4d_w(dst + kHalfBytes, &tm_k, 64, h, kv * kBN, b, bar);
             } else {
-                ptx::tma_load_4d(dst, &tm_m, 0, 0, b * H + h, 0, bar);
-                ptx::tma_load_4d(dst + kHalfBytes, &tm_m, 64, 0, b * H + h, 0, bar);
+                ptx::tma_load_4d_w(dst, &tm_m, 0, 0, b * H + h, 0, bar);
+                ptx::tma_load_4d_w(dst + kHalfBytes, &tm_m, 64, 0, b * H + h, 0, bar);
             }
             ++kc;
             return true;
         };
         auto load_v = [&](int b, int h, int kv) -> bool {
             const int s = vc & 1;
-            if (vc >= 2 && !bwait(&sm.v_empty[s], ((vc >> 1) - 1) & 1)) return false;
+            if (vc >= 2 && !wwait(&sm.v_empty[s], ((vc >> 1) - 1) & 1)) return false;
             const uint32_t bar = ptx::smem_u32(&sm.v_full[s]), dst = ptx::smem_u32(sm.v[s]);
-            ptx::mbar_arrive_expect_tx(bar, kTileBytes);
-            ptx::tma_load_4d(dst, &tm_v, 0, h, kv * kBN, b, bar);
-            ptx::tma_load_4d(dst + kHalfBytes, &tm_v, 64, h, kv * kBN, b, bar);
+            ptx::mbar_arrive_expect_tx_w(bar, kTileBytes);
+            ptx::tma_load_4d_w(dst, &tm_v, 0, h, kv * kBN, b, bar);
+            ptx::tma_load_4d_w(dst + kHalfBytes, &tm_v, 64, h, kv * kBN, b, bar);
             ++vc;
             return true;
         };
@@ -252,15 +268,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int b = bh / H, h = bh - b * H;
             const int qs = si & 1;
             // the slot's previous Q is consumed and its output staging stored
-            if (si >= 2 && !(bwait(&sm.q_empty[qs], ((si >> 1) - 1) & 1) &&
-                             bwait(&sm.stage_free[qs], ((si >> 1) - 1) & 1))) {
+            if (si >= 2 && !(wwait(&sm.q_empty[qs], ((si >> 1) - 1) & 1) &&
+                             wwait(&sm.stage_free[qs], ((si >> 1) - 1) & 1))) {
                 ok = false;
                 break;
             }
             const uint32_t qbar = ptx::smem_u32(&sm.q_full[qs]), qdst = ptx::smem_u32(sm.q[qs]);
-            ptx::mbar_arrive_expect_tx(qbar, kTileBytes);
-            ptx::tma_load_4d(qdst, &tm_q, 0, h, qt * kBM, b, qbar);
-            ptx::tma_load_4d(qdst + kHalfBytes, &tm_q, 64, h, qt * kBM, b, qbar);
+            ptx::mbar_arrive_expect_tx_w(qbar, kTileBytes);
+            ptx::tma_load_4d_w(qdst, &tm_q, 0, h, qt * kBM, b, qbar);
+            ptx::tma_load_4d_w(qdst + kHalfBytes, &tm_q, 64, h, qt * kBM, b, qbar);
             // K and V in the order the issuer consumes them:
             // K0 K1 K2 V0 K3 V1 ... V_{n-1} [M]
             const int n = sg.kv1 - sg.kv0;
@@ -279,7 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (i >= 0) ptx::mbar_wait_bounded(ptx::smem_u32(&sm.v_full[i & 1]), (i >> 1) & 1, &no_abort, kWaitLimitNs);
         for (int i = si - 2; i < si; ++i)
             if (i >= 0) ptx::mbar_wait_bounded(ptx::smem_u32(&sm.q_full[i & 1]), (i >> 1) & 1, &no_abort, kWaitLimitNs);
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
+        // (the whole warp runs the issuer; one elected lane issues)
         // ------------------------------------------------- UMMA issuer --
         constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBM, kD, false, true);
         constexpr uint32_t idesc_qm = ptx::idesc_bf16_f32(kBM, kD, false, false);
@@ -289,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         auto issue_qk = [&](uint32_t q_s, int buf, int kv) -> bool {  // S = Q K^T into buffer buf
             const int s = kc & 1;
-            if (!bwait(&sm.k_full[s], (kc >> 1) & 1)) return false;
+            if (!wwait(&sm.k_full[s], (kc >> 1) & 1)) return false;
             ptx::tc_fence_after();
             const int valid = valid_keys(L, kv);
             const uint32_t idesc = ptx::idesc_bf16_f32(kBM, (valid + 15) & ~15, false, false);
@@ -297,9 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t d = tmem + kColS + (uint32_t)buf * kBN;
 #pragma unroll
             for (int kk = 0; kk < kD / 16; ++kk)
-                ptx::umma_f16_ss(d, kmajor_desc(q_s, kk), kmajor_desc(k_s, kk), idesc, kk > 0);
-            ptx::umma_commit(ptx::smem_u32(&sm.s_full[buf]));
-            ptx::umma_commit(ptx::smem_u32(&sm.k_empty[s]));
+                ptx::umma_f16_ss_w(d, kmajor_desc(q_s, kk), kmajor_desc(k_s, kk), idesc, kk > 0);
+            ptx::umma_commit_w(ptx::smem_u32(&sm.s_full[buf]));
+            ptx::umma_commit_w(ptx::smem_u32(&sm.k_empty[s]));
             ++kc;
             return true;
         };
@@ -309,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Seg sg = seg_at(sch, rng, si);
             const int qs = si & 1;
             const int n = sg.kv1 - sg.kv0;
-            if (!bwait(&sm.q_full[qs], (si >> 1) & 1)) {
+            if (!wwait(&sm.q_full[qs], (si >> 1) & 1)) {
                 ok = false;
                 break;
             }
@@ -322,59 +339,113 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; ok && j < 3 && j < n; ++j) {
                 const int buf = (vb + j) % kSBufs;
                 if (!freed && buf == prev_oi_buf) {
-                    ok = bwait(&sm.o_free, (si - 1) & 1);
+                    ok = wwait(&sm.o_free, (si - 1) & 1);
                     freed = true;
                 }
                 if (ok) ok = issue_qk(q_s, buf, sg.kv0 + j);
             }
-            if (ok && !freed) ok = bwait(&sm.o_free, (si - 1) & 1);
+            if (ok && !freed) ok = wwait(&sm.o_free, (si - 1) & 1);
+            // O_inter = Q (W_q S) into buffer (vb + n) % 3, as soon as that
+            // buffer is free: after the P V of block n - 3, or now if n < 3.
+            const int qm_after = sg.kind == kHead ? -2 : (n >= 3 ? n - 3 : -1);
+            auto issue_qm = [&]() -> bool {
+                const int buf = (vb + n) % kSBufs;
+                const int s = kc & 1;
+                if (!wwait(&sm.k_full[s], (kc >> 1) & 1)) return false;
+                ptx::tc_fence_after();
+                const uint32_t m_s = ptx::smem_u32(sm.k[s]);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    ptx::umma_f16_ss_w(tmem + kColS + (uint32_t)buf * kBN, kmajor_desc(q_s, kk),
+                                       kmajor_desc(m_s, kk), idesc_qm, kk > 0);
+                ptx::umma_commit_w(ptx::smem_u32(&sm.k_empty[s]));
+                ++kc;
+                prev_oi_buf = buf;
+                return true;
+            };
+            prev_oi_buf = -1;
+            if (ok && qm_after == -1) ok = issue_qm();
             for (int j = 0; ok && j < n; ++j) {
                 const int buf = (vb + j) % kSBufs;
                 const int vs = vc & 1;
-                ok = bwait(&sm.p_full[buf], (p_par >> buf) & 1) && bwait(&sm.v_full[vs], (vc >> 1) & 1);
+                ok = wwait(&sm.p_full[buf], (p_par >> buf) & 1) && wwait(&sm.v_full[vs], (vc >> 1) & 1);
                 p_par ^= 1u << buf;
                 if (!ok) break;
                 ptx::tc_fence_after();
                 const int ksteps = (valid_keys(L, sg.kv0 + j) + 15) >> 4;
                 const uint32_t p_t = tmem + kColS + (uint32_t)buf * kBN;
                 const uint32_t v_s = ptx::smem_u32(sm.v[vs]);
-                for (int kk = 0; kk < ksteps; ++kk)  // O += P V, P from TMEM
-                    ptx::umma_f16_ts(tmem + kColO, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv,
-                                     (j > 0 || kk > 0) ? 1u : 0u);
-                ptx::umma_commit(ptx::smem_u32(&sm.v_empty[vs]));
-                ptx::umma_commit(ptx::smem_u32(&sm.o_ready[buf]));
+                // O += P V, P from TMEM.  The full-block case is unrolled: the
+                // issue rate of a single thread depends on a tight sequence.
+                if (ksteps == kBN / 16) {
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        ptx::umma_f16_ts_w(tmem + kColO, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv,
+                                         kk > 0 ? 1u : (j > 0 ? 1u : 0u));
+                } else {
+                    for (int kk = 0; kk < ksteps; ++kk)
+                        ptx::umma_f16_ts_w(tmem + kColO, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv,
+                                         (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                ptx::umma_commit_w(ptx::smem_u32(&sm.v_empty[vs]));
+                ptx::umma_commit_w(ptx::smem_u32(&sm.o_ready[buf]));
                 ++vc;
                 // The next QK into this S/P buffer follows the P V that reads it.
                 if (j + 3 < n) ok = issue_qk(q_s, buf, sg.kv0 + j + 3);
-            }
-            prev_oi_buf = -1;
-            if (ok && sg.kind != kHead) {
-                const int buf = (vb + n) % kSBufs;
-                const int s = kc & 1;
-                ok = bwait(&sm.k_full[s], (kc >> 1) & 1);
-                if (ok) {
-                    ptx::tc_fence_after();
-                    const uint32_t m_s = ptx::smem_u32(sm.k[s]);
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk)  // O_inter = Q (W_q S)
-                        ptx::umma_f16_ss(tmem + kColS + (uint32_t)buf * kBN, kmajor_desc(q_s, kk),
-                                         kmajor_desc(m_s, kk), idesc_qm, kk > 0);
-                    ptx::umma_commit(ptx::smem_u32(&sm.k_empty[s]));
-                    ++kc;
-                    prev_oi_buf = buf;
-                }
+                else if (ok && j == qm_after) ok = issue_qm();
             }
             if (!ok) break;
-            ptx::umma_commit(ptx::smem_u32(&sm.q_empty[qs]));
-            ptx::umma_commit(ptx::smem_u32(&sm.seg_done));
+            ptx::umma_commit_w(ptx::smem_u32(&sm.q_empty[qs]));
+            ptx::umma_commit_w(ptx::smem_u32(&sm.seg_done));
             vb += n + (sg.kind != kHead ? 1 : 0);
         }
         if (!ok) {
             fail();
             // nothing may still run on the tensor cores when TMEM is released
-            ptx::umma_commit(ptx::smem_u32(&sm.seg_done));
+            ptx::umma_commit_w(ptx::smem_u32(&sm.seg_done));
             ptx::mbar_wait_bounded(ptx::smem_u32(&sm.seg_done), si & 1, &no_abort, kWaitLimitNs);
         }
+    } else if (warp == 3) {
+        // ------------------------------------------- epilogue helper --
+        bool ok = true;
+        for (int si = 0; ok && si < rng.n_segs; ++si) {
+            const Seg sg = seg_at(sch, rng, si);
+            const int bh = sg.tile / sch.n_q, qt = sg.tile - bh * sch.n_q;
+            const int b = bh / H, h = bh - b * H;
+            if (sg.kind == kTail) {
+                // acquire the previous CTA's head partial of this tile
+                if (lane == 0) {
+                    const uint64_t t0 = ptx::globaltimer_ns();
+                    while (ptx::ld_acquire_gpu(flags + sg.tile) == 0) {
+                        if (*abort || ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    ptx::mbar_arrive(ptx::smem_u32(&sm.head_ready));
+                }
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+            }
+            ok = wwait(&sm.staged[si & 1], (si >> 1) & 1);
+            if (!ok) break;
+            if (sg.kind == kHead) {
+                // the head partial written by the softmax warps -> release flag
+                if (lane == 0) ptx::st_release_gpu(flags + sg.tile, 1);
+            } else {
+                const uint32_t stage = ptx::smem_u32(sm.q[si & 1]);
+                if (lane == 0) {
+                    if (sg.kind == kTail) flags[sg.tile] = 0;  // read: clear for the next launch
+                    ptx::tma_store_4d(&tm_o, stage, 0, h, qt * kBM, b);
+                    ptx::tma_store_4d(&tm_o, stage + kHalfBytes, 64, h, qt * kBM, b);
+                    ptx::bulk_commit_group();
+                    ptx::bulk_wait_group_read0();
+                }
+                __syncwarp();
+            }
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&sm.stage_free[si & 1]));
+        }
+        if (!ok) fail();
     } else if (warp >= 4) {
         // ---------------------------------------- softmax + epilogue --
         const int wg = (warp - 4) >> 2;               // 0: keys/cols 0-63, 1: 64-127
@@ -495,8 +566,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, bwait(&sm.seg_done, si & 1));
             if (!ok) break;
             ptx::tc_fence_after();
-            const int bh = sg.tile / sch.n_q, qt = sg.tile - bh * sch.n_q;
-            const int b = bh / H, h = bh - b * H;
             // partial of (tile, warpgroup): float4 chunk i of row r at [i][r], so
             // that the 32 lanes of a warp touch 512 consecutive bytes
             float4* pbase = reinterpret_cast<float4*>(part_o) + ((size_t)sg.tile * 2 + wg) * 16 * kBM + row;
@@ -517,28 +586,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (wg == 0)
                     *reinterpret_cast<float2*>(part_ml + ((size_t)sg.tile * kBM + row) * 2) =
                         make_float2(m_run, l_row);
-                __threadfence();
-                ok = meet_e();
-                if (!ok) break;
-                if (threadIdx.x == 128) {
-                    ptx::st_release_gpu(flags + sg.tile, 1);
-                    ptx::mbar_arrive(ptx::smem_u32(&sm.stage_free[si & 1]));  // staging unused
-                }
+                // warp 3 publishes it: these writes happen before its release
+                warp_arrive(&sm.staged[si & 1]);
             } else {
                 float a_t = 1.f, a_h = 0.f, inv_l = 1.f / l_row;
                 if (sg.kind == kTail) {
                     // the head piece of this tile was written by the previous CTA
-                    // at its start
-                    if (threadIdx.x == 128) {
-                        const uint64_t t0 = ptx::globaltimer_ns();
-                        while (ptx::ld_acquire_gpu(flags + sg.tile) == 0) {
-                            if (*abort || ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
-                                fail();
-                                break;
-                            }
-                        }
-                    }
-                    ok = meet_e();
+                    // at its start; warp 3 has acquired its flag
+                    ok = __all_sync(0xffffffffu, bwait(&sm.head_ready, 0));
                     if (!ok) break;
                     const float2 ml = __ldcg(reinterpret_cast<const float2*>(
                         part_ml + ((size_t)sg.tile * kBM + row) * 2));
@@ -586,17 +641,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 ptx::fence_proxy_async_smem();
-                // every thread has staged its row (and read the partial)
-                ok = meet_e();
-                if (!ok) break;
-                if (threadIdx.x == 128) {
-                    if (sg.kind == kTail) flags[sg.tile] = 0;  // clear for the next launch
-                    ptx::tma_store_4d(&tm_o, stage, 0, h, qt * kBM, b);
-                    ptx::tma_store_4d(&tm_o, stage + kHalfBytes, 64, h, qt * kBM, b);
-                    ptx::bulk_commit_group();
-                    ptx::bulk_wait_group_read0();
-                    ptx::mbar_arrive(ptx::smem_u32(&sm.stage_free[si & 1]));
-                }
+                // staged (and the partial read): warp 3 stores it
+                warp_arrive(&sm.staged[si & 1]);
             }
             ptx::tc_fence_before();
             warp_arrive(&sm.o_free);
