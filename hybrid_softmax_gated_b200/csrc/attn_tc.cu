@@ -25,28 +25,32 @@
 //
 // One CTA, 384 threads:
 //   warp 0       TMA producer (whole warp, one elected lane issues): Q
-//                tiles (2 slots), K and V blocks (2-stage
-//                rings), the (W_q S)^T tile through the K ring
-//   warp 1       UMMA issuer (whole warp, one elected lane issues): S = Q K^T into TMEM (three
-//                buffers, up to three key blocks ahead), O += P V with P
-//                read from TMEM, O_inter = Q M into the next free buffer
+//                tiles (2 slots), K and V blocks (2-stage rings), the
+//                (W_q S)^T tile through the K ring
+//   warp 1       UMMA issuer (whole warp, one elected lane issues)
 //   warp 2       TMEM allocator
 //   warp 3       epilogue helper: publishes head partials (release flag),
 //                acquires the flag of a tail's head partial, issues the TMA
 //                stores of staged outputs
-//   warps 4-7    softmax warpgroup 0: keys 0-63 of each block, O cols 0-63
-//   warps 8-11   softmax warpgroup 1: keys 64-127, O cols 64-127
-// Row r of a tile is TMEM lane r; both warpgroups own row r (lane quadrant
-// = warp % 4) and exchange row maxima and sums through shared memory,
-// synchronised by mbarriers (bounded waits, unlike bar.sync).
-// TMEM columns: [0,384) three S/P buffers, [384,512) O, fp32 (P: bf16
-// pairs packed over its S buffer).  Buffers rotate over "virtual blocks":
-// each key block of a segment, then (for a segment that finishes its tile)
-// one more for O_inter, read by the epilogue.
+//   warps 4-7    softmax warpgroup 0: even key blocks, accumulator O_0
+//   warps 8-11   softmax warpgroup 1: odd key blocks, accumulator O_1
+// The two warpgroups split the key blocks, not the columns: each thread
+// owns one row (TMEM lane) of a whole 128-key block, so the row max needs
+// no exchange, and each warpgroup keeps its own running max, row sum and
+// accumulator.  Their softmax work interleaves with the other's products
+// on the tensor core.  The epilogue combines (m_0, l_0, O_0) and
+// (m_1, l_1, O_1) once per segment.
+// TMEM columns: [0,256) two S/P buffers, [256,512) O_0 and O_1, fp32 (P:
+// bf16 pairs packed over the first half of its S buffer).  Buffers rotate
+// over "virtual blocks": each key block of a segment, then (for a segment
+// that finishes its tile) one more for O_inter, read by the epilogue.
+// Issue order per segment: S_0, S_1, then P V_j followed by the next item
+// into buffer j & 1 (S_{j+2}, or O_inter = Q (W_q S) after P V_{n-2}).
 // Online softmax with lazy rescaling: the running row max only moves when
 // it grows by more than 2^8; the final 1/l uses the same max as the
-// numerator, so the result is exact up to rounding.  One exponential in
-// three runs on the FMA pipe (exp2_fma) to balance it against the SFU.
+// numerator, so the result is exact up to rounding.  One pair of
+// exponentials in three runs on the FMA pipe (exp2_fma2, packed f32x2
+// arithmetic) to balance it against the SFU.
 // Outputs leave through a TMA store staged in the segment's Q slot; split
 // partials are stored so that a warp's lanes write consecutive 16 bytes.
 #include "attn_tc.h"
@@ -71,9 +75,14 @@ constexpr int kBN = 128;  // keys per block
 constexpr int kD = 128;   // head dim
 constexpr int kThreads = 384;
 constexpr int kSoftmaxWarps = 8;  // arrivals on the softmax barriers: one per warp
+constexpr int kWgWarps = 4;       // warps of one softmax warpgroup
+// Registers per thread: at launch (384 threads, one CTA per SM), then after
+// the split: warpgroup 0 (producer, issuer, allocator, helper) gives up
+// registers to the two softmax warpgroups.
+constexpr int kRegsLaunch = 168, kRegsLow = 96, kRegsHigh = 200;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 384;  // S/P buffers at 0, 128, 256
-constexpr int kSBufs = 3;
+constexpr uint32_t kColS = 0, kColO = 256;  // S/P buffers at 0, 128; O_0, O_1 at 256, 384
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -138,22 +147,21 @@ struct __align__(1024) Smem {
     uint64_t q_full[2], q_empty[2];
     uint64_t k_full[2], k_empty[2];
     uint64_t v_full[2], v_empty[2];
-    uint64_t s_full[kSBufs];
-    // Per S/P buffer: a buffer's next use needs the P V of its previous
-    // use issued, so these never run more than one phase ahead of a waiter.
-    uint64_t p_full[kSBufs];   // 8 warp arrivals: P of the buffer's block written (and O rescaled)
-    uint64_t o_ready[kSBufs];  // one commit: the P V reading the buffer is done
-    uint64_t seg_done;  // one commit per segment: its last UMMA is done
-    uint64_t o_free;    // 8 warp arrivals per segment: O and O_inter read out
-    uint64_t xch[2];    // 8 warp arrivals: row maxima of a key block exchanged
-    uint64_t ebar;      // 8 warp arrivals: epilogue exchanges
+    // Per S/P buffer b (= the softmax warpgroup that owns it): a buffer's
+    // next S needs the P V of its previous block issued, so neither barrier
+    // runs more than one phase ahead of its waiter.
+    uint64_t s_full[2];  // one commit: S of the buffer's block is in TMEM
+    uint64_t p_full[2];  // 4 warp arrivals: P written over S (and O_b rescaled)
+    uint64_t seg_done;   // one commit per segment: its last UMMA is done
+    uint64_t o_free;     // 8 warp arrivals per segment: O_0, O_1 and O_inter read out
+    uint64_t ebar;       // 8 warp arrivals: epilogue exchange of row maxima and sums
     uint64_t stage_free[2];  // 1 arrival per segment: the Q slot used as output staging is free
     uint64_t staged[2];      // 8 warp arrivals per segment (by si & 1): output staged / head
                              // partial written; a slot's next use needs stage_free, so warp 3
                              // can never fall two phases behind on one of them
     uint64_t head_ready;     // 1 arrival: the head partial of this CTA's tail piece is visible
-    float red_max[2][2][kBM];  // [block parity][warpgroup][row]
-    float red_sum[2][kBM];     // [warpgroup][row]
+    float red_m[2][kBM];     // [warpgroup][row] running max (log2 units) of the segment
+    float red_l[2][kBM];     // [warpgroup][row] row sum against that max
     uint32_t tmem_base;
     int abort;
 };
@@ -186,21 +194,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(ptx::smem_u32(&sm.k_empty[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sm.v_full[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sm.v_empty[s]), 1);
-        }
-        for (int s = 0; s < kSBufs; ++s) {
             ptx::mbar_init(ptx::smem_u32(&sm.s_full[s]), 1);
-            ptx::mbar_init(ptx::smem_u32(&sm.p_full[s]), kSoftmaxWarps);
-            ptx::mbar_init(ptx::smem_u32(&sm.o_ready[s]), 1);
+            ptx::mbar_init(ptx::smem_u32(&sm.p_full[s]), kWgWarps);
+            ptx::mbar_init(ptx::smem_u32(&sm.stage_free[s]), 1);
+            ptx::mbar_init(ptx::smem_u32(&sm.staged[s]), kSoftmaxWarps);
         }
         ptx::mbar_init(ptx::smem_u32(&sm.seg_done), 1);
         ptx::mbar_init(ptx::smem_u32(&sm.o_free), kSoftmaxWarps);
-        ptx::mbar_init(ptx::smem_u32(&sm.xch[0]), kSoftmaxWarps);
-        ptx::mbar_init(ptx::smem_u32(&sm.xch[1]), kSoftmaxWarps);
         ptx::mbar_init(ptx::smem_u32(&sm.ebar), kSoftmaxWarps);
-        ptx::mbar_init(ptx::smem_u32(&sm.stage_free[0]), 1);
-        ptx::mbar_init(ptx::smem_u32(&sm.stage_free[1]), 1);
-        ptx::mbar_init(ptx::smem_u32(&sm.staged[0]), kSoftmaxWarps);
-        ptx::mbar_init(ptx::smem_u32(&sm.staged[1]), kSoftmaxWarps);
         ptx::mbar_init(ptx::smem_u32(&sm.head_ready), 1);
         sm.abort = 0;
         ptx::fence_mbar_init();
@@ -227,6 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return __all_sync(0xffffffffu, bwait(bar, parity));
     };
 
+    if (warp < 4) ptx::setmaxnreg_dec<kRegsLow>();
     if (warp == 0) {
         // (the whole warp runs the producer; one elected lane issues)
         // ------------------------------------------------ TMA producer --
@@ -277,15 +279,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_arrive_expect_tx_w(qbar, kTileBytes);
             ptx::tma_load_4d_w(qdst, &tm_q, 0, h, qt * kBM, b, qbar);
             ptx::tma_load_4d_w(qdst + kHalfBytes, &tm_q, 64, h, qt * kBM, b, qbar);
-            // K and V in the order the issuer consumes them:
-            // K0 K1 K2 V0 K3 V1 ... V_{n-1} [M]
+            // The K ring carries the segment's key blocks, then (unless the
+            // segment is a head piece) the (W_q S)^T tile; the issuer takes
+            // items 0 and 1 first and item j + 2 after the P V of block j.
             const int n = sg.kv1 - sg.kv0;
-            for (int j = 0; ok && j < 3 && j < n; ++j) ok = load_k(b, h, sg.kv0 + j);
+            const int nk = n + (sg.kind != kHead ? 1 : 0);
+            auto load_item = [&](int i) { return load_k(b, h, i < n ? sg.kv0 + i : -1); };
+            for (int i = 0; ok && i < 2 && i < nk; ++i) ok = load_item(i);
             for (int j = 0; ok && j < n; ++j) {
                 ok = load_v(b, h, sg.kv0 + j);
-                if (ok && j + 3 < n) ok = load_k(b, h, sg.kv0 + j + 3);
+                if (ok && j + 2 < nk) ok = load_item(j + 2);
             }
-            if (ok && sg.kind != kHead) ok = load_k(b, h, -1);
         }
         if (!ok) fail();
         // Drain: the last loads of each ring have landed before exit.
@@ -298,75 +302,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // (the whole warp runs the issuer; one elected lane issues)
         // ------------------------------------------------- UMMA issuer --
-        constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBM, kD, false, true);
-        constexpr uint32_t idesc_qm = ptx::idesc_bf16_f32(kBM, kD, false, false);
+        const uint32_t idesc_pv = ptx::idesc_bf16_f32(kBM, kD, false, true);  // V: MN-major
+        const uint32_t idesc_qm = ptx::idesc_bf16_f32(kBM, kD, false, false);
         int kc = 0, vc = 0;
-        int vb = 0;           // virtual blocks so far: buffer of the next one is vb % 3
+        int vb = 0;           // virtual blocks so far: block vb + j of a segment uses buffer (vb + j) & 1
         uint32_t p_par = 0;   // bit b: phase parity of p_full[b] to wait for
+        int prev_oi_buf = -1; // buffer holding the previous segment's O_inter
         bool ok = true;
-        auto issue_qk = [&](uint32_t q_s, int buf, int kv) -> bool {  // S = Q K^T into buffer buf
-            const int s = kc & 1;
-            if (!wwait(&sm.k_full[s], (kc >> 1) & 1)) return false;
-            ptx::tc_fence_after();
-            const int valid = valid_keys(L, kv);
-            const uint32_t idesc = ptx::idesc_bf16_f32(kBM, (valid + 15) & ~15, false, false);
-            const uint32_t k_s = ptx::smem_u32(sm.k[s]);
-            const uint32_t d = tmem + kColS + (uint32_t)buf * kBN;
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk)
-                ptx::umma_f16_ss_w(d, kmajor_desc(q_s, kk), kmajor_desc(k_s, kk), idesc, kk > 0);
-            ptx::umma_commit_w(ptx::smem_u32(&sm.s_full[buf]));
-            ptx::umma_commit_w(ptx::smem_u32(&sm.k_empty[s]));
-            ++kc;
-            return true;
-        };
         int si = 0;
-        int prev_oi_buf = -1;  // buffer holding the previous segment's O_inter
         for (; ok && si < rng.n_segs; ++si) {
             const Seg sg = seg_at(sch, rng, si);
             const int qs = si & 1;
             const int n = sg.kv1 - sg.kv0;
+            const int nk = n + (sg.kind != kHead ? 1 : 0);
             if (!wwait(&sm.q_full[qs], (si >> 1) & 1)) {
                 ok = false;
                 break;
             }
             const uint32_t q_s = ptx::smem_u32(sm.q[qs]);
-            // Up to three blocks ahead.  A buffer last used by a key block is
-            // free (its P V was issued before); the buffer with the previous
-            // segment's O_inter, and O itself, are free once the epilogue of
-            // that segment has read them (o_free).
+            // O_0, O_1 and the buffer with the previous segment's O_inter are
+            // free once that segment's epilogue has read them (o_free).
             bool freed = si == 0;
-            for (int j = 0; ok && j < 3 && j < n; ++j) {
-                const int buf = (vb + j) % kSBufs;
-                if (!freed && buf == prev_oi_buf) {
-                    ok = wwait(&sm.o_free, (si - 1) & 1);
-                    freed = true;
-                }
-                if (ok) ok = issue_qk(q_s, buf, sg.kv0 + j);
-            }
-            if (ok && !freed) ok = wwait(&sm.o_free, (si - 1) & 1);
-            // O_inter = Q (W_q S) into buffer (vb + n) % 3, as soon as that
-            // buffer is free: after the P V of block n - 3, or now if n < 3.
-            const int qm_after = sg.kind == kHead ? -2 : (n >= 3 ? n - 3 : -1);
-            auto issue_qm = [&]() -> bool {
-                const int buf = (vb + n) % kSBufs;
+            auto make_free = [&](int buf) -> bool {
+                if (freed || (buf >= 0 && buf != prev_oi_buf)) return true;
+                freed = true;
+                return wwait(&sm.o_free, (si - 1) & 1);
+            };
+            // K-ring item i: S = Q K_i^T (i < n) or O_inter = Q (W_q S) (i == n),
+            // into buffer (vb + i) & 1
+            auto issue_item = [&](int i) -> bool {
+                const int buf = (vb + i) & 1;
+                if (!make_free(buf)) return false;
                 const int s = kc & 1;
                 if (!wwait(&sm.k_full[s], (kc >> 1) & 1)) return false;
                 ptx::tc_fence_after();
-                const uint32_t m_s = ptx::smem_u32(sm.k[s]);
+                const uint32_t k_s = ptx::smem_u32(sm.k[s]);
+                const uint32_t d = tmem + kColS + (uint32_t)buf * kBN;
+                if (i < n) {
+                    const int valid = valid_keys(L, sg.kv0 + i);
+                    const uint32_t idesc = ptx::idesc_bf16_f32(kBM, (valid + 15) & ~15, false, false);
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)
-                    ptx::umma_f16_ss_w(tmem + kColS + (uint32_t)buf * kBN, kmajor_desc(q_s, kk),
-                                       kmajor_desc(m_s, kk), idesc_qm, kk > 0);
+                    for (int kk = 0; kk < kD / 16; ++kk)
+                        ptx::umma_f16_ss_w(d, kmajor_desc(q_s, kk), kmajor_desc(k_s, kk), idesc, kk > 0);
+                    ptx::umma_commit_w(ptx::smem_u32(&sm.s_full[buf]));
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk)
+                        ptx::umma_f16_ss_w(d, kmajor_desc(q_s, kk), kmajor_desc(k_s, kk), idesc_qm, kk > 0);
+                }
                 ptx::umma_commit_w(ptx::smem_u32(&sm.k_empty[s]));
                 ++kc;
-                prev_oi_buf = buf;
                 return true;
             };
-            prev_oi_buf = -1;
-            if (ok && qm_after == -1) ok = issue_qm();
+            for (int i = 0; ok && i < 2 && i < nk; ++i) ok = issue_item(i);
+            if (ok) ok = make_free(-1);  // the first P V of each O_b starts it afresh
             for (int j = 0; ok && j < n; ++j) {
-                const int buf = (vb + j) % kSBufs;
+                const int buf = (vb + j) & 1;
                 const int vs = vc & 1;
                 ok = wwait(&sm.p_full[buf], (p_par >> buf) & 1) && wwait(&sm.v_full[vs], (vc >> 1) & 1);
                 p_par ^= 1u << buf;
@@ -374,30 +365,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tc_fence_after();
                 const int ksteps = (valid_keys(L, sg.kv0 + j) + 15) >> 4;
                 const uint32_t p_t = tmem + kColS + (uint32_t)buf * kBN;
+                const uint32_t o_t = tmem + kColO + (uint32_t)buf * kD;
                 const uint32_t v_s = ptx::smem_u32(sm.v[vs]);
-                // O += P V, P from TMEM.  The full-block case is unrolled: the
+                const uint32_t acc0 = j >= 2 ? 1u : 0u;
+                // O_b += P V, P from TMEM.  The full-block case is unrolled: the
                 // issue rate of a single thread depends on a tight sequence.
                 if (ksteps == kBN / 16) {
 #pragma unroll
                     for (int kk = 0; kk < kBN / 16; ++kk)
-                        ptx::umma_f16_ts_w(tmem + kColO, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv,
-                                         kk > 0 ? 1u : (j > 0 ? 1u : 0u));
+                        ptx::umma_f16_ts_w(o_t, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv,
+                                           kk > 0 ? 1u : acc0);
                 } else {
                     for (int kk = 0; kk < ksteps; ++kk)
-                        ptx::umma_f16_ts_w(tmem + kColO, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv,
-                                         (j > 0 || kk > 0) ? 1u : 0u);
+                        ptx::umma_f16_ts_w(o_t, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv,
+                                           kk > 0 ? 1u : acc0);
                 }
                 ptx::umma_commit_w(ptx::smem_u32(&sm.v_empty[vs]));
-                ptx::umma_commit_w(ptx::smem_u32(&sm.o_ready[buf]));
                 ++vc;
-                // The next QK into this S/P buffer follows the P V that reads it.
-                if (j + 3 < n) ok = issue_qk(q_s, buf, sg.kv0 + j + 3);
-                else if (ok && j == qm_after) ok = issue_qm();
+                // The next item into this buffer follows the P V that reads it.
+                if (j + 2 < nk) ok = issue_item(j + 2);
             }
             if (!ok) break;
             ptx::umma_commit_w(ptx::smem_u32(&sm.q_empty[qs]));
             ptx::umma_commit_w(ptx::smem_u32(&sm.seg_done));
-            vb += n + (sg.kind != kHead ? 1 : 0);
+            prev_oi_buf = sg.kind != kHead ? (vb + n) & 1 : -1;
+            vb += nk;
         }
         if (!ok) {
             fail();
@@ -448,15 +440,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) fail();
     } else if (warp >= 4) {
         // ---------------------------------------- softmax + epilogue --
-        const int wg = (warp - 4) >> 2;               // 0: keys/cols 0-63, 1: 64-127
+        ptx::setmaxnreg_inc<kRegsHigh>();
+        const int wg = (warp - 4) >> 2;               // S/P buffer, O accumulator and key blocks
         const int row = ((warp & 3) << 5) + lane;     // tile row = TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t col0 = (uint32_t)wg * 64;
-        int rb = 0;                  // key blocks processed so far (all segments)
+        const uint32_t sbuf = tmem + lane_base + kColS + (uint32_t)wg * kBN;
+        const uint32_t obuf = tmem + lane_base + kColO + (uint32_t)wg * kD;
         int vb = 0;                  // virtual blocks so far (see the issuer)
-        uint32_t s_par = 0;          // bit b: phase parity of s_full[b] to wait for
-        uint32_t o_par = 0;          // bit b: parity of the blocks processed on buffer b
-        uint32_t e_uses = 0;  // completed uses of ebar
+        uint32_t s_par = 0;          // phase parity of s_full[wg] to wait for
+        uint32_t e_uses = 0;         // completed uses of ebar
         bool ok = true;
         // One arrival per warp on the softmax barriers: the warp's lanes
         // are synchronised (and their shared-memory writes ordered) by
@@ -465,131 +457,152 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(bar));
         };
-        // all 8 softmax warps meet at bar (arrive, then a bounded wait)
-        auto meet = [&](uint64_t* bar, uint32_t parity) -> bool {
-            warp_arrive(bar);
-            return __all_sync(0xffffffffu, bwait(bar, parity));
+        // all 8 softmax warps meet at ebar (arrive, then a bounded wait)
+        auto meet_e = [&]() -> bool {
+            warp_arrive(&sm.ebar);
+            return __all_sync(0xffffffffu, bwait(&sm.ebar, (e_uses++) & 1));
         };
-        auto meet_e = [&]() -> bool { return meet(&sm.ebar, (e_uses++) & 1); };
+        const float2 sl2 = make_float2(scale_log2, scale_log2);
         for (int si = 0; ok && si < rng.n_segs; ++si) {
             const Seg sg = seg_at(sch, rng, si);
             const int n = sg.kv1 - sg.kv0;
-            float m_run = -INFINITY, l_part = 0.f;
-            for (int j = 0; j < n; ++j) {
-                const int blk = rb + j;
-                const int buf = (vb + j) % kSBufs;
-                const uint32_t sbuf = tmem + lane_base + kColS + (uint32_t)buf * kBN;
-                ok = __all_sync(0xffffffffu, bwait(&sm.s_full[buf], (s_par >> buf) & 1));
-                s_par ^= 1u << buf;
+            float m_run = -INFINITY, l_run = 0.f;
+            // this warpgroup's blocks of the segment: j = j0, j0 + 2, ...
+            const int j0 = ((vb & 1) == wg) ? 0 : 1;
+            for (int j = j0; j < n; j += 2) {
+                ok = __all_sync(0xffffffffu, bwait(&sm.s_full[wg], s_par));
+                s_par ^= 1u;
                 if (!ok) break;
                 ptx::tc_fence_after();
-                uint32_t raw[2][32];
-                ptx::tmem_ld32(sbuf + col0, raw[0]);
-                ptx::tmem_ld32(sbuf + col0 + 32, raw[1]);
+                uint32_t raw[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) ptx::tmem_ld32(sbuf + (uint32_t)c * 32, raw[c]);
                 ptx::tmem_wait_ld();
-                ptx::reg_fence(raw[0]);
-                ptx::reg_fence(raw[1]);
-                float x[64];
 #pragma unroll
-                for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(raw[i >> 5][i & 31]);
-                const int valid = valid_keys(L, sg.kv0 + j) - (int)col0;  // valid keys in my 64
-                if (valid < 64) {
+                for (int c = 0; c < 4; ++c) ptx::reg_fence(raw[c]);
+                float x[128];
 #pragma unroll
-                    for (int i = 0; i < 64; ++i)
+                for (int i = 0; i < 128; ++i) x[i] = __uint_as_float(raw[i >> 5][i & 31]);
+                const int valid = valid_keys(L, sg.kv0 + j);
+                if (valid < kBN) {
+#pragma unroll
+                    for (int i = 0; i < 128; ++i)
                         if (i >= valid) x[i] = -INFINITY;
                 }
-                // row max of my 64 columns: 3-input max tree
-                float m8[8];
+                // row max: 3-input max tree
+                float m16[16];
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    m8[i] = ptx::max3(ptx::max3(x[8 * i], x[8 * i + 1], x[8 * i + 2]),
-                                      ptx::max3(x[8 * i + 3], x[8 * i + 4], x[8 * i + 5]),
-                                      fmaxf(x[8 * i + 6], x[8 * i + 7]));
-                float mx = ptx::max3(ptx::max3(m8[0], m8[1], m8[2]), ptx::max3(m8[3], m8[4], m8[5]),
-                                     fmaxf(m8[6], m8[7]));
-                sm.red_max[blk & 1][wg][row] = mx;
-                ok = meet(&sm.xch[blk & 1], (blk >> 1) & 1);
-                if (!ok) break;
-                mx = fmaxf(mx, sm.red_max[blk & 1][wg ^ 1][row]);
+                for (int i = 0; i < 16; ++i)
+                    m16[i] = ptx::max3(ptx::max3(x[8 * i], x[8 * i + 1], x[8 * i + 2]),
+                                       ptx::max3(x[8 * i + 3], x[8 * i + 4], x[8 * i + 5]),
+                                       fmaxf(x[8 * i + 6], x[8 * i + 7]));
+                float m4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    m4[i] = ptx::max3(m16[4 * i], m16[4 * i + 1], fmaxf(m16[4 * i + 2], m16[4 * i + 3]));
+                const float mx = ptx::max3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
                 const float m_new = fmaxf(m_run, mx * scale_log2);
                 const bool need = m_new > m_run + kRescaleLog2;
                 const float m_use = need ? m_new : m_run;
                 const float corr = need ? ptx::ex2(m_run - m_new) : 1.f;
-                const float neg_m = -m_use;
-                float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-                uint32_t pk[32];
+                const float2 nm = make_float2(-m_use, -m_use);
+                float2 sum4[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+                uint32_t pk[64];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    // every third exponential on the FMA pipe, the rest on the SFU
-                    const float a0 = fmaf(x[2 * i], scale_log2, neg_m);
-                    const float a1 = fmaf(x[2 * i + 1], scale_log2, neg_m);
-                    const float p0 = ((2 * i) % 3 == 2) ? ptx::exp2_fma(a0) : ptx::ex2(a0);
-                    const float p1 = ((2 * i + 1) % 3 == 2) ? ptx::exp2_fma(a1) : ptx::ex2(a1);
-                    sum4[i & 3] += p0 + p1;
-                    pk[i] = ptx::pack_bf16x2(p0, p1);
+                for (int i = 0; i < 64; ++i) {
+                    // a pair in three on the FMA pipe, the rest on the SFU
+                    const float2 a = ptx::fma2(make_float2(x[2 * i], x[2 * i + 1]), sl2, nm);
+                    float2 p;
+                    if (i % 3 == 2) {
+                        p = ptx::exp2_fma2(a);
+                    } else {
+                        p.x = ptx::ex2(a.x);
+                        p.y = ptx::ex2(a.y);
+                    }
+                    sum4[i & 3] = ptx::add2(sum4[i & 3], p);
+                    pk[i] = ptx::pack_bf16x2(p.x, p.y);
                 }
-                l_part = l_part * corr + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+                const float2 s2 = ptx::add2(ptx::add2(sum4[0], sum4[1]), ptx::add2(sum4[2], sum4[3]));
+                l_run = l_run * corr + (s2.x + s2.y);
                 m_run = m_use;
-                // P over my half of the S columns (both warpgroups finished
-                // reading S at the barrier above)
-                ptx::tmem_st32_u(sbuf + (uint32_t)wg * 32, pk);
-                if (j >= 1 && __any_sync(0xffffffffu, need)) {
-                    // rescale my half of O once the previous block's P V is done
-                    // (its commit is the latest on that buffer)
-                    const int pb = (vb + j - 1) % kSBufs;
-                    ok = __all_sync(0xffffffffu, bwait(&sm.o_ready[pb], ((o_par >> pb) & 1) ^ 1));
-                    if (!ok) break;
-                    ptx::tc_fence_after();
+                // P (bf16 pairs) over the first 64 columns of the S buffer
+                ptx::tmem_st32_u(sbuf, pk);
+                ptx::tmem_st32_u(sbuf + 32, pk + 32);
+                if (j >= 2 && __any_sync(0xffffffffu, need)) {
+                    // rescale O_wg: S of this block was committed after the
+                    // P V of this warpgroup's previous block, so that is done
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
+                    for (int c = 0; c < 4; ++c) {
                         uint32_t o[32];
-                        const uint32_t ta = tmem + lane_base + kColO + col0 + (uint32_t)c * 32;
-                        ptx::tmem_ld32(ta, o);
+                        ptx::tmem_ld32(obuf + (uint32_t)c * 32, o);
                         ptx::tmem_wait_ld();
                         ptx::reg_fence(o);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
-                        ptx::tmem_st32(ta, o);
+                        ptx::tmem_st32(obuf + (uint32_t)c * 32, o);
                     }
                 }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                warp_arrive(&sm.p_full[buf]);
-                o_par ^= 1u << buf;
+                warp_arrive(&sm.p_full[wg]);
             }
             if (!ok) break;
             // ------------------------------------------------ epilogue --
-            sm.red_sum[wg][row] = l_part;
+            // combine the two warpgroups' running (max, sum) of each row
+            const bool has0 = n >= 2 || (vb & 1) == 0;
+            const bool has1 = n >= 2 || (vb & 1) == 1;
+            sm.red_m[wg][row] = m_run;
+            sm.red_l[wg][row] = l_run;
             ok = meet_e();
             if (!ok) break;
-            const float l_row = l_part + sm.red_sum[wg ^ 1][row];
+            const float m0 = sm.red_m[0][row], m1 = sm.red_m[1][row];
+            const float l0 = sm.red_l[0][row], l1 = sm.red_l[1][row];
+            const float m_seg = fmaxf(has0 ? m0 : -INFINITY, has1 ? m1 : -INFINITY);
+            const float a0 = has0 ? ptx::ex2(m0 - m_seg) : 0.f;
+            const float a1 = has1 ? ptx::ex2(m1 - m_seg) : 0.f;
+            const float l_seg = a0 * l0 + a1 * l1;
             ok = __all_sync(0xffffffffu, bwait(&sm.seg_done, si & 1));
             if (!ok) break;
             ptx::tc_fence_after();
-            // partial of (tile, warpgroup): float4 chunk i of row r at [i][r], so
+            // this warpgroup's output columns [64 wg, 64 wg + 64) of
+            // a0 O_0 + a1 O_1 (unnormalised, against m_seg)
+            const uint32_t ocol = tmem + lane_base + kColO + (uint32_t)wg * 64;
+            auto load_acc = [&](int c, float (&acc)[32]) {
+                // (a warpgroup without blocks in this segment left its O stale:
+                // it is loaded but not used)
+                uint32_t o0[32], o1[32];
+                ptx::tmem_ld32(ocol + (uint32_t)c * 32, o0);
+                ptx::tmem_ld32(ocol + kD + (uint32_t)c * 32, o1);
+                ptx::tmem_wait_ld();
+                ptx::reg_fence(o0);
+                ptx::reg_fence(o1);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float v0 = has0 ? a0 * __uint_as_float(o0[i]) : 0.f;
+                    acc[i] = has1 ? fmaf(a1, __uint_as_float(o1[i]), v0) : v0;
+                }
+            };
+            // partial of (tile, column half): float4 chunk i of row r at [i][r], so
             // that the 32 lanes of a warp touch 512 consecutive bytes
             float4* pbase = reinterpret_cast<float4*>(part_o) + ((size_t)sg.tile * 2 + wg) * 16 * kBM + row;
             if (sg.kind == kHead) {
                 // unnormalised O, running max and row sum -> partial, then the flag
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
-                    uint32_t o[32];
-                    ptx::tmem_ld32(tmem + lane_base + kColO + col0 + (uint32_t)c * 32, o);
-                    ptx::tmem_wait_ld();
-                    ptx::reg_fence(o);
+                    float acc[32];
+                    load_acc(c, acc);
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
                         pbase[(size_t)(c * 8 + i) * kBM] =
-                            make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                        __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+                            make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
                 }
                 if (wg == 0)
                     *reinterpret_cast<float2*>(part_ml + ((size_t)sg.tile * kBM + row) * 2) =
-                        make_float2(m_run, l_row);
+                        make_float2(m_seg, l_seg);
                 // warp 3 publishes it: these writes happen before its release
                 warp_arrive(&sm.staged[si & 1]);
             } else {
-                float a_t = 1.f, a_h = 0.f, inv_l = 1.f / l_row;
+                float a_t = 1.f, a_h = 0.f, inv_l = 1.f / l_seg;
                 if (sg.kind == kTail) {
                     // the head piece of this tile was written by the previous CTA
                     // at its start; warp 3 has acquired its flag
@@ -597,25 +610,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     const float2 ml = __ldcg(reinterpret_cast<const float2*>(
                         part_ml + ((size_t)sg.tile * kBM + row) * 2));
-                    const float mm = fmaxf(ml.x, m_run);
+                    const float mm = fmaxf(ml.x, m_seg);
                     a_h = ptx::ex2(ml.x - mm);
-                    a_t = ptx::ex2(m_run - mm);
-                    inv_l = 1.f / (a_h * ml.y + a_t * l_row);
+                    a_t = ptx::ex2(m_seg - mm);
+                    inv_l = 1.f / (a_h * ml.y + a_t * l_seg);
                 }
                 const uint32_t stage = ptx::smem_u32(sm.q[si & 1]);  // the segment's Q slot
+                const uint32_t oi_col = tmem + lane_base + kColS + (uint32_t)((vb + n) & 1) * kBN + (uint32_t)wg * 64;
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
-                    uint32_t o[32], oi[32];
-                    ptx::tmem_ld32(tmem + lane_base + kColO + col0 + (uint32_t)c * 32, o);
-                    ptx::tmem_ld32(tmem + lane_base + kColS + (uint32_t)((vb + n) % kSBufs) * kBN + col0 +
-                                       (uint32_t)c * 32,
-                                   oi);
-                    ptx::tmem_wait_ld();
-                    ptx::reg_fence(o);
-                    ptx::reg_fence(oi);
                     float acc[32];
+                    load_acc(c, acc);
+                    uint32_t oi[32];
+                    ptx::tmem_ld32(oi_col + (uint32_t)c * 32, oi);
+                    ptx::tmem_wait_ld();
+                    ptx::reg_fence(oi);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[i] = a_t * __uint_as_float(o[i]);
+                    for (int i = 0; i < 32; ++i) acc[i] *= a_t;
                     if (sg.kind == kTail) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
@@ -646,7 +657,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ptx::tc_fence_before();
             warp_arrive(&sm.o_free);
-            rb += n;
             vb += n + (sg.kind != kHead ? 1 : 0);
         }
         if (!ok) fail();
@@ -683,6 +693,12 @@ AttnTc* attn_tc_create(Dims dm, void* workspace, int max_ctas) {
     if (dm.d != kD || dm.L < 1 || dm.H < 1 || dm.B < 1 || !tma_available() || !workspace) return nullptr;
     if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    // the warpgroups' register split needs the launch count it was sized for
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, attn_tc_kernel) != cudaSuccess || fa.numRegs != kRegsLaunch) {
         cudaGetLastError();
         return nullptr;
     }
