@@ -122,7 +122,7 @@ arl2_status refresh_derived(arl2_handle* h, cudaStream_t st) {
 arl2_status clean_update(arl2_handle* h, const void* k, const void* v, const float* alpha,
                          const float* beta, cudaStream_t st) {
     if (h->use_tc) {
-        h->launches += 3;
+        h->launches += 2;
         return arl2::update_tc_launch(h->up, *h->maps, k, v, alpha, beta, h->err, st) == cudaSuccess
                    ? ARL2_OK
                    : ARL2_ERR_CUDA;

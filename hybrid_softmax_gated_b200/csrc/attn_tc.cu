@@ -13,15 +13,17 @@
 //
 // Work decomposition.  A tile is 128 query rows of one (stream, head); a
 // unit is one tile against one block of 128 keys.  When there are more
-// tiles than SMs the grid is persistent (one CTA per SM, cooperative launch
-// so that all CTAs are resident) and CTA c takes the contiguous unit range
+// tiles than SMs the grid is persistent (at most one CTA per SM) and CTA c
+// takes the contiguous unit range
 // [c U / G, (c+1) U / G).  A tile cut by a range boundary has a head piece
 // (its first key blocks, at the end of CTA c's range) and a tail piece (the
 // rest, at the start of CTA c+1's range).  Each CTA runs its head piece
 // FIRST and writes it as an fp32 partial (unnormalised O, running max, row
 // sum) with a release flag; it runs its tail piece LAST, then acquires the
 // flag of the partial the previous CTA wrote at its start and merges the
-// two.  Waits are bounded.  With no more tiles than SMs, one CTA per tile.
+// two.  A CTA only ever waits for the CTA before it, which the block
+// scheduler has dispatched first; the waits are bounded all the same.  With
+// no more tiles than SMs, one CTA per tile.
 //
 // One CTA, 384 threads:
 //   warp 0       TMA producer (whole warp, one elected lane issues): Q
@@ -215,6 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    // The next kernel may launch now and run its own set-up; nothing of this
+    // kernel touches global memory before the previous kernel has finished.
+    ptx::pdl_trigger();
+    ptx::pdl_wait();
 
     auto fail = [&]() {
         atomicOr(err, kErrTimeoutAttn);
@@ -751,9 +757,11 @@ cudaError_t attn_tc_launch(AttnTc* t, TokenMapCache& maps, const void* q, const 
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = st;
+    // Programmatic dependent launch: the CTAs start (set-up only) while the
+    // previous kernel drains.
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = t->sch.split ? 1 : 0;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, attn_tc_kernel, cq, ck, cv, t->tm_m, co, t->part_o, t->part_ml,

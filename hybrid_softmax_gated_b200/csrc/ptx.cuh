@@ -259,6 +259,18 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ---- programmatic dependent launch -----------------------------------------
+// pdl_trigger: this CTA allows the next kernel in the stream to be launched
+// (it starts once every CTA of this grid has triggered or exited).
+// pdl_wait: block until the previous kernel in the stream has completed and
+// its memory operations are visible; returns at once without such a kernel.
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---- register reallocation between warpgroups ------------------------------
 // Every warp of a warpgroup executes the same one.  The increases of a CTA
 // draw on the registers it was launched with (threads x registers per

@@ -8,7 +8,6 @@
 //   attn     softmax(Q K^T s) V + (Q W_q) S_{N-1}          §2.1 items 1-2, Output
 //   residual r = v' - k' S_{N-1}                           §2.1 State Update
 //   accum    S = alpha S + k'^T diag(beta) r               §2.1 State Update
-//   fold     (W_q S)^T and S in bf16 for the tensor-core path
 #include "internal.h"
 
 #include <cmath>
@@ -241,58 +240,6 @@ __global__ void __launch_bounds__(128) accum_simt_kernel(const float* __restrict
     }
 }
 
-// --------------------------------------------------------------- fold ----
-// Copies of the state derived from S alone, for the tensor-core path:
-//   Mt[b][h][n][a] = bf16(sum_c Wq[h][a][c] S[b][h][c][n])   ((W_q S)^T)
-//   Sb[b][h][c][n] = bf16(S[b][h][c][n])
-// One CTA: 16 rows a of W_q S (and rows c = a of Sb); thread n owns column
-// n.  S of the (stream, head) is staged in shared memory first so that the
-// product loop reads no global memory.
-constexpr int kFoldRows = 16;
-
-__global__ void __launch_bounds__(128) fold_state_kernel(const __nv_bfloat16* __restrict__ wq,
-                                                         const float* __restrict__ S,
-                                                         __nv_bfloat16* __restrict__ Mt,
-                                                         __nv_bfloat16* __restrict__ Sb, Dims dm) {
-    extern __shared__ float fsm[];
-    const int d = dm.d;
-    float* Ss = fsm;                 // [d][d]
-    float* Ws = fsm + d * d;         // [kFoldRows][d]
-    const int a0 = blockIdx.x * kFoldRows, h = blockIdx.y, b = blockIdx.z;
-    const int n = threadIdx.x;
-    const size_t base = ((size_t)b * dm.H + h) * d * d;
-    const __nv_bfloat16* W = wq + (size_t)h * d * d;
-    if ((d & 3) == 0) {
-        // float4 copies, unrolled so that many loads are in flight at once
-        const float4* src = reinterpret_cast<const float4*>(S + base);
-        float4* dst = reinterpret_cast<float4*>(Ss);
-        const int n4 = d * d / 4;
-#pragma unroll 8
-        for (int i = threadIdx.x; i < n4; i += blockDim.x) dst[i] = src[i];
-    } else {
-        for (int i = threadIdx.x; i < d * d; i += blockDim.x) Ss[i] = S[base + i];
-    }
-    for (int i = threadIdx.x; i < kFoldRows * d; i += blockDim.x) {
-        const int r = i / d, c = i - r * d;
-        Ws[i] = a0 + r < d ? __bfloat162float(W[(size_t)(a0 + r) * d + c]) : 0.f;
-    }
-    __syncthreads();
-    if (n >= d) return;
-    float acc[kFoldRows];
-#pragma unroll
-    for (int i = 0; i < kFoldRows; ++i) acc[i] = 0.f;
-    for (int c = 0; c < d; ++c) {
-        const float s = Ss[c * d + n];
-#pragma unroll
-        for (int i = 0; i < kFoldRows; ++i) acc[i] = fmaf(Ws[i * d + c], s, acc[i]);
-    }
-#pragma unroll
-    for (int i = 0; i < kFoldRows; ++i) {
-        if (a0 + i >= d) break;
-        Mt[base + (size_t)n * d + a0 + i] = __float2bfloat16_rn(acc[i]);
-        Sb[base + (size_t)(a0 + i) * d + n] = __float2bfloat16_rn(Ss[(a0 + i) * d + n]);
-    }
-}
 
 template <typename K>
 cudaError_t set_smem(K kernel, size_t bytes) {
@@ -304,7 +251,6 @@ constexpr size_t kPhiSmemMax = sizeof(float) * (128 * 128 + 2 * kPhiRows * 128);
 constexpr size_t kAttnSmemMax =
     sizeof(float) * (kAQ * 128 + kAK * 129 + kAK * 128 + kAQ * (kAK + 1) + 128 * 128);
 constexpr size_t kResidualSmemMax = sizeof(float) * (128 * 128 + kRRows * 128);
-constexpr size_t kFoldSmemMax = sizeof(float) * (128 * 128 + kFoldRows * 128);
 
 }  // namespace
 
@@ -314,7 +260,6 @@ cudaError_t simt_init() {
     if ((e = set_smem(phi_simt_kernel<__nv_bfloat16>, kPhiSmemMax)) != cudaSuccess) return e;
     if ((e = set_smem(attn_simt_kernel<float>, kAttnSmemMax)) != cudaSuccess) return e;
     if ((e = set_smem(attn_simt_kernel<__nv_bfloat16>, kAttnSmemMax)) != cudaSuccess) return e;
-    if ((e = set_smem(fold_state_kernel, kFoldSmemMax)) != cudaSuccess) return e;
     return set_smem(residual_simt_kernel, kResidualSmemMax);
 }
 
@@ -366,13 +311,5 @@ cudaError_t launch_accum_simt(const float* kp, const float* r, const float* alph
     return cudaGetLastError();
 }
 
-cudaError_t launch_fold_state(const void* wq_bf16, const float* S, void* Mt, void* Sb, Dims dm,
-                              cudaStream_t st) {
-    const dim3 grid((dm.d + kFoldRows - 1) / kFoldRows, dm.H, dm.B);
-    const size_t smem = sizeof(float) * ((size_t)dm.d * dm.d + (size_t)kFoldRows * dm.d);
-    fold_state_kernel<<<grid, 128, smem, st>>>((const __nv_bfloat16*)wq_bf16, S, (__nv_bfloat16*)Mt,
-                                            (__nv_bfloat16*)Sb, dm);
-    return cudaGetLastError();
-}
 
 }  // namespace arl2

@@ -16,13 +16,14 @@
 //   KS = K' S_{N-1}                            (S_{N-1} as bf16)
 //   beta R = beta (Vp - KS)    -> bf16 tile    (epilogue)
 //   dS = K'^T (beta R)                         (the same K' tile read MN-major)
-// and writes dS as an fp32 partial.  update_finalize_kernel sums the
+// and writes dS as an fp32 partial.  finalize_fold_kernel sums the
 // partials in chunk order (deterministic) and applies the forget gate,
 //   S_N = alpha S_{N-1} + sum dS,
-// and the fold kernel then derives from S_N alone the bf16 copy of S and
-// Mt = (W_q S_N)^T, the matrix the attention kernel reads (so that the
-// inter-frame read Q' S = Q (W_q S) needs no per-token phi_q product, and a
-// restored checkpoint reproduces Mt exactly).
+// and derives from S_N alone the bf16 copy of S and Mt = (W_q S_N)^T, the
+// matrix the attention kernel reads (so that the inter-frame read
+// Q' S = Q (W_q S) needs no per-token phi_q product, and a restored
+// checkpoint reproduces Mt exactly: the same kernel, without partials,
+// derives them after a state restore).
 #include "update_tc.h"
 #include "ptx.cuh"
 
@@ -30,6 +31,7 @@
 
 #include <cmath>
 #include <new>
+#include <utility>
 
 namespace arl2 {
 namespace {
@@ -90,6 +92,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    // set-up done: let the next kernel launch; wait for the previous one
+    ptx::pdl_trigger();
+    ptx::pdl_wait();
     auto fail = [&]() {
         atomicOr(err, kErrTimeoutUpdate);
         *abort = 1;
@@ -253,39 +258,93 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// Deterministic reduction of the chunk partials and the forget gate:
-// S_N = alpha S_{N-1} + sum over chunks (in chunk order) of dS.
-// One CTA: 8 rows of S of one (stream, head); one float4 per thread.
-__global__ void __launch_bounds__(256) update_finalize_kernel(const float* __restrict__ part_s,
-                                                              const float* __restrict__ alpha,
-                                                              float* __restrict__ S, int n_chunks,
-                                                              int H) {
-    const int h = blockIdx.y, b = blockIdx.z, bh = b * H + h;
-    const int e = blockIdx.x * 1024 + threadIdx.x * 4;  // element of the 128x128 matrix
-    const float a = alpha[bh];
-    const size_t base = (size_t)bh * kD * kD + e;
-    const size_t pbase = (size_t)bh * n_chunks * kD * kD + e;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    // Loads in groups of 8 so that they are in flight together; the sum
-    // itself stays in chunk order.
-    for (int c0 = 0; c0 < n_chunks; c0 += 8) {
-        float4 p[8];
+// Deterministic reduction of the chunk partials and the forget gate,
+//   S_N = alpha S_{N-1} + sum over chunks (in chunk order) of dS,
+// then the copies the attention and update kernels read: Sb = bf16(S_N)
+// and Mt = (W_q S_N)^T in bf16.  One CTA: 8 columns n0..n0+7 of S of one
+// (stream, head), 128 threads.  Thread r reduces row r of those columns;
+// then thread a forms M[a][n] = sum_c W_q[a][c] S_N[c][n] (c in order, fp32)
+// for the 8 columns, which are whole rows n of Mt.  With n_chunks = 0 and
+// no alpha it only derives Sb and Mt from S (a restored state).
+constexpr int kFoldCols = 8;
+__global__ void __launch_bounds__(kD) finalize_fold_kernel(const float* __restrict__ part_s,
+                                                           const float* __restrict__ alpha,
+                                                           float* __restrict__ S,
+                                                           const __nv_bfloat16* __restrict__ wq,
+                                                           __nv_bfloat16* __restrict__ Mt,
+                                                           __nv_bfloat16* __restrict__ Sb, int n_chunks,
+                                                           int H) {
+    __shared__ __align__(16) float scol[kD][kFoldCols];
+    ptx::pdl_trigger();
+    ptx::pdl_wait();
+    const int n0 = blockIdx.x * kFoldCols, h = blockIdx.y, b = blockIdx.z, bh = b * H + h;
+    const int r = threadIdx.x;
+    const size_t e = (size_t)bh * kD * kD + (size_t)r * kD + n0;
+    float4 s0 = *reinterpret_cast<const float4*>(S + e);
+    float4 s1 = *reinterpret_cast<const float4*>(S + e + 4);
+    if (alpha) {
+        const float a = alpha[bh];
+        float4 c0 = make_float4(0.f, 0.f, 0.f, 0.f), c1 = c0;
+        const size_t pb = (size_t)bh * n_chunks * kD * kD + (size_t)r * kD + n0;
+        // Loads in groups of 8 so that they are in flight together; the sum
+        // itself stays in chunk order.
+        for (int g = 0; g < n_chunks; g += 8) {
+            float4 p[8][2];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (c0 + i < n_chunks)
-                p[i] = __ldcg(reinterpret_cast<const float4*>(part_s + pbase + (size_t)(c0 + i) * kD * kD));
+            for (int i = 0; i < 8; ++i)
+                if (g + i < n_chunks) {
+                    const float4* src = reinterpret_cast<const float4*>(part_s + pb + (size_t)(g + i) * kD * kD);
+                    p[i][0] = __ldcg(src);
+                    p[i][1] = __ldcg(src + 1);
+                }
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (c0 + i < n_chunks) {
-                acc.x += p[i].x;
-                acc.y += p[i].y;
-                acc.z += p[i].z;
-                acc.w += p[i].w;
-            }
+            for (int i = 0; i < 8; ++i)
+                if (g + i < n_chunks) {
+                    c0.x += p[i][0].x; c0.y += p[i][0].y; c0.z += p[i][0].z; c0.w += p[i][0].w;
+                    c1.x += p[i][1].x; c1.y += p[i][1].y; c1.z += p[i][1].z; c1.w += p[i][1].w;
+                }
+        }
+        s0 = make_float4(fmaf(a, s0.x, c0.x), fmaf(a, s0.y, c0.y), fmaf(a, s0.z, c0.z), fmaf(a, s0.w, c0.w));
+        s1 = make_float4(fmaf(a, s1.x, c1.x), fmaf(a, s1.y, c1.y), fmaf(a, s1.z, c1.z), fmaf(a, s1.w, c1.w));
+        *reinterpret_cast<float4*>(S + e) = s0;
+        *reinterpret_cast<float4*>(S + e + 4) = s1;
     }
-    float4 s = *reinterpret_cast<const float4*>(S + base);
-    s = make_float4(fmaf(a, s.x, acc.x), fmaf(a, s.y, acc.y), fmaf(a, s.z, acc.z), fmaf(a, s.w, acc.w));
-    *reinterpret_cast<float4*>(S + base) = s;
+    uint4 sb;
+    sb.x = ptx::pack_bf16x2(s0.x, s0.y);
+    sb.y = ptx::pack_bf16x2(s0.z, s0.w);
+    sb.z = ptx::pack_bf16x2(s1.x, s1.y);
+    sb.w = ptx::pack_bf16x2(s1.z, s1.w);
+    *reinterpret_cast<uint4*>(Sb + e) = sb;
+    *reinterpret_cast<float4*>(&scol[r][0]) = s0;
+    *reinterpret_cast<float4*>(&scol[r][4]) = s1;
+    __syncthreads();
+    // M[a][n0 + j] = sum_c W_q[a][c] S_N[c][n0 + j]; thread a = r
+    const uint4* wrow = reinterpret_cast<const uint4*>(wq + ((size_t)h * kD + r) * kD);
+    float acc[kFoldCols];
+#pragma unroll
+    for (int j = 0; j < kFoldCols; ++j) acc[j] = 0.f;
+    for (int c8 = 0; c8 < kD / 8; ++c8) {
+        const uint4 w8 = __ldg(wrow + c8);
+        const uint32_t wv[4] = {w8.x, w8.y, w8.z, w8.w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const uint32_t pr = wv[k >> 1];
+            const float w = __uint_as_float((k & 1) ? (pr & 0xffff0000u) : (pr << 16));
+            const float4 x0 = *reinterpret_cast<const float4*>(&scol[c8 * 8 + k][0]);
+            const float4 x1 = *reinterpret_cast<const float4*>(&scol[c8 * 8 + k][4]);
+            acc[0] = fmaf(w, x0.x, acc[0]);
+            acc[1] = fmaf(w, x0.y, acc[1]);
+            acc[2] = fmaf(w, x0.z, acc[2]);
+            acc[3] = fmaf(w, x0.w, acc[3]);
+            acc[4] = fmaf(w, x1.x, acc[4]);
+            acc[5] = fmaf(w, x1.y, acc[5]);
+            acc[6] = fmaf(w, x1.z, acc[6]);
+            acc[7] = fmaf(w, x1.w, acc[7]);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kFoldCols; ++j)
+        Mt[((size_t)bh * kD + n0 + j) * kD + r] = __float2bfloat16_rn(acc[j]);
 }
 
 }  // namespace
@@ -321,19 +380,46 @@ UpdateTc* update_tc_create(const Dims& dm, const UpdateBuffers& buf) {
 
 void update_tc_destroy(UpdateTc* u) { delete u; }
 
+// Launch with programmatic stream serialisation: the kernel's CTAs may
+// start while the previous kernel drains; each waits (griddepcontrol) before
+// it touches global memory.
+template <typename... P, typename... A>
+static cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              A&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
+
 cudaError_t update_tc_launch(UpdateTc* u, TokenMapCache& maps, const void* k, const void* v,
                              const float* alpha, const float* beta, int* err, cudaStream_t st) {
     const Dims& dm = u->dm;
     CUtensorMap ck, cv;
     if (!maps.get(k, &ck) || !maps.get(v, &cv)) return cudaErrorInvalidValue;
-    update_chunk_kernel<<<dim3(u->n_chunks, dm.H, dm.B), kThreads, kSmemBytes, st>>>(
-        ck, cv, u->tm_w, u->tm_sb, beta, u->buf.part_s, dm.L, dm.H, err);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(update_chunk_kernel, dim3(u->n_chunks, dm.H, dm.B), dim3(kThreads), kSmemBytes,
+                               st, ck, cv, u->tm_w, u->tm_sb, beta, u->buf.part_s, dm.L, dm.H, err);
     if (e != cudaSuccess) return e;
-    update_finalize_kernel<<<dim3(kD * kD / 1024, dm.H, dm.B), 256, 0, st>>>(
-        u->buf.part_s, alpha, u->buf.S, u->n_chunks, dm.H);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    return launch_fold_state(u->buf.w_all, u->buf.S, u->buf.Mt, u->buf.Sb, dm, st);
+    return launch_pdl(finalize_fold_kernel, dim3(kD / kFoldCols, dm.H, dm.B), dim3(kD), 0, st,
+                      static_cast<const float*>(u->buf.part_s), alpha, u->buf.S,
+                      static_cast<const __nv_bfloat16*>(u->buf.w_all), static_cast<__nv_bfloat16*>(u->buf.Mt),
+                      static_cast<__nv_bfloat16*>(u->buf.Sb), u->n_chunks, dm.H);
+}
+
+cudaError_t launch_fold_state(const void* wq_bf16, const float* S, void* Mt, void* Sb, Dims dm,
+                              cudaStream_t st) {
+    if (dm.d != kD) return cudaErrorInvalidValue;
+    return launch_pdl(finalize_fold_kernel, dim3(kD / kFoldCols, dm.H, dm.B), dim3(kD), 0, st,
+                      static_cast<const float*>(nullptr), static_cast<const float*>(nullptr),
+                      const_cast<float*>(S), static_cast<const __nv_bfloat16*>(wq_bf16),
+                      static_cast<__nv_bfloat16*>(Mt), static_cast<__nv_bfloat16*>(Sb), 0, dm.H);
 }
 
 }  // namespace arl2
