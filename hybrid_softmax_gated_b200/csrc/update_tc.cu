@@ -261,12 +261,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Deterministic reduction of the chunk partials and the forget gate,
 //   S_N = alpha S_{N-1} + sum over chunks (in chunk order) of dS,
 // then the copies the attention and update kernels read: Sb = bf16(S_N)
-// and Mt = (W_q S_N)^T in bf16.  One CTA: 8 columns n0..n0+7 of S of one
+// and Mt = (W_q S_N)^T in bf16.  One CTA: 4 columns n0..n0+3 of S of one
 // (stream, head), 128 threads.  Thread r reduces row r of those columns;
 // then thread a forms M[a][n] = sum_c W_q[a][c] S_N[c][n] (c in order, fp32)
-// for the 8 columns, which are whole rows n of Mt.  With n_chunks = 0 and
+// for the 4 columns, which are whole rows n of Mt.  With n_chunks = 0 and
 // no alpha it only derives Sb and Mt from S (a restored state).
-constexpr int kFoldCols = 8;
+constexpr int kFoldCols = 4;
+constexpr int kMaxChunksInFlight = 16;
 __global__ void __launch_bounds__(kD) finalize_fold_kernel(const float* __restrict__ part_s,
                                                            const float* __restrict__ alpha,
                                                            float* __restrict__ S,
@@ -275,71 +276,58 @@ __global__ void __launch_bounds__(kD) finalize_fold_kernel(const float* __restri
                                                            __nv_bfloat16* __restrict__ Sb, int n_chunks,
                                                            int H) {
     __shared__ __align__(16) float scol[kD][kFoldCols];
-    ptx::pdl_trigger();
-    ptx::pdl_wait();
     const int n0 = blockIdx.x * kFoldCols, h = blockIdx.y, b = blockIdx.z, bh = b * H + h;
     const int r = threadIdx.x;
+    // W_q is fixed for the layer's lifetime: its row is fetched before the
+    // wait for the previous kernel.
+    const uint4* wrow = reinterpret_cast<const uint4*>(wq + ((size_t)h * kD + r) * kD);
+    uint4 w8[kD / 8];
+#pragma unroll
+    for (int c8 = 0; c8 < kD / 8; ++c8) w8[c8] = __ldg(wrow + c8);
+    ptx::pdl_trigger();
+    ptx::pdl_wait();
     const size_t e = (size_t)bh * kD * kD + (size_t)r * kD + n0;
-    float4 s0 = *reinterpret_cast<const float4*>(S + e);
-    float4 s1 = *reinterpret_cast<const float4*>(S + e + 4);
+    float4 s = *reinterpret_cast<const float4*>(S + e);
     if (alpha) {
         const float a = alpha[bh];
-        float4 c0 = make_float4(0.f, 0.f, 0.f, 0.f), c1 = c0;
+        float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
         const size_t pb = (size_t)bh * n_chunks * kD * kD + (size_t)r * kD + n0;
-        // Loads in groups of 8 so that they are in flight together; the sum
-        // itself stays in chunk order.
-        for (int g = 0; g < n_chunks; g += 8) {
-            float4 p[8][2];
+        // loads in flight together; the sum itself in chunk order
+        for (int g = 0; g < n_chunks; g += kMaxChunksInFlight) {
+            float4 p[kMaxChunksInFlight];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (g + i < n_chunks) {
-                    const float4* src = reinterpret_cast<const float4*>(part_s + pb + (size_t)(g + i) * kD * kD);
-                    p[i][0] = __ldcg(src);
-                    p[i][1] = __ldcg(src + 1);
-                }
+            for (int i = 0; i < kMaxChunksInFlight; ++i)
+                if (g + i < n_chunks)
+                    p[i] = __ldcg(reinterpret_cast<const float4*>(part_s + pb + (size_t)(g + i) * kD * kD));
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < kMaxChunksInFlight; ++i)
                 if (g + i < n_chunks) {
-                    c0.x += p[i][0].x; c0.y += p[i][0].y; c0.z += p[i][0].z; c0.w += p[i][0].w;
-                    c1.x += p[i][1].x; c1.y += p[i][1].y; c1.z += p[i][1].z; c1.w += p[i][1].w;
+                    c.x += p[i].x;
+                    c.y += p[i].y;
+                    c.z += p[i].z;
+                    c.w += p[i].w;
                 }
         }
-        s0 = make_float4(fmaf(a, s0.x, c0.x), fmaf(a, s0.y, c0.y), fmaf(a, s0.z, c0.z), fmaf(a, s0.w, c0.w));
-        s1 = make_float4(fmaf(a, s1.x, c1.x), fmaf(a, s1.y, c1.y), fmaf(a, s1.z, c1.z), fmaf(a, s1.w, c1.w));
-        *reinterpret_cast<float4*>(S + e) = s0;
-        *reinterpret_cast<float4*>(S + e + 4) = s1;
+        s = make_float4(fmaf(a, s.x, c.x), fmaf(a, s.y, c.y), fmaf(a, s.z, c.z), fmaf(a, s.w, c.w));
+        *reinterpret_cast<float4*>(S + e) = s;
     }
-    uint4 sb;
-    sb.x = ptx::pack_bf16x2(s0.x, s0.y);
-    sb.y = ptx::pack_bf16x2(s0.z, s0.w);
-    sb.z = ptx::pack_bf16x2(s1.x, s1.y);
-    sb.w = ptx::pack_bf16x2(s1.z, s1.w);
-    *reinterpret_cast<uint4*>(Sb + e) = sb;
-    *reinterpret_cast<float4*>(&scol[r][0]) = s0;
-    *reinterpret_cast<float4*>(&scol[r][4]) = s1;
+    *reinterpret_cast<uint2*>(Sb + e) = make_uint2(ptx::pack_bf16x2(s.x, s.y), ptx::pack_bf16x2(s.z, s.w));
+    *reinterpret_cast<float4*>(&scol[r][0]) = s;
     __syncthreads();
     // M[a][n0 + j] = sum_c W_q[a][c] S_N[c][n0 + j]; thread a = r
-    const uint4* wrow = reinterpret_cast<const uint4*>(wq + ((size_t)h * kD + r) * kD);
-    float acc[kFoldCols];
+    float acc[kFoldCols] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int j = 0; j < kFoldCols; ++j) acc[j] = 0.f;
     for (int c8 = 0; c8 < kD / 8; ++c8) {
-        const uint4 w8 = __ldg(wrow + c8);
-        const uint32_t wv[4] = {w8.x, w8.y, w8.z, w8.w};
+        const uint32_t wv[4] = {w8[c8].x, w8[c8].y, w8[c8].z, w8[c8].w};
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const uint32_t pr = wv[k >> 1];
             const float w = __uint_as_float((k & 1) ? (pr & 0xffff0000u) : (pr << 16));
-            const float4 x0 = *reinterpret_cast<const float4*>(&scol[c8 * 8 + k][0]);
-            const float4 x1 = *reinterpret_cast<const float4*>(&scol[c8 * 8 + k][4]);
-            acc[0] = fmaf(w, x0.x, acc[0]);
-            acc[1] = fmaf(w, x0.y, acc[1]);
-            acc[2] = fmaf(w, x0.z, acc[2]);
-            acc[3] = fmaf(w, x0.w, acc[3]);
-            acc[4] = fmaf(w, x1.x, acc[4]);
-            acc[5] = fmaf(w, x1.y, acc[5]);
-            acc[6] = fmaf(w, x1.z, acc[6]);
-            acc[7] = fmaf(w, x1.w, acc[7]);
+            const float4 x = *reinterpret_cast<const float4*>(&scol[c8 * 8 + k][0]);
+            acc[0] = fmaf(w, x.x, acc[0]);
+            acc[1] = fmaf(w, x.y, acc[1]);
+            acc[2] = fmaf(w, x.z, acc[2]);
+            acc[3] = fmaf(w, x.w, acc[3]);
         }
     }
 #pragma unroll
