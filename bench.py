@@ -135,11 +135,18 @@ def barrier(ws):
 
 
 def max_over_ranks(x: float, ws: int) -> float:
+    """The slowest rank's time (NCCL on the GPU; gloo keeps the tensor on the host)."""
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(frames_per_rank: int, ws: int, t_max_ms: float) -> float:
+    """Frames per second of the whole job: every rank's frames over the slowest rank's time."""
+    return frames_per_rank * ws / (t_max_ms / 1e3)
 
 
 # -------------------------------------------------------------- CPU side --
@@ -362,8 +369,7 @@ def main():
     if status != 0:
         raise SystemExit(f"device status {status}")
     t_max = max_over_ranks(elapsed_ms, ws)
-    frames_total = args.steps * w.frames * w.batch * ws
-    value = frames_total / (t_max / 1e3)
+    value = whole_job_rate(args.steps * w.frames * w.batch, ws, t_max)
     del graphs
 
     # Fused-kernel duration: the same steps again, with an event pair around
