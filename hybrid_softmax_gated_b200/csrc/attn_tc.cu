@@ -154,7 +154,7 @@ struct __align__(1024) Smem {
     // runs more than one phase ahead of its waiter.
     uint64_t s_full[2];  // one commit: S of the buffer's block is in TMEM
     uint64_t p_full[2];  // 4 warp arrivals: P written over S (and O_b rescaled)
-    uint64_t seg_done;   // one commit per segment: its last UMMA is done
+    uint64_t drain;      // the issuer's last commit before it gives up after a failed wait
     uint64_t o_free;     // 8 warp arrivals per segment: O_0, O_1 and O_inter read out
     uint64_t ebar;       // 8 warp arrivals: epilogue exchange of row maxima and sums
     uint64_t stage_free[2];  // 1 arrival per segment: the Q slot used as output staging is free
@@ -187,6 +187,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort = &sm.abort;
     const int no_abort = 0;
     const CtaRange rng = cta_range(sch, blockIdx.x);
+    if (threadIdx.x == 0 && rng.n_segs > 0) {
+        // Warm L2 with the first tiles this CTA reads (Q, K_0, K_1, V_0) while
+        // the previous kernel may still be running: only a hint, the loads
+        // proper follow the wait for that kernel.
+        const Seg sg = seg_at(sch, rng, 0);
+        const int bh = sg.tile / sch.n_q, qt = sg.tile - bh * sch.n_q;
+        const int b = bh / H, h = bh - b * H;
+        for (int half = 0; half < 2; ++half) {
+            ptx::tma_prefetch_l2_4d(&tm_q, half * 64, h, qt * kBM, b);
+            ptx::tma_prefetch_l2_4d(&tm_v, half * 64, h, sg.kv0 * kBN, b);
+            for (int i = 0; i < 2 && sg.kv0 + i < sg.kv1; ++i)
+                ptx::tma_prefetch_l2_4d(&tm_k, half * 64, h, (sg.kv0 + i) * kBN, b);
+        }
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
@@ -201,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(ptx::smem_u32(&sm.stage_free[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sm.staged[s]), kSoftmaxWarps);
         }
-        ptx::mbar_init(ptx::smem_u32(&sm.seg_done), 1);
+        ptx::mbar_init(ptx::smem_u32(&sm.drain), 1);
         ptx::mbar_init(ptx::smem_u32(&sm.o_free), kSoftmaxWarps);
         ptx::mbar_init(ptx::smem_u32(&sm.ebar), kSoftmaxWarps);
         ptx::mbar_init(ptx::smem_u32(&sm.head_ready), 1);
@@ -226,12 +240,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicOr(err, kErrTimeoutAttn);
         *abort = 1;
     };
-    auto bwait = [&](uint64_t* bar, uint32_t parity) {
-        return ptx::mbar_wait_bounded(ptx::smem_u32(bar), parity, abort, kWaitLimitNs);
-    };
-    // bounded wait with a warp-uniform result (for the full-warp roles)
+    // bounded wait with a warp-uniform result (every role runs as whole warps)
     auto wwait = [&](uint64_t* bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, bwait(bar, parity));
+        return ptx::mbar_wait_warp(ptx::smem_u32(bar), parity, abort, kWaitLimitNs);
     };
 
     if (warp < 4) ptx::setmaxnreg_dec<kRegsLow>();
@@ -243,10 +254,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tma_prefetch_desc(&tm_v);
         ptx::tma_prefetch_desc(&tm_m);
         int kc = 0, vc = 0;  // ring counters (same sequence as the UMMA issuer)
+        // A K slot is free again once its previous item is consumed: a key
+        // block is released by the softmax warpgroup that saw its S (k_empty,
+        // one phase per key block in the slot), the (W_q S)^T tile by the
+        // commit after O_inter (q_empty of its segment).
+        int m_seg0 = -1, m_seg1 = -1;  // segment whose (W_q S)^T tile is in slot 0 / 1, or -1
+        uint32_t kr_par = 0;            // bit s: parity of the next k_empty[s] phase
+        int si = 0;
         bool ok = true;
         auto load_k = [&](int b, int h, int kv) -> bool {  // kv < 0: the (W_q S)^T tile
             const int s = kc & 1;
-            if (kc >= 2 && !wwait(&sm.k_empty[s], ((kc >> 1) - 1) & 1)) return false;
+            const int m_seg = s ? m_seg1 : m_seg0;
+            if (kc >= 2) {
+                bool w;
+                if (m_seg >= 0) {
+                    w = wwait(&sm.q_empty[m_seg & 1], (m_seg >> 1) & 1);
+                } else {
+                    w = wwait(&sm.k_empty[s], (kr_par >> s) & 1);
+                    kr_par ^= 1u << s;
+                }
+                if (!w) return false;
+            }
+            if (s)
+                m_seg1 = kv < 0 ? si : -1;
+            else
+                m_seg0 = kv < 0 ? si : -1;
             const uint32_t bar = ptx::smem_u32(&sm.k_full[s]), dst = ptx::smem_u32(sm.k[s]);
             ptx::mbar_arrive_expect_tx_w(bar, kTileBytes);
             if (kv >= 0) {
@@ -269,7 +301,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++vc;
             return true;
         };
-        int si = 0;
         for (; ok && si < rng.n_segs; ++si) {
             const Seg sg = seg_at(sch, rng, si);
             const int bh = sg.tile / sch.n_q, qt = sg.tile - bh * sch.n_q;
@@ -347,16 +378,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (i < n) {
                     const int valid = valid_keys(L, sg.kv0 + i);
                     const uint32_t idesc = ptx::idesc_bf16_f32(kBM, (valid + 15) & ~15, false, false);
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk)
-                        ptx::umma_f16_ss_w(d, kmajor_desc(q_s, kk), kmajor_desc(k_s, kk), idesc, kk > 0);
+                    ptx::umma_ss8_kk(d, kmajor_desc(q_s, 0), kmajor_desc(k_s, 0), idesc, 0u);
                     ptx::umma_commit_w(ptx::smem_u32(&sm.s_full[buf]));
+                    // a head piece's last use of Q (once per CTA at most)
+                    if (sg.kind == kHead && i == n - 1) ptx::umma_commit_w(ptx::smem_u32(&sm.q_empty[qs]));
                 } else {
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk)
-                        ptx::umma_f16_ss_w(d, kmajor_desc(q_s, kk), kmajor_desc(k_s, kk), idesc_qm, kk > 0);
+                    // O_inter: the last use of Q and of the (W_q S)^T tile
+                    ptx::umma_ss8_kk(d, kmajor_desc(q_s, 0), kmajor_desc(k_s, 0), idesc_qm, 0u);
+                    ptx::umma_commit_w(ptx::smem_u32(&sm.q_empty[qs]));
                 }
-                ptx::umma_commit_w(ptx::smem_u32(&sm.k_empty[s]));
                 ++kc;
                 return true;
             };
@@ -374,13 +404,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t o_t = tmem + kColO + (uint32_t)buf * kD;
                 const uint32_t v_s = ptx::smem_u32(sm.v[vs]);
                 const uint32_t acc0 = j >= 2 ? 1u : 0u;
-                // O_b += P V, P from TMEM.  The full-block case is unrolled: the
-                // issue rate of a single thread depends on a tight sequence.
+                // O_b += P V, P from TMEM.  A full block is one short issue
+                // sequence (the issue rate of a single warp bounds the tensor pipe).
                 if (ksteps == kBN / 16) {
-#pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)
-                        ptx::umma_f16_ts_w(o_t, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv,
-                                           kk > 0 ? 1u : acc0);
+                    ptx::umma_ts8_mn(o_t, p_t, mnmajor_desc(v_s, 0), idesc_pv, acc0);
                 } else {
                     for (int kk = 0; kk < ksteps; ++kk)
                         ptx::umma_f16_ts_w(o_t, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv,
@@ -392,16 +419,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (j + 2 < nk) ok = issue_item(j + 2);
             }
             if (!ok) break;
-            ptx::umma_commit_w(ptx::smem_u32(&sm.q_empty[qs]));
-            ptx::umma_commit_w(ptx::smem_u32(&sm.seg_done));
             prev_oi_buf = sg.kind != kHead ? (vb + n) & 1 : -1;
             vb += nk;
         }
         if (!ok) {
             fail();
             // nothing may still run on the tensor cores when TMEM is released
-            ptx::umma_commit_w(ptx::smem_u32(&sm.seg_done));
-            ptx::mbar_wait_bounded(ptx::smem_u32(&sm.seg_done), si & 1, &no_abort, kWaitLimitNs);
+            ptx::umma_commit_w(ptx::smem_u32(&sm.drain));
+            ptx::mbar_wait_bounded(ptx::smem_u32(&sm.drain), 0, &no_abort, kWaitLimitNs);
         }
     } else if (warp == 3) {
         // ------------------------------------------- epilogue helper --
@@ -453,6 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sbuf = tmem + lane_base + kColS + (uint32_t)wg * kBN;
         const uint32_t obuf = tmem + lane_base + kColO + (uint32_t)wg * kD;
         int vb = 0;                  // virtual blocks so far (see the issuer)
+        int kc0 = 0, vc0 = 0;        // K-ring items and P V products before this segment
         uint32_t s_par = 0;          // phase parity of s_full[wg] to wait for
         uint32_t e_uses = 0;         // completed uses of ebar
         bool ok = true;
@@ -466,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // all 8 softmax warps meet at ebar (arrive, then a bounded wait)
         auto meet_e = [&]() -> bool {
             warp_arrive(&sm.ebar);
-            return __all_sync(0xffffffffu, bwait(&sm.ebar, (e_uses++) & 1));
+            return wwait(&sm.ebar, (e_uses++) & 1);
         };
         const float2 sl2 = make_float2(scale_log2, scale_log2);
         for (int si = 0; ok && si < rng.n_segs; ++si) {
@@ -476,9 +502,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // this warpgroup's blocks of the segment: j = j0, j0 + 2, ...
             const int j0 = ((vb & 1) == wg) ? 0 : 1;
             for (int j = j0; j < n; j += 2) {
-                ok = __all_sync(0xffffffffu, bwait(&sm.s_full[wg], s_par));
+                ok = wwait(&sm.s_full[wg], s_par);
                 s_par ^= 1u;
                 if (!ok) break;
+                // S is done: the K tile it was computed from may be reloaded
+                if ((warp & 3) == 0 && lane == 0) ptx::mbar_arrive(ptx::smem_u32(&sm.k_empty[(kc0 + j) & 1]));
                 ptx::tc_fence_after();
                 uint32_t raw[4][32];
 #pragma unroll
@@ -567,7 +595,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float a0 = has0 ? ptx::ex2(m0 - m_seg) : 0.f;
             const float a1 = has1 ? ptx::ex2(m1 - m_seg) : 0.f;
             const float l_seg = a0 * l0 + a1 * l1;
-            ok = __all_sync(0xffffffffu, bwait(&sm.seg_done, si & 1));
+            // the segment's last P V: its commit covers every product before it
+            ok = wwait(&sm.v_empty[(vc0 + n - 1) & 1], ((vc0 + n - 1) >> 1) & 1);
             if (!ok) break;
             ptx::tc_fence_after();
             // this warpgroup's output columns [64 wg, 64 wg + 64) of
@@ -612,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (sg.kind == kTail) {
                     // the head piece of this tile was written by the previous CTA
                     // at its start; warp 3 has acquired its flag
-                    ok = __all_sync(0xffffffffu, bwait(&sm.head_ready, 0));
+                    ok = wwait(&sm.head_ready, 0);
                     if (!ok) break;
                     const float2 ml = __ldcg(reinterpret_cast<const float2*>(
                         part_ml + ((size_t)sg.tile * kBM + row) * 2));
@@ -664,6 +693,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_before();
             warp_arrive(&sm.o_free);
             vb += n + (sg.kind != kHead ? 1 : 0);
+            kc0 += n + (sg.kind != kHead ? 1 : 0);
+            vc0 += n;
         }
         if (!ok) fail();
     }

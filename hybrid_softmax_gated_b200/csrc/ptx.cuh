@@ -61,6 +61,20 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// Warp-uniform bounded wait: every lane of a converged warp calls it with
+// the same arguments and gets the same answer.  The fast path is one
+// try_wait per lane and one vote, with no divergent branch (a per-lane wait
+// loop followed by a vote costs a reconvergence on every call).
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const volatile int* abort,
+                                               uint64_t limit_ns) {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+        if (__any_sync(0xffffffffu, *abort != 0 || globaltimer_ns() - t0 > limit_ns)) return false;
+    }
+}
+
 // ---- proxies and fences ---------------------------------------------------
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor core operand reads).
@@ -200,6 +214,15 @@ __device__ __forceinline__ void tma_load_4d_w(uint32_t dst, const CUtensorMap* m
         " [%0], [%1, {%2, %3, %4, %5}], [%6];\n\t}" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
         : "memory");
+}
+
+// L2 prefetch of a TMA tile (a hint: no shared memory is written and no
+// completion is tracked).
+__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* m, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
 }
 
 // ---- tcgen05: TMEM <-> registers (32 lanes x 32 columns of 32 bit) --------
@@ -431,6 +454,72 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
 // 64-wide halves 16 KB apart): k-step kk starts 16 rows = 2048 bytes on.
 __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk) {
     return sdesc_sw128(tile + (uint32_t)kk * 2048u, kHalfBytes, 1024u);
+}
+
+// ---- eight k-steps of a 128x128x128 product in one issue sequence ---------
+// One elected lane issues all eight MMAs of a 128-deep product.  The
+// descriptors of k-step kk differ from those of step 0 only in the
+// start-address field (bits 0-13 of the low word, address >> 4), and
+// shared-memory addresses stay below 2^18 so that the field never carries:
+// the steps are plain 32-bit adds on the low word.
+//   K-major SW128 operand: + ((kk >> 2) * 16 KB + (kk & 3) * 32 B) >> 4
+//   MN-major SW128 operand: + (kk * 2048 B) >> 4
+// acc0 is the accumulate flag of the first step (the others accumulate).
+__device__ __forceinline__ void umma_ss8_kk(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                            uint32_t acc0) {
+    const uint32_t alo = (uint32_t)a0, ahi = (uint32_t)(a0 >> 32);
+    const uint32_t blo = (uint32_t)b0, bhi = (uint32_t)(b0 >> 32);
+    asm volatile(
+        "{\n\t.reg .pred e, p, one;\n\t.reg .b64 a, b;\n\t.reg .b32 x, y;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "setp.eq.b32 one, %6, %6;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "mov.b64 a, {%1, %2};\n\tmov.b64 b, {%3, %4};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, p;\n\t"
+        "add.u32 x, %1, 2;\n\tadd.u32 y, %3, 2;\n\tmov.b64 a, {x, %2};\n\tmov.b64 b, {y, %4};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, one;\n\t"
+        "add.u32 x, %1, 4;\n\tadd.u32 y, %3, 4;\n\tmov.b64 a, {x, %2};\n\tmov.b64 b, {y, %4};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, one;\n\t"
+        "add.u32 x, %1, 6;\n\tadd.u32 y, %3, 6;\n\tmov.b64 a, {x, %2};\n\tmov.b64 b, {y, %4};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, one;\n\t"
+        "add.u32 x, %1, 1024;\n\tadd.u32 y, %3, 1024;\n\tmov.b64 a, {x, %2};\n\tmov.b64 b, {y, %4};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, one;\n\t"
+        "add.u32 x, %1, 1026;\n\tadd.u32 y, %3, 1026;\n\tmov.b64 a, {x, %2};\n\tmov.b64 b, {y, %4};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, one;\n\t"
+        "add.u32 x, %1, 1028;\n\tadd.u32 y, %3, 1028;\n\tmov.b64 a, {x, %2};\n\tmov.b64 b, {y, %4};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, one;\n\t"
+        "add.u32 x, %1, 1030;\n\tadd.u32 y, %3, 1030;\n\tmov.b64 a, {x, %2};\n\tmov.b64 b, {y, %4};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, one;\n\t}" ::"r"(d_tmem),
+        "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "r"(idesc), "r"(acc0)
+        : "memory");
+}
+// A from TMEM (a_tmem, 8 columns of bf16 pairs per k-step), B MN-major.
+__device__ __forceinline__ void umma_ts8_mn(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0, uint32_t idesc,
+                                            uint32_t acc0) {
+    const uint32_t blo = (uint32_t)b0, bhi = (uint32_t)(b0 >> 32);
+    asm volatile(
+        "{\n\t.reg .pred e, p, one;\n\t.reg .b64 b;\n\t.reg .b32 t, y;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "setp.eq.b32 one, %5, %5;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "mov.b64 b, {%2, %3};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b, %4, p;\n\t"
+        "add.u32 t, %1, 8;\n\tadd.u32 y, %2, 128;\n\tmov.b64 b, {y, %3};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, one;\n\t"
+        "add.u32 t, %1, 16;\n\tadd.u32 y, %2, 256;\n\tmov.b64 b, {y, %3};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, one;\n\t"
+        "add.u32 t, %1, 24;\n\tadd.u32 y, %2, 384;\n\tmov.b64 b, {y, %3};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, one;\n\t"
+        "add.u32 t, %1, 32;\n\tadd.u32 y, %2, 512;\n\tmov.b64 b, {y, %3};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, one;\n\t"
+        "add.u32 t, %1, 40;\n\tadd.u32 y, %2, 640;\n\tmov.b64 b, {y, %3};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, one;\n\t"
+        "add.u32 t, %1, 48;\n\tadd.u32 y, %2, 768;\n\tmov.b64 b, {y, %3};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, one;\n\t"
+        "add.u32 t, %1, 56;\n\tadd.u32 y, %2, 896;\n\tmov.b64 b, {y, %3};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, one;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(blo), "r"(bhi), "r"(idesc), "r"(acc0)
+        : "memory");
 }
 
 // Byte offset of the 16-byte chunk c16 (0..15 along a 128-element bf16

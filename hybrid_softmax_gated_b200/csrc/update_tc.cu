@@ -102,6 +102,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto wait = [&](uint64_t* bar) {
         return ptx::mbar_wait_bounded(ptx::smem_u32(bar), 0, abort, kWaitLimitNs);
     };
+    // warp-uniform variant for code run by whole warps
+    auto wwait = [&](uint64_t* bar) {
+        return ptx::mbar_wait_warp(ptx::smem_u32(bar), 0, abort, kWaitLimitNs);
+    };
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------ TMA producer --
@@ -173,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float beta_t = t < L ? beta[(size_t)bh * L + t] : 0.f;
         const uint32_t xk = ptx::smem_u32(sm.xk), xv = ptx::smem_u32(sm.xv);
         const size_t part_row = (((size_t)bh * n_chunks + chunk) * kD + r) * kD;
-        bool ok = __all_sync(0xffffffffu, wait(&sm.proj));
+        bool ok = wwait(&sm.proj);
         if (ok) {
             // K' = Kp / max(|Kp|, 1e-6) -> bf16 into xk (the K tile is consumed)
             ptx::tc_fence_after();
@@ -201,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             ptx::mbar_arrive(ptx::smem_u32(&sm.kp_ready));
-            ok = __all_sync(0xffffffffu, wait(&sm.ks));
+            ok = wwait(&sm.ks);
         }
         if (ok) {
             // beta R = beta (Vp - K' S) -> bf16 into xv (the V tile is consumed)
@@ -228,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             ptx::mbar_arrive(ptx::smem_u32(&sm.r_ready));
-            ok = __all_sync(0xffffffffu, wait(&sm.ds));
+            ok = wwait(&sm.ds);
         }
         if (ok) {
             // dS row r (key feature r): fp32 partial out
