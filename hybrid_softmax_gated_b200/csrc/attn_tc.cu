@@ -63,6 +63,7 @@
 #include <cmath>
 #include <cstring>
 #include <new>
+#include <type_traits>
 
 namespace arl2 {
 namespace {
@@ -187,21 +188,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort = &sm.abort;
     const int no_abort = 0;
     const CtaRange rng = cta_range(sch, blockIdx.x);
-    if (threadIdx.x == 0 && rng.n_segs > 0) {
-        // Warm L2 with the first tiles this CTA reads (Q, K_0, K_1, V_0) while
-        // the previous kernel may still be running: only a hint, the loads
-        // proper follow the wait for that kernel.
-        const Seg sg = seg_at(sch, rng, 0);
-        const int bh = sg.tile / sch.n_q, qt = sg.tile - bh * sch.n_q;
-        const int b = bh / H, h = bh - b * H;
-        for (int half = 0; half < 2; ++half) {
-            ptx::tma_prefetch_l2_4d(&tm_q, half * 64, h, qt * kBM, b);
-            ptx::tma_prefetch_l2_4d(&tm_v, half * 64, h, sg.kv0 * kBN, b);
-            for (int i = 0; i < 2 && sg.kv0 + i < sg.kv1; ++i)
-                ptx::tma_prefetch_l2_4d(&tm_k, half * 64, h, (sg.kv0 + i) * kBN, b);
-        }
-    }
-
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(ptx::smem_u32(&sm.q_full[s]), 1);
@@ -231,10 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    // The next kernel may launch now and run its own set-up; nothing of this
-    // kernel touches global memory before the previous kernel has finished.
+    // The next kernel may launch now and run its own set-up.  Nothing of this
+    // kernel touches global memory before the previous kernel has finished:
+    // every role starts with that wait (griddepcontrol.wait).
     ptx::pdl_trigger();
-    ptx::pdl_wait();
 
     auto fail = [&]() {
         atomicOr(err, kErrTimeoutAttn);
@@ -245,10 +231,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         return ptx::mbar_wait_warp(ptx::smem_u32(bar), parity, abort, kWaitLimitNs);
     };
 
+    // Warpgroup 0 (producer, issuer, allocator, helper) hands registers to
+    // the two softmax warpgroups, before it has any asynchronous copy in
+    // flight (the hand-off would wait for those).
     if (warp < 4) ptx::setmaxnreg_dec<kRegsLow>();
     if (warp == 0) {
         // (the whole warp runs the producer; one elected lane issues)
         // ------------------------------------------------ TMA producer --
+        ptx::pdl_wait();
         ptx::tma_prefetch_desc(&tm_q);
         ptx::tma_prefetch_desc(&tm_k);
         ptx::tma_prefetch_desc(&tm_v);
@@ -339,6 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // (the whole warp runs the issuer; one elected lane issues)
         // ------------------------------------------------- UMMA issuer --
+        ptx::pdl_wait();
         const uint32_t idesc_pv = ptx::idesc_bf16_f32(kBM, kD, false, true);  // V: MN-major
         const uint32_t idesc_qm = ptx::idesc_bf16_f32(kBM, kD, false, false);
         int kc = 0, vc = 0;
@@ -430,6 +421,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 3) {
         // ------------------------------------------- epilogue helper --
+        if (lane == 0 && rng.n_segs > 0) {
+            // Warm L2 with the first tiles this CTA reads (Q, K_0, K_1, V_0) while
+            // the previous kernel may still be running: only a hint, the loads
+            // proper follow the wait for that kernel.  (After the register
+            // hand-off, which would otherwise wait for these to complete.)
+            const Seg sg = seg_at(sch, rng, 0);
+            const int bh = sg.tile / sch.n_q, qt = sg.tile - bh * sch.n_q;
+            const int b = bh / H, h = bh - b * H;
+            for (int half = 0; half < 2; ++half) {
+                ptx::tma_prefetch_l2_4d(&tm_q, half * 64, h, qt * kBM, b);
+                ptx::tma_prefetch_l2_4d(&tm_v, half * 64, h, sg.kv0 * kBN, b);
+                for (int i = 0; i < 2 && sg.kv0 + i < sg.kv1; ++i)
+                    ptx::tma_prefetch_l2_4d(&tm_k, half * 64, h, (sg.kv0 + i) * kBN, b);
+            }
+        }
+        __syncwarp();
+        ptx::pdl_wait();
         bool ok = true;
         for (int si = 0; ok && si < rng.n_segs; ++si) {
             const Seg sg = seg_at(sch, rng, si);
@@ -472,6 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= 4) {
         // ---------------------------------------- softmax + epilogue --
         ptx::setmaxnreg_inc<kRegsHigh>();
+        ptx::pdl_wait();
         const int wg = (warp - 4) >> 2;               // S/P buffer, O accumulator and key blocks
         const int row = ((warp & 3) << 5) + lane;     // tile row = TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -602,15 +611,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             // this warpgroup's output columns [64 wg, 64 wg + 64) of
             // a0 O_0 + a1 O_1 (unnormalised, against m_seg)
             const uint32_t ocol = tmem + lane_base + kColO + (uint32_t)wg * 64;
-            auto load_acc = [&](int c, float (&acc)[32]) {
+            // a0 O_0 + a1 O_1 over 32 columns, and (with_oi) O_inter's, in one round trip
+            auto load_acc = [&](int c, float (&acc)[32], auto with_oi, uint32_t oi_col, uint32_t (&oi)[32]) {
                 // (a warpgroup without blocks in this segment left its O stale:
                 // it is loaded but not used)
                 uint32_t o0[32], o1[32];
                 ptx::tmem_ld32(ocol + (uint32_t)c * 32, o0);
                 ptx::tmem_ld32(ocol + kD + (uint32_t)c * 32, o1);
+                if constexpr (decltype(with_oi)::value) ptx::tmem_ld32(oi_col + (uint32_t)c * 32, oi);
                 ptx::tmem_wait_ld();
                 ptx::reg_fence(o0);
                 ptx::reg_fence(o1);
+                if constexpr (decltype(with_oi)::value) ptx::reg_fence(oi);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const float v0 = has0 ? a0 * __uint_as_float(o0[i]) : 0.f;
@@ -625,7 +637,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     float acc[32];
-                    load_acc(c, acc);
+                    uint32_t unused[32];
+                    load_acc(c, acc, std::false_type{}, 0u, unused);
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
                         pbase[(size_t)(c * 8 + i) * kBM] =
@@ -655,11 +668,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     float acc[32];
-                    load_acc(c, acc);
                     uint32_t oi[32];
-                    ptx::tmem_ld32(oi_col + (uint32_t)c * 32, oi);
-                    ptx::tmem_wait_ld();
-                    ptx::reg_fence(oi);
+                    load_acc(c, acc, std::true_type{}, oi_col, oi);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) acc[i] *= a_t;
                     if (sg.kind == kTail) {
