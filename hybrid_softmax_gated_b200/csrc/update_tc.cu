@@ -9,15 +9,17 @@
 //   K' = rownorm(K W_k),  V' = V W_v.
 //
 // The sum over the frame's tokens splits into 128-token chunks that are
-// independent given S_{N-1}.  update_chunk_kernel (one CTA per chunk, head
-// and stream) computes, on tcgen05 with fp32 accumulators in TMEM:
+// independent given S_{N-1}.  update_chunk_kernel (one CTA per two chunks of
+// one head and stream) computes for each chunk, on tcgen05 with fp32
+// accumulators in TMEM:
 //   Kp = K W_k, Vp = V W_v                     (bf16 x bf16)
 //   K' = Kp / max(|Kp|, 1e-6)  -> bf16 tile    (epilogue)
 //   KS = K' S_{N-1}                            (S_{N-1} as bf16)
 //   beta R = beta (Vp - KS)    -> bf16 tile    (epilogue)
 //   dS = K'^T (beta R)                         (the same K' tile read MN-major)
-// and writes dS as an fp32 partial.  finalize_fold_kernel sums the
-// partials in chunk order (deterministic) and applies the forget gate,
+// and writes the two chunks' dS (summed in TMEM) as one fp32 partial.
+// finalize_fold_kernel sums the partials in order (deterministic) and
+// applies the forget gate,
 //   S_N = alpha S_{N-1} + sum dS,
 // and derives from S_N alone the bf16 copy of S and Mt = (W_q S_N)^T, the
 // matrix the attention kernel reads (so that the inter-frame read
@@ -43,23 +45,34 @@ using ptx::mnmajor_desc;
 
 constexpr int kD = 128;
 constexpr int kChunk = 128;
-constexpr int kThreads = 256;
+constexpr int kChunksPerCta = 2;
+constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColKp = 0, kColVp = 128, kColKS = 256, kColDS = 384;
+// TMEM columns per chunk c (0, 1): Kp then KS at 256 c, Vp at 256 c + 128;
+// dS of both chunks accumulates over chunk 0's Vp once that is consumed.
+constexpr uint32_t kColDS = 128;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
 struct __align__(1024) Smem {
-    uint8_t xk[kTileBytes];  // K chunk -> K' (bf16)
-    uint8_t xv[kTileBytes];  // V chunk -> beta R (bf16)
-    uint8_t wk[kTileBytes];  // W_k[h], rows = input feature
-    uint8_t wv[kTileBytes];  // W_v[h]
-    uint8_t sb[kTileBytes];  // S_{N-1} bf16, rows = key feature
-    uint64_t ld_k, ld_v, proj, kp_ready, ks, r_ready, ds;
+    uint8_t xk[kChunksPerCta][kTileBytes];  // K chunk -> K' (bf16)
+    uint8_t xv[kChunksPerCta][kTileBytes];  // V chunk -> beta R (bf16)
+    uint8_t wk[kTileBytes];                 // W_k[h], rows = input feature
+    uint8_t wv[kTileBytes];                 // W_v[h]
+    uint8_t sb[kTileBytes];                 // S_{N-1} bf16, rows = key feature
+    uint64_t ld_k[kChunksPerCta];  // K tile of the chunk (and W_k with chunk 0)
+    uint64_t ld_v[kChunksPerCta];  // V tile of the chunk (and W_v, S with chunk 0)
+    uint64_t proj[kChunksPerCta];  // Kp, Vp of the chunk in TMEM
+    uint64_t kp_ready[kChunksPerCta], ks[kChunksPerCta], r_ready[kChunksPerCta];
+    uint64_t ds;                   // dS of both chunks in TMEM
     uint32_t tmem_base;
     int abort;
 };
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 
+// One CTA: chunks 2 p and 2 p + 1 of one (stream, head).  Warps 4-7 run
+// chunk 0's epilogue steps and warps 8-11 chunk 1's, so the two dependent
+// chains overlap; W_k, W_v and S are loaded once.  A chunk past the frame's
+// end is all zeros after the (zero-filled) loads and adds nothing to dS.
 __global__ void __launch_bounds__(kThreads, 1)
     update_chunk_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sb,
@@ -69,17 +82,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                         ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int n_chunks = gridDim.x;
+    const int pair = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int n_parts = gridDim.x;
     const int bh = b * H + h;
     volatile int* abort = &sm.abort;
     const int no_abort = 0;
 
     if (threadIdx.x == 0) {
-        uint64_t* bars[] = {&sm.ld_k, &sm.ld_v, &sm.proj, &sm.ks, &sm.ds};
-        for (uint64_t* p : bars) ptx::mbar_init(ptx::smem_u32(p), 1);
-        ptx::mbar_init(ptx::smem_u32(&sm.kp_ready), 128);
-        ptx::mbar_init(ptx::smem_u32(&sm.r_ready), 128);
+        for (int c = 0; c < kChunksPerCta; ++c) {
+            ptx::mbar_init(ptx::smem_u32(&sm.ld_k[c]), 1);
+            ptx::mbar_init(ptx::smem_u32(&sm.ld_v[c]), 1);
+            ptx::mbar_init(ptx::smem_u32(&sm.proj[c]), 1);
+            ptx::mbar_init(ptx::smem_u32(&sm.ks[c]), 1);
+            ptx::mbar_init(ptx::smem_u32(&sm.kp_ready[c]), 128);
+            ptx::mbar_init(ptx::smem_u32(&sm.r_ready[c]), 128);
+        }
+        ptx::mbar_init(ptx::smem_u32(&sm.ds), 1);
         sm.abort = 0;
         ptx::fence_mbar_init();
         ptx::fence_proxy_async_smem();
@@ -109,59 +127,80 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------ TMA producer --
-        const int t0 = chunk * kChunk;
-        const uint32_t bk = ptx::smem_u32(&sm.ld_k), bv = ptx::smem_u32(&sm.ld_v);
-        ptx::mbar_arrive_expect_tx(bk, 2 * kTileBytes);
-        ptx::tma_load_4d(ptx::smem_u32(sm.xk), &tm_k, 0, h, t0, b, bk);
-        ptx::tma_load_4d(ptx::smem_u32(sm.xk) + kHalfBytes, &tm_k, 64, h, t0, b, bk);
-        ptx::tma_load_4d(ptx::smem_u32(sm.wk), &tm_w, 0, 0, H + h, 0, bk);
-        ptx::tma_load_4d(ptx::smem_u32(sm.wk) + kHalfBytes, &tm_w, 64, 0, H + h, 0, bk);
-        ptx::mbar_arrive_expect_tx(bv, 3 * kTileBytes);
-        ptx::tma_load_4d(ptx::smem_u32(sm.xv), &tm_v, 0, h, t0, b, bv);
-        ptx::tma_load_4d(ptx::smem_u32(sm.xv) + kHalfBytes, &tm_v, 64, h, t0, b, bv);
-        ptx::tma_load_4d(ptx::smem_u32(sm.wv), &tm_w, 0, 0, 2 * H + h, 0, bv);
-        ptx::tma_load_4d(ptx::smem_u32(sm.wv) + kHalfBytes, &tm_w, 64, 0, 2 * H + h, 0, bv);
-        ptx::tma_load_4d(ptx::smem_u32(sm.sb), &tm_sb, 0, 0, bh, 0, bv);
-        ptx::tma_load_4d(ptx::smem_u32(sm.sb) + kHalfBytes, &tm_sb, 64, 0, bh, 0, bv);
+        for (int c = 0; c < kChunksPerCta; ++c) {
+            const int t0 = (pair * kChunksPerCta + c) * kChunk;
+            const uint32_t bk = ptx::smem_u32(&sm.ld_k[c]), bv = ptx::smem_u32(&sm.ld_v[c]);
+            const uint32_t xk = ptx::smem_u32(sm.xk[c]), xv = ptx::smem_u32(sm.xv[c]);
+            ptx::mbar_arrive_expect_tx(bk, (c == 0 ? 2 : 1) * kTileBytes);
+            ptx::tma_load_4d(xk, &tm_k, 0, h, t0, b, bk);
+            ptx::tma_load_4d(xk + kHalfBytes, &tm_k, 64, h, t0, b, bk);
+            if (c == 0) {
+                ptx::tma_load_4d(ptx::smem_u32(sm.wk), &tm_w, 0, 0, H + h, 0, bk);
+                ptx::tma_load_4d(ptx::smem_u32(sm.wk) + kHalfBytes, &tm_w, 64, 0, H + h, 0, bk);
+            }
+            ptx::mbar_arrive_expect_tx(bv, (c == 0 ? 3 : 1) * kTileBytes);
+            ptx::tma_load_4d(xv, &tm_v, 0, h, t0, b, bv);
+            ptx::tma_load_4d(xv + kHalfBytes, &tm_v, 64, h, t0, b, bv);
+            if (c == 0) {
+                ptx::tma_load_4d(ptx::smem_u32(sm.wv), &tm_w, 0, 0, 2 * H + h, 0, bv);
+                ptx::tma_load_4d(ptx::smem_u32(sm.wv) + kHalfBytes, &tm_w, 64, 0, 2 * H + h, 0, bv);
+                ptx::tma_load_4d(ptx::smem_u32(sm.sb), &tm_sb, 0, 0, bh, 0, bv);
+                ptx::tma_load_4d(ptx::smem_u32(sm.sb) + kHalfBytes, &tm_sb, 64, 0, bh, 0, bv);
+            }
+        }
         // The loads have landed before the CTA may exit.
-        ptx::mbar_wait_bounded(bk, 0, &no_abort, kWaitLimitNs);
-        ptx::mbar_wait_bounded(bv, 0, &no_abort, kWaitLimitNs);
+        for (int c = 0; c < kChunksPerCta; ++c) {
+            ptx::mbar_wait_bounded(ptx::smem_u32(&sm.ld_k[c]), 0, &no_abort, kWaitLimitNs);
+            ptx::mbar_wait_bounded(ptx::smem_u32(&sm.ld_v[c]), 0, &no_abort, kWaitLimitNs);
+        }
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------- UMMA issuer --
         constexpr uint32_t id_k_mn = ptx::idesc_bf16_f32(128, 128, false, true);
         constexpr uint32_t id_mn_mn = ptx::idesc_bf16_f32(128, 128, true, true);
-        const uint32_t xk = ptx::smem_u32(sm.xk), xv = ptx::smem_u32(sm.xv);
         const uint32_t wk = ptx::smem_u32(sm.wk), wv = ptx::smem_u32(sm.wv);
         const uint32_t sb = ptx::smem_u32(sm.sb);
-        bool ok = wait(&sm.ld_k);
-        if (ok) {
+        bool ok = true;
+        // Kp = K W_k and Vp = V W_v of both chunks as soon as their tiles land
+        for (int c = 0; ok && c < kChunksPerCta; ++c) {
+            const uint32_t xk = ptx::smem_u32(sm.xk[c]), xv = ptx::smem_u32(sm.xv[c]);
+            const uint32_t col = tmem + 256u * c;
+            ok = wait(&sm.ld_k[c]);
+            if (!ok) break;
             ptx::tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // Kp = K W_k
-                ptx::umma_f16_ss(tmem + kColKp, kmajor_desc(xk, kk), mnmajor_desc(wk, kk), id_k_mn, kk > 0);
-            ok = wait(&sm.ld_v);
+            for (int kk = 0; kk < 8; ++kk)
+                ptx::umma_f16_ss(col, kmajor_desc(xk, kk), mnmajor_desc(wk, kk), id_k_mn, kk > 0);
+            ok = wait(&sm.ld_v[c]);
+            if (!ok) break;
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                ptx::umma_f16_ss(col + 128, kmajor_desc(xv, kk), mnmajor_desc(wv, kk), id_k_mn, kk > 0);
+            ptx::umma_commit(ptx::smem_u32(&sm.proj[c]));
+        }
+        // KS = K' S_{N-1} (into Kp's columns, read out already)
+        for (int c = 0; ok && c < kChunksPerCta; ++c) {
+            ok = wait(&sm.kp_ready[c]);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const uint32_t xk = ptx::smem_u32(sm.xk[c]);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                ptx::umma_f16_ss(tmem + 256u * c, kmajor_desc(xk, kk), mnmajor_desc(sb, kk), id_k_mn, kk > 0);
+            ptx::umma_commit(ptx::smem_u32(&sm.ks[c]));
+        }
+        // dS = sum over both chunks of K'^T (beta R), over chunk 0's Vp columns
+        for (int c = 0; ok && c < kChunksPerCta; ++c) {
+            ok = wait(&sm.r_ready[c]);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const uint32_t xk = ptx::smem_u32(sm.xk[c]), xv = ptx::smem_u32(sm.xv[c]);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                ptx::umma_f16_ss(tmem + kColDS, mnmajor_desc(xk, kk), mnmajor_desc(xv, kk), id_mn_mn,
+                                 (c > 0 || kk > 0) ? 1u : 0u);
         }
         if (ok) {
-            ptx::tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // Vp = V W_v
-                ptx::umma_f16_ss(tmem + kColVp, kmajor_desc(xv, kk), mnmajor_desc(wv, kk), id_k_mn, kk > 0);
-            ptx::umma_commit(ptx::smem_u32(&sm.proj));
-            ok = wait(&sm.kp_ready);
-        }
-        if (ok) {
-            ptx::tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // KS = K' S_{N-1}
-                ptx::umma_f16_ss(tmem + kColKS, kmajor_desc(xk, kk), mnmajor_desc(sb, kk), id_k_mn, kk > 0);
-            ptx::umma_commit(ptx::smem_u32(&sm.ks));
-            ok = wait(&sm.r_ready);
-        }
-        if (ok) {
-            ptx::tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // dS = K'^T (beta R): sum over the chunk's tokens
-                ptx::umma_f16_ss(tmem + kColDS, mnmajor_desc(xk, kk), mnmajor_desc(xv, kk), id_mn_mn, kk > 0);
             ptx::umma_commit(ptx::smem_u32(&sm.ds));
         } else {
             fail();
@@ -171,27 +210,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 4) {
         // --------------------------------------------------- epilogue --
-        const int r = threadIdx.x - 128;  // TMEM lane = tile row
+        const int c = (warp - 4) >> 2;     // chunk of this warpgroup
+        const int r = threadIdx.x & 127;   // TMEM lane = token row of the chunk, then dS row
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const int t = chunk * kChunk + r;
+        const uint32_t col = tmem + lane_base + 256u * c;
+        const int t = (pair * kChunksPerCta + c) * kChunk + r;
         const float beta_t = t < L ? beta[(size_t)bh * L + t] : 0.f;
-        const uint32_t xk = ptx::smem_u32(sm.xk), xv = ptx::smem_u32(sm.xv);
-        const size_t part_row = (((size_t)bh * n_chunks + chunk) * kD + r) * kD;
-        bool ok = wwait(&sm.proj);
+        const uint32_t xk = ptx::smem_u32(sm.xk[c]), xv = ptx::smem_u32(sm.xv[c]);
+        bool ok = wwait(&sm.proj[c]);
         if (ok) {
             // K' = Kp / max(|Kp|, 1e-6) -> bf16 into xk (the K tile is consumed)
             ptx::tc_fence_after();
             uint32_t raw[4][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tmem + lane_base + kColKp + c * 32, raw[c]);
+            for (int q = 0; q < 4; ++q) ptx::tmem_ld32(col + q * 32, raw[q]);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 4; ++c) ptx::reg_fence(raw[c]);
+            for (int q = 0; q < 4; ++q) ptx::reg_fence(raw[q]);
             float ss = 0.f;
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int q = 0; q < 4; ++q)
 #pragma unroll
-                for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(raw[c][i]), __uint_as_float(raw[c][i]), ss);
+                for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(raw[q][i]), __uint_as_float(raw[q][i]), ss);
             const float inv = 1.f / fmaxf(sqrtf(ss), 1e-6f);
 #pragma unroll
             for (int c16 = 0; c16 < 16; ++c16) {
@@ -204,17 +244,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
-            ptx::mbar_arrive(ptx::smem_u32(&sm.kp_ready));
-            ok = wwait(&sm.ks);
+            ptx::mbar_arrive(ptx::smem_u32(&sm.kp_ready[c]));
+            ok = wwait(&sm.ks[c]);
         }
         if (ok) {
             // beta R = beta (Vp - K' S) -> bf16 into xv (the V tile is consumed)
             ptx::tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int q = 0; q < 4; ++q) {
                 uint32_t vp[32], ks[32];
-                ptx::tmem_ld32(tmem + lane_base + kColVp + c * 32, vp);
-                ptx::tmem_ld32(tmem + lane_base + kColKS + c * 32, ks);
+                ptx::tmem_ld32(col + 128 + q * 32, vp);
+                ptx::tmem_ld32(col + q * 32, ks);
                 ptx::tmem_wait_ld();
                 ptx::reg_fence(vp);
                 ptx::reg_fence(ks);
@@ -224,26 +264,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         rr[e] = beta_t * (__uint_as_float(vp[g * 8 + e]) - __uint_as_float(ks[g * 8 + e]));
-                    ptx::st_shared_v4(xv + ptx::tile_chunk_offset(r, c * 4 + g), ptx::pack_bf16x2(rr[0], rr[1]),
+                    ptx::st_shared_v4(xv + ptx::tile_chunk_offset(r, q * 4 + g), ptx::pack_bf16x2(rr[0], rr[1]),
                                       ptx::pack_bf16x2(rr[2], rr[3]), ptx::pack_bf16x2(rr[4], rr[5]),
                                       ptx::pack_bf16x2(rr[6], rr[7]));
                 }
             }
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
-            ptx::mbar_arrive(ptx::smem_u32(&sm.r_ready));
+            ptx::mbar_arrive(ptx::smem_u32(&sm.r_ready[c]));
             ok = wwait(&sm.ds);
         }
         if (ok) {
-            // dS row r (key feature r): fp32 partial out
+            // dS row r (key feature r), columns [64 c, 64 c + 64): fp32 partial out
             ptx::tc_fence_after();
+            const size_t part_row = (((size_t)bh * n_parts + pair) * kD + r) * kD;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int q = 0; q < 2; ++q) {
                 uint32_t ds[32];
-                ptx::tmem_ld32(tmem + lane_base + kColDS + c * 32, ds);
+                ptx::tmem_ld32(tmem + lane_base + kColDS + 64u * c + q * 32, ds);
                 ptx::tmem_wait_ld();
                 ptx::reg_fence(ds);
-                float4* dst = reinterpret_cast<float4*>(part_s + part_row + c * 32);
+                float4* dst = reinterpret_cast<float4*>(part_s + part_row + 64 * c + q * 32);
 #pragma unroll
                 for (int g = 0; g < 8; ++g)
                     dst[g] = make_float4(__uint_as_float(ds[4 * g]), __uint_as_float(ds[4 * g + 1]),
@@ -348,7 +389,9 @@ struct UpdateTc {
     CUtensorMap tm_w{}, tm_sb{};
 };
 
-int update_tc_chunks(const Dims& dm) { return (dm.L + kChunk - 1) / kChunk; }
+int update_tc_chunks(const Dims& dm) {
+    return ((dm.L + kChunk - 1) / kChunk + kChunksPerCta - 1) / kChunksPerCta;
+}
 
 UpdateTc* update_tc_create(const Dims& dm, const UpdateBuffers& buf) {
     if (dm.d != kD || !tma_available()) return nullptr;
