@@ -50,9 +50,10 @@
 // into buffer j & 1 (S_{j+2}, or O_inter = Q (W_q S) after P V_{n-2}).
 // Online softmax with lazy rescaling: the running row max only moves when
 // it grows by more than 2^8; the final 1/l uses the same max as the
-// numerator, so the result is exact up to rounding.  One pair of
-// exponentials in three runs on the FMA pipe (exp2_fma2, packed f32x2
-// arithmetic) to balance it against the SFU.
+// numerator, so the result is exact up to rounding.  Exponentials run on
+// the SFU (ex2.approx); the packed f32x2 polynomial (exp2_fma2) can take a
+// share of them (kPolyPairEvery), which measured slower here: the softmax
+// warps are bound by instruction issue, not by the SFU.
 // Outputs leave through a TMA store staged in the segment's Q slot; split
 // partials are stored so that a warp's lanes write consecutive 16 bytes.
 #include "attn_tc.h"
@@ -88,6 +89,12 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;  // S/P buffers at 0, 128; O_0, O_1 at 256, 384
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
+// One pair of exponentials in kPolyPairEvery runs on the FMA pipe (0: none).
+constexpr int kPolyPairEvery = 0;
+__device__ __forceinline__ constexpr bool poly_pair(int i) {
+    constexpr int every = kPolyPairEvery > 0 ? kPolyPairEvery : 1;
+    return kPolyPairEvery > 0 && i % every == every - 1;
+}
 
 enum SegKind : int { kFull = 0, kHead = 1, kTail = 2 };
 
@@ -553,10 +560,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t pk[64];
 #pragma unroll
                 for (int i = 0; i < 64; ++i) {
-                    // a pair in three on the FMA pipe, the rest on the SFU
+                    // SFU exponentials, with kPolyPairEvery > 0 a share on the FMA pipe
                     const float2 a = ptx::fma2(make_float2(x[2 * i], x[2 * i + 1]), sl2, nm);
                     float2 p;
-                    if (i % 3 == 2) {
+                    if (poly_pair(i)) {
                         p = ptx::exp2_fma2(a);
                     } else {
                         p.x = ptx::ex2(a.x);
