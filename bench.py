@@ -54,6 +54,24 @@ def frame_flops(w: workloads.Workload) -> float:
     return B * (w.passes * per_pass + 8.0 * L * d * d * H)
 
 
+def measured_traffic() -> int | None:
+    """DRAM bytes per launch of the fused kernel from the last ncu capture
+    (profiles/attn_tc_traffic.json), or None once the kernel source has
+    changed since that capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "attn_tc_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        h = hashlib.sha256()
+        for rel in d["source_files"]:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+        return int(d["dram_bytes_per_launch"]) if h.hexdigest() == d["source_sha256"] else None
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def load_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -425,7 +443,7 @@ def main():
     achieved = attn_flops(w) / (k_ms / 1e3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "kernel": "attn_tc_kernel",
+                "frac": achieved / peak, "traffic": measured_traffic(), "kernel": "attn_tc_kernel",
                 "kernel_ms": k_ms, "flops_per_launch": attn_flops(w),
                 "peak_kind": f"bf16 sustained ({peaks['source']})",
                 "frac_of_burst": achieved / peaks["bf16_tflops"]}
