@@ -51,9 +51,11 @@ def _load():
             lib.arl2_oracle_pass.argtypes = [I, I, I, I, D, P, P, P, P, P, P, P, P, I, P, P]
             lib.arl2_oracle_rows.argtypes = [I, I, I, I, D, P, P, P, P, P, I, P, P, P]
             lib.arl2_oracle_state_update.argtypes = [I, I, I, I, P, P, P, P, P, P, P]
+            lib.arl2_oracle_state_update_gated.argtypes = [I, I, I, I, P, P, P, P, P, I, P, P]
             lib.arl2_oracle_phi.argtypes = [I, I, I, I, P, P, I, P]
             for f in (lib.arl2_oracle_pass, lib.arl2_oracle_rows,
-                      lib.arl2_oracle_state_update, lib.arl2_oracle_phi):
+                      lib.arl2_oracle_state_update, lib.arl2_oracle_state_update_gated,
+                      lib.arl2_oracle_phi):
                 f.restype = I
             _lib = lib
     return _lib
@@ -91,10 +93,14 @@ def frame_pass(q, k, v, w_q, w_k, w_v, alpha, beta, S, clean: bool, scale=None):
     S2 = f64(S).copy()
     out = np.zeros_like(q)
     sc = default_scale(d) if scale is None else float(scale)
+    per_key = alpha.ndim == 3  # elementwise gating: the update runs separately
     rc = _load().arl2_oracle_pass(B, H, d, L, sc, _p(q), _p(k), _p(v), _p(w_q), _p(w_k),
-                                  _p(w_v), _p(alpha), _p(beta), int(bool(clean)), _p(S2), _p(out))
+                                  _p(w_v), _p(alpha), _p(beta), int(bool(clean) and not per_key),
+                                  _p(S2), _p(out))
     if rc != 0:
         raise RuntimeError("arl2_oracle_pass failed")
+    if clean and per_key:
+        S2 = state_update(k, v, w_k, w_v, alpha, beta, S2)
     return out, S2
 
 
@@ -115,15 +121,23 @@ def rows(q, k, v, w_q, S, rows_b, rows_t, scale=None):
 
 
 def state_update(k, v, w_k, w_v, alpha, beta, S):
-    """Clean-pass update; returns the new state (input S untouched)."""
+    """Clean-pass update; returns the new state (input S untouched).
+
+    alpha [B, H] is the headwise forget gate (S_N = alpha S + ...); alpha
+    [B, H, d] gates each key feature (elementwise gating, S_N = diag(alpha) S
+    + ...), the variant the atlas summary's "Surprising findings" compares.
+    """
     k, v, w_k, w_v = f64(k), f64(v), f64(w_k), f64(w_v)
     alpha, beta = f64(alpha), f64(beta)
     B, H, d, L = _dims(k)
+    per_key = alpha.ndim == 3
+    if alpha.shape != ((B, H, d) if per_key else (B, H)):
+        raise ValueError(f"alpha shape {alpha.shape}")
     S2 = f64(S).copy()
-    rc = _load().arl2_oracle_state_update(B, H, d, L, _p(k), _p(v), _p(w_k), _p(w_v),
-                                          _p(alpha), _p(beta), _p(S2))
+    rc = _load().arl2_oracle_state_update_gated(B, H, d, L, _p(k), _p(v), _p(w_k), _p(w_v),
+                                                _p(alpha), int(per_key), _p(beta), _p(S2))
     if rc != 0:
-        raise RuntimeError("arl2_oracle_state_update failed")
+        raise RuntimeError("arl2_oracle_state_update_gated failed")
     return S2
 
 

@@ -26,7 +26,8 @@
  * Layouts (all dense, row-major, double):
  *   q, k, v, out : [B][L][H][d]    token-major, as a DiT's QKV output
  *   w_q, w_k, w_v: [H][d][d]       row = input feature, column = output
- *   alpha        : [B][H]          forget gate of the frame
+ *   alpha        : [B][H]          forget gate of the frame (headwise), or
+ *                  [B][H][d]       one per key feature (elementwise gating)
  *   beta         : [B][H][L]       per-token rate
  *   S            : [B][H][d][d]    row = key feature, column = value feature
  *
@@ -115,7 +116,7 @@ static void inter_row(int d, const double* qi, const double* Wq, const double* S
  * against the pre-update S for every token (frame-level access). */
 static int update_head(int B, int H, int d, int L, int b, int h, const double* k,
                        const double* v, const double* w_k, const double* w_v,
-                       const double* alpha, const double* beta, double* S_all) {
+                       const double* alpha, int alpha_per_key, const double* beta, double* S_all) {
     (void)B;
     double* kp = (double*)malloc(sizeof(double) * (size_t)L * d);
     double* vp = (double*)malloc(sizeof(double) * (size_t)L * d);
@@ -145,10 +146,13 @@ static int update_head(int B, int H, int d, int L, int b, int h, const double* k
             dS[(size_t)c * d + n] = acc;
         }
     }
-    const double a = alpha[(size_t)b * H + h];
-    for (int c = 0; c < d; ++c)
+    /* headwise gate: one alpha for the whole state; elementwise gate: one
+     * alpha per key feature c, i.e. diag(alpha) S (row c of S scaled) */
+    for (int c = 0; c < d; ++c) {
+        const double a = alpha_per_key ? alpha[((size_t)b * H + h) * d + c] : alpha[(size_t)b * H + h];
         for (int n = 0; n < d; ++n)
             S[(size_t)c * d + n] = a * S[(size_t)c * d + n] + dS[(size_t)c * d + n];
+    }
     free(kp); free(vp); free(r); free(dS);
     return 0;
 }
@@ -199,17 +203,27 @@ int arl2_oracle_rows(int B, int H, int d, int L, double scale, const double* q,
     return err ? -1 : 0;
 }
 
-/* Clean-pass state update of every (b, h), in place. */
-int arl2_oracle_state_update(int B, int H, int d, int L, const double* k, const double* v,
-                             const double* w_k, const double* w_v, const double* alpha,
-                             const double* beta, double* S) {
+/* Clean-pass state update of every (b, h), in place.  alpha_per_key = 0:
+ * alpha is [B][H] (headwise gating, the form the pages adopt); 1: alpha is
+ * [B][H][d], one gate per key feature, S_N = diag(alpha) S_{N-1} + ... (the
+ * elementwise gating the pages compare it with, atlas summary "Surprising
+ * findings"). */
+int arl2_oracle_state_update_gated(int B, int H, int d, int L, const double* k, const double* v,
+                                   const double* w_k, const double* w_v, const double* alpha,
+                                   int alpha_per_key, const double* beta, double* S) {
     if (bad_dims(B, H, d, L) || !k || !v || !w_k || !w_v || !alpha || !beta || !S) return -1;
     int err = 0;
 #pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : err)
     for (int b = 0; b < B; ++b)
         for (int h = 0; h < H; ++h)
-            if (update_head(B, H, d, L, b, h, k, v, w_k, w_v, alpha, beta, S)) err |= 1;
+            if (update_head(B, H, d, L, b, h, k, v, w_k, w_v, alpha, alpha_per_key, beta, S)) err |= 1;
     return err ? -1 : 0;
+}
+
+int arl2_oracle_state_update(int B, int H, int d, int L, const double* k, const double* v,
+                             const double* w_k, const double* w_v, const double* alpha,
+                             const double* beta, double* S) {
+    return arl2_oracle_state_update_gated(B, H, d, L, k, v, w_k, w_v, alpha, 0, beta, S);
 }
 
 /* One full pass: out for every token, then (clean != 0) the state update.

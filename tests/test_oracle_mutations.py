@@ -41,6 +41,11 @@ MUTATIONS = {
         "acc += bt[t] * kp[(size_t)t * d + n] * r[(size_t)t * d + c];"),
     "update_on_every_pass": ("if (clean) return arl2_oracle_state_update(",
                              "if (1) return arl2_oracle_state_update("),
+    "elementwise_gate_on_value_features": (
+        "S[(size_t)c * d + n] = a * S[(size_t)c * d + n] + dS[(size_t)c * d + n];",
+        "S[(size_t)c * d + n] = (alpha_per_key ? alpha[((size_t)b * H + h) * d + n] : a)"
+        " * S[(size_t)c * d + n] + dS[(size_t)c * d + n];"),
+    "elementwise_gate_one_value": ("alpha[((size_t)b * H + h) * d + c]", "alpha[((size_t)b * H + h) * d]"),
 }
 
 

@@ -86,7 +86,9 @@ def test_hand_worked_case(case):
     wk = w_from(case.get("w_k", "identity"), d)
     wv = w_from(case.get("w_v", "identity"), d)
     S = s_from(case.get("S_prev", "zero"), d)
-    alpha = np.array([[case.get("alpha", 1.0)]])
+    a = case.get("alpha", 1.0)
+    # a list: one gate per key feature (elementwise gating), else headwise
+    alpha = np.asarray(a, dtype=np.float64)[None, None] if isinstance(a, list) else np.array([[a]])
     beta = np.asarray(case.get("beta", [0.0] * L), dtype=np.float64)[None, None]
     clean = "expected_S" in case
     out, S_new = oracle.frame_pass(q, k, v, wq, wk, wv, alpha, beta, S, clean)
@@ -334,3 +336,46 @@ def test_oracle_rejects_bad_arguments():
     with pytest.raises(RuntimeError):
         oracle.rows(np.zeros((1, 2, 1, 4)), np.zeros((1, 2, 1, 4)), np.zeros((1, 2, 1, 4)),
                     np.zeros((1, 4, 4)), np.zeros((1, 1, 4, 4)), [0], [2])
+
+
+# --------------------------------------------------------------------------
+# Elementwise gating (atlas summary, "Surprising findings": one forget gate
+# per key feature instead of one per head; S_N = diag(alpha) S_{N-1} + ...)
+# --------------------------------------------------------------------------
+
+def _update_inputs(seed, B=2, H=2, d=6, L=7):
+    rng = np.random.default_rng(seed)
+    k = rng.normal(size=(B, L, H, d))
+    v = rng.normal(size=(B, L, H, d))
+    wk = rng.normal(size=(H, d, d))
+    wv = rng.normal(size=(H, d, d))
+    beta = rng.random((B, H, L))
+    S = rng.normal(size=(B, H, d, d))
+    return rng, k, v, wk, wv, beta, S
+
+
+def test_uniform_elementwise_gate_equals_headwise_gate():
+    rng, k, v, wk, wv, beta, S = _update_inputs(41)
+    a = rng.random((2, 2))
+    s_head = oracle.state_update(k, v, wk, wv, a, beta, S)
+    s_elem = oracle.state_update(k, v, wk, wv, np.repeat(a[:, :, None], 6, axis=2), beta, S)
+    assert np.array_equal(s_head, s_elem)
+
+
+def test_elementwise_gate_zero_clears_and_one_keeps_a_key_row():
+    _, k, v, wk, wv, beta, S = _update_inputs(42)
+    a = np.tile(np.array([0.0, 1.0, 0.0, 1.0, 1.0, 0.0]), (2, 2, 1))
+    S_new = oracle.state_update(k, v, wk, wv, a, np.zeros_like(beta), S)
+    for c in range(6):
+        if a[0, 0, c] == 0.0:
+            assert not S_new[:, :, c, :].any()
+        else:
+            assert np.array_equal(S_new[:, :, c, :], S[:, :, c, :])
+
+
+def test_elementwise_gate_enters_as_a_row_scaling_of_the_previous_state():
+    rng, k, v, wk, wv, beta, S = _update_inputs(43)
+    a = rng.random((2, 2, 6))
+    with_gate = oracle.state_update(k, v, wk, wv, a, beta, S)
+    no_gate = oracle.state_update(k, v, wk, wv, np.zeros_like(a), beta, S)
+    np.testing.assert_allclose(with_gate - no_gate, a[:, :, :, None] * S, rtol=0, atol=1e-12)
