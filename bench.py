@@ -287,6 +287,8 @@ def main():
     ap.add_argument("--workload", default="480p_bf16")
     ap.add_argument("--impl", default="arl2", choices=["arl2", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--gating", default="headwise", choices=["headwise", "elementwise"],
+                    help="forget gate per head (the pages' form) or per key feature")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-passes", type=int, default=0,
                     help="profiling case: run this many read-only passes over a ring of inputs "
@@ -310,11 +312,12 @@ def main():
     stream_idx = rank  # each rank: its own independent stream (replica)
     wq, wk, wv = workloads.phi_weights(w, 0)
     lay = Arl2Layer(w.batch, w.heads, w.head_dim, w.tokens, wq.cuda(), wk.cuda(), wv.cuda(),
-                    dtype=w.torch_dtype, host_staging=True)
+                    dtype=w.torch_dtype, host_staging=True, gating=args.gating)
+    gate_draw = workloads.frame_gates_elementwise if args.gating == "elementwise" else workloads.frame_gates
     # all inputs of the stream, resident in HBM before timing
     ins, gates = [], []
     for f in range(w.frames):
-        a, b = workloads.frame_gates(w, stream_idx, f)
+        a, b = gate_draw(w, stream_idx, f)
         gates.append((a.cuda(), b.cuda()))
         for p in range(w.passes):
             ins.append(workloads.pass_inputs(w, stream_idx, f, p, device="cuda"))
@@ -461,7 +464,8 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
                    "tokens_per_frame": w.tokens, "frames_per_step": w.frames, "passes": w.passes,
-                   "parallelism": f"replicas{ws}", "l2": "inputs larger than L2 (1.2 GB ring)"},
+                   "parallelism": f"replicas{ws}", "l2": "inputs larger than L2 (1.2 GB ring)",
+                   "gating": args.gating},
         "tokens_per_s": value * w.tokens,
         "tflops_per_frame_algorithmic": frame_flops(w) / 1e12,
         "roofline": roofline, "clocks": clk,

@@ -27,6 +27,7 @@ ARL2_OK = 0
 ARL2_ERR_TIMEOUT = -6
 ARL2_BF16, ARL2_FP32 = 0, 1
 ARL2_IMPL_AUTO, ARL2_IMPL_SIMT = 0, 1
+ARL2_GATE_HEADWISE, ARL2_GATE_ELEMENTWISE = 0, 1
 
 EXPORTED = (
     "arl2_create", "arl2_frame_forward", "arl2_frame_forward_host", "arl2_state_reset",
@@ -43,7 +44,7 @@ class Arl2Config(ctypes.Structure):
         ("tokens_per_frame", ctypes.c_int), ("dtype", ctypes.c_int),
         ("w_q", ctypes.c_void_p), ("w_k", ctypes.c_void_p), ("w_v", ctypes.c_void_p),
         ("softmax_scale", ctypes.c_float), ("host_staging", ctypes.c_int), ("impl", ctypes.c_int),
-        ("max_ctas", ctypes.c_int),
+        ("max_ctas", ctypes.c_int), ("gating", ctypes.c_int),
     ]
 
 
@@ -129,7 +130,8 @@ class Arl2Layer:
 
     def __init__(self, batch: int, heads: int, head_dim: int, tokens: int, w_q, w_k, w_v, *,
                  dtype: torch.dtype = torch.bfloat16, softmax_scale: float = 0.0,
-                 host_staging: bool = False, impl: str = "auto", max_ctas: int = 0, stream=None):
+                 host_staging: bool = False, impl: str = "auto", max_ctas: int = 0,
+                 gating: str = "headwise", stream=None):
         if dtype not in (torch.bfloat16, torch.float32):
             raise ValueError("dtype must be torch.bfloat16 or torch.float32")
         for w in (w_q, w_k, w_v):
@@ -144,7 +146,9 @@ class Arl2Layer:
                          ARL2_BF16 if dtype == torch.bfloat16 else ARL2_FP32,
                          w_q.data_ptr(), w_k.data_ptr(), w_v.data_ptr(), float(softmax_scale),
                          1 if host_staging else 0,
-                         {"auto": ARL2_IMPL_AUTO, "simt": ARL2_IMPL_SIMT}[impl], int(max_ctas))
+                         {"auto": ARL2_IMPL_AUTO, "simt": ARL2_IMPL_SIMT}[impl], int(max_ctas),
+                         {"headwise": ARL2_GATE_HEADWISE, "elementwise": ARL2_GATE_ELEMENTWISE}[gating])
+        self.alpha_shape = lambda B, H: (B, H, head_dim) if gating == "elementwise" else (B, H)
         h = ctypes.c_void_p()
         with torch.cuda.device(self.device):
             _check(_lib.arl2_create(ctypes.byref(cfg), _stream(stream), ctypes.byref(h)), "arl2_create")
@@ -167,8 +171,9 @@ class Arl2Layer:
     # -- C ABI calls ----------------------------------------------------
     def forward(self, q, k, v, alpha=None, beta=None, clean_pass: bool = False, out=None,
                 stream=None):
-        """One denoising pass; returns out [B, L, H, d].  alpha [B, H] and
-        beta [B, H, L] (fp32 CUDA) are needed on the clean pass only."""
+        """One denoising pass; returns out [B, L, H, d].  alpha [B, H] ([B, H, d]
+        with elementwise gating) and beta [B, H, L] (fp32 CUDA) are needed on
+        the clean pass only."""
         self._tok(q, "q"), self._tok(k, "k"), self._tok(v, "v")
         if out is None:
             out = torch.empty_like(q)
@@ -178,8 +183,8 @@ class Arl2Layer:
             if alpha is None or beta is None:
                 raise ValueError("the clean pass needs alpha and beta")
             if not (alpha.is_cuda and alpha.dtype == torch.float32 and alpha.is_contiguous()
-                    and tuple(alpha.shape) == (B, H)):
-                raise ValueError("alpha must be a contiguous fp32 CUDA tensor [B, H]")
+                    and tuple(alpha.shape) == self.alpha_shape(B, H)):
+                raise ValueError(f"alpha must be a contiguous fp32 CUDA tensor {list(self.alpha_shape(B, H))}")
             if not (beta.is_cuda and beta.dtype == torch.float32 and beta.is_contiguous()
                     and tuple(beta.shape) == (B, H, L)):
                 raise ValueError("beta must be a contiguous fp32 CUDA tensor [B, H, L]")

@@ -58,6 +58,7 @@ struct arl2_handle {
     void* stage_tok[4] = {nullptr, nullptr, nullptr, nullptr};  // q, k, v, out
     float* stage_alpha = nullptr;
     float* stage_beta = nullptr;
+    int alpha_per_key = 0;    // elementwise gating: alpha [B][H][d] instead of [B][H]
     int* err = nullptr;       // device error word
     unsigned long long launches = 0;  // kernels enqueued by this handle
 };
@@ -123,7 +124,8 @@ arl2_status clean_update(arl2_handle* h, const void* k, const void* v, const flo
                          const float* beta, cudaStream_t st) {
     if (h->use_tc) {
         h->launches += 2;
-        return arl2::update_tc_launch(h->up, *h->maps, k, v, alpha, beta, h->err, st) == cudaSuccess
+        return arl2::update_tc_launch(h->up, *h->maps, k, v, alpha, h->alpha_per_key, beta, h->err, st) ==
+                       cudaSuccess
                    ? ARL2_OK
                    : ARL2_ERR_CUDA;
     }
@@ -132,7 +134,7 @@ arl2_status clean_update(arl2_handle* h, const void* k, const void* v, const flo
     if (arl2::launch_phi_simt(bf16, k, h->w[1], true, h->kp, nullptr, h->dm, st) != cudaSuccess ||
         arl2::launch_phi_simt(bf16, v, h->w[2], false, h->vp, nullptr, h->dm, st) != cudaSuccess ||
         arl2::launch_residual_simt(h->kp, h->vp, h->S, h->dm, st) != cudaSuccess ||
-        arl2::launch_accum_simt(h->kp, h->vp, alpha, beta, h->S, h->dm, st) != cudaSuccess)
+        arl2::launch_accum_simt(h->kp, h->vp, alpha, h->alpha_per_key, beta, h->S, h->dm, st) != cudaSuccess)
         return ARL2_ERR_CUDA;
     return ARL2_OK;
 }
@@ -169,6 +171,8 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
         return ARL2_ERR_SHAPE;
     if (!(cfg->softmax_scale >= 0.f) || std::isinf(cfg->softmax_scale)) return ARL2_ERR_INVALID_ARG;
     if (cfg->max_ctas < 0) return ARL2_ERR_INVALID_ARG;
+    if (cfg->gating != ARL2_GATE_HEADWISE && cfg->gating != ARL2_GATE_ELEMENTWISE)
+        return ARL2_ERR_INVALID_ARG;
     if (!aligned16(cfg->w_q) || !aligned16(cfg->w_k) || !aligned16(cfg->w_v)) return ARL2_ERR_ALIGN;
     const bool use_tc = cfg->impl == ARL2_IMPL_AUTO && cfg->dtype == ARL2_BF16;
     if (use_tc && cfg->head_dim != 128) return ARL2_ERR_UNSUPPORTED;
@@ -183,6 +187,7 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
     h->dtype = cfg->dtype;
     h->impl = cfg->impl;
     h->use_tc = use_tc;
+    h->alpha_per_key = cfg->gating == ARL2_GATE_ELEMENTWISE ? 1 : 0;
     h->scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->head_dim);
     h->esz = cfg->dtype == ARL2_BF16 ? 2 : 4;
     const Dims& dm = h->dm;
@@ -209,7 +214,8 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
     }
     if (s == ARL2_OK && cfg->host_staging) {
         for (int i = 0; i < 4 && s == ARL2_OK; ++i) s = dalloc(h, &h->stage_tok[i], h->n_tok * h->esz);
-        if (s == ARL2_OK) s = dalloc(h, &h->stage_alpha, (size_t)dm.B * dm.H * sizeof(float));
+        if (s == ARL2_OK)
+            s = dalloc(h, &h->stage_alpha, (size_t)dm.B * dm.H * (h->alpha_per_key ? dm.d : 1) * sizeof(float));
         if (s == ARL2_OK) s = dalloc(h, &h->stage_beta, (size_t)dm.B * dm.H * dm.L * sizeof(float));
     }
     if (s == ARL2_OK && arl2::simt_init() != cudaSuccess) s = ARL2_ERR_CUDA;
@@ -286,7 +292,7 @@ arl2_status arl2_frame_forward_host(arl2_handle* h, const void* q, const void* k
     const float* b_dev = nullptr;
     if (clean_pass) {
         const Dims& dm = h->dm;
-        if (cudaMemcpyAsync(h->stage_alpha, alpha, (size_t)dm.B * dm.H * sizeof(float),
+        if (cudaMemcpyAsync(h->stage_alpha, alpha, (size_t)dm.B * dm.H * (h->alpha_per_key ? dm.d : 1) * sizeof(float),
                             cudaMemcpyHostToDevice, stream) != cudaSuccess ||
             cudaMemcpyAsync(h->stage_beta, beta, (size_t)dm.B * dm.H * dm.L * sizeof(float),
                             cudaMemcpyHostToDevice, stream) != cudaSuccess)

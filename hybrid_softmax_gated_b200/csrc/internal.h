@@ -42,7 +42,7 @@ cudaError_t launch_residual_simt(const float* kp, float* vp_to_r, const float* S
                                  cudaStream_t st);
 
 // S = alpha S + kp^T diag(beta) r, in place.
-cudaError_t launch_accum_simt(const float* kp, const float* r, const float* alpha,
+cudaError_t launch_accum_simt(const float* kp, const float* r, const float* alpha, int alpha_per_key,
                               const float* beta, float* S, Dims dm, cudaStream_t st);
 
 // Copies of the state derived from S alone, used by the tensor-core kernels:

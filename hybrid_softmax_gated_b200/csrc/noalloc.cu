@@ -83,7 +83,7 @@ extern "C" arl2_status arl2_state_update_noalloc(int batch, int heads, int head_
     if (arl2::launch_phi_simt(bf16, k, w_k, true, kp, nullptr, dm, stream) != cudaSuccess ||
         arl2::launch_phi_simt(bf16, v, w_v, false, vr, nullptr, dm, stream) != cudaSuccess ||
         arl2::launch_residual_simt(kp, vr, state, dm, stream) != cudaSuccess ||
-        arl2::launch_accum_simt(kp, vr, alpha, beta, state, dm, stream) != cudaSuccess)
+        arl2::launch_accum_simt(kp, vr, alpha, 0, beta, state, dm, stream) != cudaSuccess)
         return ARL2_ERR_CUDA;
     return ARL2_OK;
 }

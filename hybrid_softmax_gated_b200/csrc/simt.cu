@@ -213,6 +213,7 @@ constexpr int kCRows = 8;
 __global__ void __launch_bounds__(128) accum_simt_kernel(const float* __restrict__ kp,
                                                          const float* __restrict__ r,
                                                          const float* __restrict__ alpha,
+                                                         int alpha_per_key,
                                                          const float* __restrict__ beta,
                                                          float* __restrict__ S, Dims dm) {
     const int d = dm.d;
@@ -231,12 +232,13 @@ __global__ void __launch_bounds__(128) accum_simt_kernel(const float* __restrict
         for (int i = 0; i < kCRows; ++i)
             if (c0 + i < d) acc[i] = fmaf(krow[c0 + i], rb, acc[i]);
     }
-    const float a = alpha[(size_t)b * dm.H + h];
+    // headwise: one gate for the head; elementwise: one per key feature c
+    const float* a_bh = alpha + ((size_t)b * dm.H + h) * (alpha_per_key ? d : 1);
     float* Sbh = S + ((size_t)b * dm.H + h) * d * d;
 #pragma unroll
     for (int i = 0; i < kCRows; ++i) {
         const int c = c0 + i;
-        if (c < d) Sbh[c * d + n] = fmaf(a, Sbh[c * d + n], acc[i]);
+        if (c < d) Sbh[c * d + n] = fmaf(a_bh[alpha_per_key ? c : 0], Sbh[c * d + n], acc[i]);
     }
 }
 
@@ -304,10 +306,10 @@ cudaError_t launch_residual_simt(const float* kp, float* vp_to_r, const float* S
     return cudaGetLastError();
 }
 
-cudaError_t launch_accum_simt(const float* kp, const float* r, const float* alpha,
+cudaError_t launch_accum_simt(const float* kp, const float* r, const float* alpha, int alpha_per_key,
                               const float* beta, float* S, Dims dm, cudaStream_t st) {
     const dim3 grid((dm.d + kCRows - 1) / kCRows, dm.H, dm.B);
-    accum_simt_kernel<<<grid, 128, 0, st>>>(kp, r, alpha, beta, S, dm);
+    accum_simt_kernel<<<grid, 128, 0, st>>>(kp, r, alpha, alpha_per_key, beta, S, dm);
     return cudaGetLastError();
 }
 

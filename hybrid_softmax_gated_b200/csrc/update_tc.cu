@@ -315,6 +315,7 @@ constexpr int kFoldCols = 4;
 constexpr int kMaxChunksInFlight = 16;
 __global__ void __launch_bounds__(kD) finalize_fold_kernel(const float* __restrict__ part_s,
                                                            const float* __restrict__ alpha,
+                                                           int alpha_per_key,
                                                            float* __restrict__ S,
                                                            const __nv_bfloat16* __restrict__ wq,
                                                            __nv_bfloat16* __restrict__ Mt,
@@ -334,7 +335,8 @@ __global__ void __launch_bounds__(kD) finalize_fold_kernel(const float* __restri
     const size_t e = (size_t)bh * kD * kD + (size_t)r * kD + n0;
     float4 s = *reinterpret_cast<const float4*>(S + e);
     if (alpha) {
-        const float a = alpha[bh];
+        // headwise: one gate for the head; elementwise: row r = key feature r
+        const float a = alpha_per_key ? alpha[(size_t)bh * kD + r] : alpha[bh];
         float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
         const size_t pb = (size_t)bh * n_chunks * kD * kD + (size_t)r * kD + n0;
         // loads in flight together; the sum itself in chunk order
@@ -435,7 +437,8 @@ static cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_
 }
 
 cudaError_t update_tc_launch(UpdateTc* u, TokenMapCache& maps, const void* k, const void* v,
-                             const float* alpha, const float* beta, int* err, cudaStream_t st) {
+                             const float* alpha, int alpha_per_key, const float* beta, int* err,
+                             cudaStream_t st) {
     const Dims& dm = u->dm;
     CUtensorMap ck, cv;
     if (!maps.get(k, &ck) || !maps.get(v, &cv)) return cudaErrorInvalidValue;
@@ -443,7 +446,7 @@ cudaError_t update_tc_launch(UpdateTc* u, TokenMapCache& maps, const void* k, co
                                st, ck, cv, u->tm_w, u->tm_sb, beta, u->buf.part_s, dm.L, dm.H, err);
     if (e != cudaSuccess) return e;
     return launch_pdl(finalize_fold_kernel, dim3(kD / kFoldCols, dm.H, dm.B), dim3(kD), 0, st,
-                      static_cast<const float*>(u->buf.part_s), alpha, u->buf.S,
+                      static_cast<const float*>(u->buf.part_s), alpha, alpha_per_key, u->buf.S,
                       static_cast<const __nv_bfloat16*>(u->buf.w_all), static_cast<__nv_bfloat16*>(u->buf.Mt),
                       static_cast<__nv_bfloat16*>(u->buf.Sb), u->n_chunks, dm.H);
 }
@@ -452,7 +455,7 @@ cudaError_t launch_fold_state(const void* wq_bf16, const float* S, void* Mt, voi
                               cudaStream_t st) {
     if (dm.d != kD) return cudaErrorInvalidValue;
     return launch_pdl(finalize_fold_kernel, dim3(kD / kFoldCols, dm.H, dm.B), dim3(kD), 0, st,
-                      static_cast<const float*>(nullptr), static_cast<const float*>(nullptr),
+                      static_cast<const float*>(nullptr), static_cast<const float*>(nullptr), 0,
                       const_cast<float*>(S), static_cast<const __nv_bfloat16*>(wq_bf16),
                       static_cast<__nv_bfloat16*>(Mt), static_cast<__nv_bfloat16*>(Sb), 0, dm.H);
 }

@@ -31,6 +31,7 @@ void update_tc_destroy(UpdateTc* u);
 // fold).  k, v: token
 // tensors of the pass; alpha [B][H], beta [B][H][L] fp32.
 cudaError_t update_tc_launch(UpdateTc* u, TokenMapCache& maps, const void* k, const void* v,
-                             const float* alpha, const float* beta, int* err, cudaStream_t st);
+                             const float* alpha, int alpha_per_key, const float* beta, int* err,
+                             cudaStream_t st);
 
 }  // namespace arl2

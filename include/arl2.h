@@ -24,7 +24,11 @@
  *   - The state S is fp32 [B][H][d][d], row = key feature, column = value
  *     feature.  It is owned by the handle.
  *   - alpha is fp32 [B][H] (one forget gate per stream and head for the
- *     frame), beta is fp32 [B][H][L] (one rate per token).
+ *     frame; headwise gating, the form the pages adopt), or, for a handle
+ *     created with gating = ARL2_GATE_ELEMENTWISE, fp32 [B][H][d] (one gate
+ *     per key feature: S_N = diag(alpha) S_{N-1} + ..., the variant the
+ *     atlas summary's "Surprising findings" compares).  beta is fp32
+ *     [B][H][L] (one rate per token).
  *   - Every call is asynchronous and stream-ordered on the given stream: it
  *     makes no host synchronisation and allocates nothing after
  *     arl2_create.  A call that returns anything but ARL2_OK enqueued
@@ -66,6 +70,9 @@ typedef enum { ARL2_BF16 = 0, ARL2_FP32 = 1 } arl2_dtype;
  * back to it. */
 typedef enum { ARL2_IMPL_AUTO = 0, ARL2_IMPL_SIMT = 1 } arl2_impl;
 
+/* Granularity of the forget gate alpha (see the conventions above). */
+typedef enum { ARL2_GATE_HEADWISE = 0, ARL2_GATE_ELEMENTWISE = 1 } arl2_gating;
+
 typedef struct arl2_handle arl2_handle;
 
 typedef struct {
@@ -84,6 +91,7 @@ typedef struct {
     int max_ctas;          /* 0: the tensor-core attention kernel may use every
                               SM; > 0 caps its persistent grid (co-scheduling
                               with other work, tests of the split schedule)   */
+    arl2_gating gating;    /* HEADWISE: alpha [B][H]; ELEMENTWISE: [B][H][d]  */
 } arl2_config;
 
 /* Create a layer on the current device.  Validates cfg, allocates the zeroed
@@ -98,7 +106,8 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
  * clean_pass is nonzero, then also updates the state in place to S_N; alpha
  * and beta are read only in that case and may be NULL otherwise.
  * q, k, v, out: device [B][L][H][d] dtype, 16-byte aligned; out must not
- * alias q, k or v.  alpha: device fp32 [B][H]; beta: device fp32 [B][H][L]. */
+ * alias q, k or v.  alpha: device fp32 [B][H] ([B][H][d] with elementwise
+ * gating); beta: device fp32 [B][H][L]. */
 arl2_status arl2_frame_forward(arl2_handle* h, const void* q, const void* k, const void* v,
                                const float* alpha, const float* beta, int clean_pass,
                                void* out, cudaStream_t stream);

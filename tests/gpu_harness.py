@@ -29,23 +29,25 @@ def err(x, ref) -> float:
 
 def run_and_check(w: workloads.Workload, *, impl: str = "auto", layer: int = 0, frames=None,
                   full_rows=lambda f, p: True, sample_rows: int = 64, seed: int = 0,
-                  device_inputs: bool = False, layer_kw=None):
+                  device_inputs: bool = False, layer_kw=None, gating: str = "headwise"):
     """Run frames of workload w on the GPU and on the oracle.
 
     full_rows(frame, pass) selects passes whose every output row is
     compared; other passes compare `sample_rows` random (stream, token)
     rows.  The state is compared in full after every clean pass.  Returns
-    the worst output and state errors.
+    the worst output and state errors.  gating="elementwise" draws one forget
+    gate per key feature.
     """
     tol = TOL[w.dtype]
-    lay, (wq, wk, wv) = make_layer(w, layer, impl, **(layer_kw or {}))
+    lay, (wq, wk, wv) = make_layer(w, layer, impl, gating=gating, **(layer_kw or {}))
+    gates = workloads.frame_gates_elementwise if gating == "elementwise" else workloads.frame_gates
     rng = np.random.default_rng(seed)
     S_ref = oracle.zero_state(w.batch, w.heads, w.head_dim)
     worst_o = worst_s = 0.0
     dev = "cuda" if device_inputs else "cpu"
     try:
         for f in range(w.frames if frames is None else frames):
-            alpha, beta = workloads.frame_gates(w, layer, f)
+            alpha, beta = gates(w, layer, f)
             a_d, b_d = alpha.cuda(), beta.cuda()
             for p in range(w.passes):
                 q, k, v = workloads.pass_inputs(w, layer, f, p, device=dev)

@@ -79,3 +79,13 @@ def test_shape_and_alignment_checks_come_before_cuda():
     assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1
     cfg = arl2.Arl2Config(1, 1, 16, 16, 1, fake, fake, fake, -1.0, 0, 0)  # bad scale
     assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1
+
+
+def test_gating_mode_is_validated_before_cuda():
+    lib = arl2._lib
+    h = ctypes.c_void_p()
+    fake = 0x1000
+    cfg = arl2.Arl2Config(1, 1, 16, 16, 1, fake, fake, fake, 0.0, 0, 0, 0, 5)  # no such gating
+    assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1
+    cfg = arl2.Arl2Config(1, 1, 16, 16, 1, fake, fake, fake, 0.0, 0, 0, -1, arl2.ARL2_GATE_ELEMENTWISE)
+    assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1  # (max_ctas < 0)

@@ -13,6 +13,7 @@ Value recipe (identical for every workload, per stream b and layer l):
   q, k, v       ~ N(0, 1), shape [B, L, H, d], one draw per (frame, pass)
   W_q, W_k, W_v = I + N(0, 0.02) per head, shape [H, d, d], one per layer
   alpha         = sigmoid(N(2, 0.5)), shape [B, H], one per frame
+                  (elementwise gating: shape [B, H, d], same distribution)
   beta          = sigmoid(N(0, 1)) / L, shape [B, H, L], one per frame
 Every tensor is rounded to the run's dtype (q, k, v and W) or kept fp32
 (alpha, beta); the same rounded values go to the GPU and to the oracle.
@@ -81,7 +82,7 @@ def stream_base(layer: int, stream: int) -> int:
     return SEED_BASE + 1000 * layer + stream
 
 
-_TAG_QKV, _TAG_GATES, _TAG_W = 1, 2, 3
+_TAG_QKV, _TAG_GATES, _TAG_W, _TAG_GATES_ELEM = 1, 2, 3, 4
 
 
 def _gen(*parts: int, device: str = "cpu") -> torch.Generator:
@@ -133,6 +134,19 @@ def frame_gates(w: Workload, layer: int, frame: int):
         alpha[b] = torch.sigmoid(2.0 + 0.5 * torch.randn(H, generator=g))
         beta[b] = torch.sigmoid(torch.randn(H, L, generator=g)) / L
     return alpha.contiguous(), beta.contiguous()
+
+
+def frame_gates_elementwise(w: Workload, layer: int, frame: int):
+    """alpha [B, H, d] (one forget gate per key feature) and beta [B, H, L],
+    fp32, for one frame: alpha = sigmoid(N(2, 0.5)) per entry, beta as in
+    frame_gates (the same draw, so the two gatings share their beta)."""
+    B, L, H, d = w.batch, w.tokens, w.heads, w.head_dim
+    _, beta = frame_gates(w, layer, frame)
+    alpha = torch.empty(B, H, d, dtype=torch.float32)
+    for b in range(B):
+        g = _gen(stream_base(layer, b), _TAG_GATES_ELEM, frame)
+        alpha[b] = torch.sigmoid(2.0 + 0.5 * torch.randn(H, d, generator=g))
+    return alpha.contiguous(), beta
 
 
 def is_clean(w: Workload, pass_idx: int) -> bool:
