@@ -53,9 +53,11 @@ def _load():
             lib.arl2_oracle_state_update.argtypes = [I, I, I, I, P, P, P, P, P, P, P]
             lib.arl2_oracle_state_update_gated.argtypes = [I, I, I, I, P, P, P, P, P, I, P, P]
             lib.arl2_oracle_phi.argtypes = [I, I, I, I, P, P, I, P]
+            lib.arl2_oracle_pass_token_level.argtypes = [I, I, I, I, D, P, P, P, P, P, P, P, I, P, I,
+                                                         P, P]
             for f in (lib.arl2_oracle_pass, lib.arl2_oracle_rows,
                       lib.arl2_oracle_state_update, lib.arl2_oracle_state_update_gated,
-                      lib.arl2_oracle_phi):
+                      lib.arl2_oracle_phi, lib.arl2_oracle_pass_token_level):
                 f.restype = I
             _lib = lib
     return _lib
@@ -101,6 +103,31 @@ def frame_pass(q, k, v, w_q, w_k, w_v, alpha, beta, S, clean: bool, scale=None):
         raise RuntimeError("arl2_oracle_pass failed")
     if clean and per_key:
         S2 = state_update(k, v, w_k, w_v, alpha, beta, S2)
+    return out, S2
+
+
+def frame_pass_token_level(q, k, v, w_q, w_k, w_v, alpha, beta, S, clean: bool, scale=None):
+    """One pass with token-level (sequential) state access, the ablation the
+    pages compare with frame-level access: token i reads the state left by
+    tokens 0..i-1, then updates it (delta rule); the forget gate acts once,
+    with token 0's update.  alpha [B, H] (or [B, H, d] per key feature) and
+    beta [B, H, L] are used on every pass; only a clean pass keeps the final
+    state.  Returns (out, S_after); S is not modified."""
+    q, k, v = f64(q), f64(k), f64(v)
+    w_q, w_k, w_v = f64(w_q), f64(w_k), f64(w_v)
+    B, H, d, L = _dims(q)
+    alpha, beta = f64(alpha), f64(beta)
+    per_key = alpha.ndim == 3
+    if alpha.shape != ((B, H, d) if per_key else (B, H)) or beta.shape != (B, H, L):
+        raise ValueError("alpha/beta shape")
+    S2 = f64(S).copy()
+    out = np.zeros_like(q)
+    sc = default_scale(d) if scale is None else float(scale)
+    rc = _load().arl2_oracle_pass_token_level(B, H, d, L, sc, _p(q), _p(k), _p(v), _p(w_q), _p(w_k),
+                                              _p(w_v), _p(alpha), int(per_key), _p(beta),
+                                              int(bool(clean)), _p(S2), _p(out))
+    if rc != 0:
+        raise RuntimeError("arl2_oracle_pass_token_level failed")
     return out, S2
 
 

@@ -253,3 +253,81 @@ int arl2_oracle_pass(int B, int H, int d, int L, double scale, const double* q,
     if (clean) return arl2_oracle_state_update(B, H, d, L, k, v, w_k, w_v, alpha, beta, S);
     return 0;
 }
+
+/* Token-level (sequential) state access: the ablation the pages compare with
+ * frame-level access (technical summary section 2.2 "Frame-Level Access";
+ * atlas summary "Surprising findings").  Within the frame, token i reads the
+ * state left by tokens 0..i-1 and then updates it with the delta rule; the
+ * frame's forget gate acts once, with token 0's update:
+ *   S^(0)   = S_{N-1}
+ *   o_i     = intra_i + q'_i S^(i)
+ *   S^(i+1) = G_i S^(i) + beta_i k'_i^T (v'_i - k'_i S^(i)),
+ *             G_0 = alpha (diag(alpha) with per-key gates), G_i = I for i > 0
+ * With one token per frame this is the frame-level rule.  Every pass reads
+ * through its own sequential states; only the clean pass keeps S^(L) as S_N
+ * ("Clean-Pass Updates").  Tokens are taken in their order in the frame. */
+static int token_level_head(int H, int d, int L, int b, int h, double scale, const double* q,
+                            const double* k, const double* v, const double* w_q, const double* w_k,
+                            const double* w_v, const double* alpha, int alpha_per_key,
+                            const double* beta, int clean, double* S_all, double* out) {
+    double* qp = (double*)malloc(sizeof(double) * (size_t)L * d);
+    double* kp = (double*)malloc(sizeof(double) * (size_t)L * d);
+    double* vp = (double*)malloc(sizeof(double) * (size_t)L * d);
+    double* St = (double*)malloc(sizeof(double) * (size_t)d * d);
+    double* u = (double*)malloc(sizeof(double) * (size_t)d);
+    double* s = (double*)malloc(sizeof(double) * (size_t)L);
+    if (!qp || !kp || !vp || !St || !u || !s) {
+        free(qp); free(kp); free(vp); free(St); free(u); free(s);
+        return -1;
+    }
+    double* S = S_all + IDX4(b, h, 0, 0, H, d, d);
+    phi_map_head(H, d, L, b, h, q, w_q, 0, qp);
+    phi_map_head(H, d, L, b, h, k, w_k, 1, kp);
+    phi_map_head(H, d, L, b, h, v, w_v, 0, vp);
+    for (size_t e = 0; e < (size_t)d * d; ++e) St[e] = S[e];
+    const double* bt = beta + IDX4(0, b, h, 0, 1, H, L);
+    for (int i = 0; i < L; ++i) {
+        double* o = out + IDX4(b, i, h, 0, L, H, d);
+        intra_row(H, d, L, b, h, i, scale, q, k, v, s, o);
+        /* read the state before this token's update */
+        for (int n = 0; n < d; ++n) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c) acc += qp[(size_t)i * d + c] * St[(size_t)c * d + n];
+            o[n] += acc;
+        }
+        /* u = v'_i - k'_i S^(i) */
+        for (int n = 0; n < d; ++n) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c) acc += kp[(size_t)i * d + c] * St[(size_t)c * d + n];
+            u[n] = vp[(size_t)i * d + n] - acc;
+        }
+        for (int c = 0; c < d; ++c) {
+            double g = 1.0;
+            if (i == 0) g = alpha_per_key ? alpha[((size_t)b * H + h) * d + c] : alpha[(size_t)b * H + h];
+            for (int n = 0; n < d; ++n)
+                St[(size_t)c * d + n] = g * St[(size_t)c * d + n] + bt[i] * kp[(size_t)i * d + c] * u[n];
+        }
+    }
+    if (clean)
+        for (size_t e = 0; e < (size_t)d * d; ++e) S[e] = St[e];
+    free(qp); free(kp); free(vp); free(St); free(u); free(s);
+    return 0;
+}
+
+int arl2_oracle_pass_token_level(int B, int H, int d, int L, double scale, const double* q,
+                                 const double* k, const double* v, const double* w_q,
+                                 const double* w_k, const double* w_v, const double* alpha,
+                                 int alpha_per_key, const double* beta, int clean, double* S,
+                                 double* out) {
+    if (bad_dims(B, H, d, L) || !q || !k || !v || !w_q || !w_k || !w_v || !alpha || !beta || !S ||
+        !out)
+        return -1;
+    int err = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : err)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h)
+            if (token_level_head(H, d, L, b, h, scale, q, k, v, w_q, w_k, w_v, alpha, alpha_per_key,
+                                 beta, clean, S, out))
+                err |= 1;
+    return err ? -1 : 0;
+}

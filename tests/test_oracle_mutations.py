@@ -46,6 +46,13 @@ MUTATIONS = {
         "S[(size_t)c * d + n] = (alpha_per_key ? alpha[((size_t)b * H + h) * d + n] : a)"
         " * S[(size_t)c * d + n] + dS[(size_t)c * d + n];"),
     "elementwise_gate_one_value": ("alpha[((size_t)b * H + h) * d + c]", "alpha[((size_t)b * H + h) * d]"),
+    "token_level_reads_frame_state": (
+        "for (int c = 0; c < d; ++c) acc += qp[(size_t)i * d + c] * St[(size_t)c * d + n];",
+        "for (int c = 0; c < d; ++c) acc += qp[(size_t)i * d + c] * S[(size_t)c * d + n];"),
+    "token_level_residual_against_frame_state": (
+        "for (int c = 0; c < d; ++c) acc += kp[(size_t)i * d + c] * St[(size_t)c * d + n];",
+        "for (int c = 0; c < d; ++c) acc += kp[(size_t)i * d + c] * S[(size_t)c * d + n];"),
+    "token_level_gate_every_token": ("if (i == 0) g = alpha_per_key", "if (1) g = alpha_per_key"),
 }
 
 

@@ -91,7 +91,8 @@ def test_hand_worked_case(case):
     alpha = np.asarray(a, dtype=np.float64)[None, None] if isinstance(a, list) else np.array([[a]])
     beta = np.asarray(case.get("beta", [0.0] * L), dtype=np.float64)[None, None]
     clean = "expected_S" in case
-    out, S_new = oracle.frame_pass(q, k, v, wq, wk, wv, alpha, beta, S, clean)
+    run_pass = oracle.frame_pass_token_level if case.get("access") == "token" else oracle.frame_pass
+    out, S_new = run_pass(q, k, v, wq, wk, wv, alpha, beta, S, clean)
     if "expected_out" in case:
         np.testing.assert_allclose(out[0, :, 0, :], case["expected_out"], rtol=0, atol=1e-12)
     if clean:
@@ -379,3 +380,102 @@ def test_elementwise_gate_enters_as_a_row_scaling_of_the_previous_state():
     with_gate = oracle.state_update(k, v, wk, wv, a, beta, S)
     no_gate = oracle.state_update(k, v, wk, wv, np.zeros_like(a), beta, S)
     np.testing.assert_allclose(with_gate - no_gate, a[:, :, :, None] * S, rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Token-level (sequential) access: the ablation of technical summary §2.2
+# "Frame-Level Access" (atlas summary, "Surprising findings")
+# --------------------------------------------------------------------------
+
+def _pass_inputs(seed, B=2, H=2, d=6, L=9):
+    rng = np.random.default_rng(seed)
+    x = {n: rng.normal(size=(B, L, H, d)) for n in ("q", "k", "v")}
+    x.update({n: np.eye(d) + 0.3 * rng.normal(size=(H, d, d)) for n in ("wq", "wk", "wv")})
+    x["alpha"] = rng.random((B, H))
+    x["beta"] = rng.random((B, H, L))
+    x["S"] = rng.normal(size=(B, H, d, d))
+    return rng, x
+
+
+def _tl(x, clean=True, **kw):
+    y = dict(x, **kw)
+    return oracle.frame_pass_token_level(y["q"], y["k"], y["v"], y["wq"], y["wk"], y["wv"],
+                                         y["alpha"], y["beta"], y["S"], clean)
+
+
+def _fl(x, clean=True, **kw):
+    y = dict(x, **kw)
+    return oracle.frame_pass(y["q"], y["k"], y["v"], y["wq"], y["wk"], y["wv"], y["alpha"], y["beta"],
+                             y["S"], clean)
+
+
+def test_token_level_with_one_token_is_the_frame_level_rule():
+    _, x = _pass_inputs(51, L=1)
+    o_t, s_t = _tl(x)
+    o_f, s_f = _fl(x)
+    assert np.array_equal(o_t, o_f) and np.array_equal(s_t, s_f)
+
+
+def test_token_level_without_writes_reads_the_frame_state():
+    # beta = 0 and alpha = 1: no token changes the state, so every token
+    # reads S_{N-1} exactly as under frame-level access
+    _, x = _pass_inputs(52)
+    kw = dict(beta=np.zeros_like(x["beta"]), alpha=np.ones_like(x["alpha"]))
+    o_t, s_t = _tl(x, **kw)
+    o_f, s_f = _fl(x, **kw)
+    np.testing.assert_allclose(o_t, o_f, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(s_t, x["S"], rtol=0, atol=0)
+
+
+def test_token_level_orthonormal_keys_end_in_the_frame_level_state():
+    # with orthonormal k' (L <= d) and alpha = 1 each token's residual is the
+    # same against S^(i) as against S_{N-1}: the final states agree, and
+    # token i's read differs by q'_i sum_{j<i} beta_j k'_j^T u_j
+    rng, x = _pass_inputs(53, B=1, H=1, d=8, L=5)
+    Qm, _ = np.linalg.qr(rng.normal(size=(8, 8)))
+    k = Qm[:5][None, :, None, :]
+    kw = dict(k=k, wk=np.eye(8)[None], alpha=np.ones((1, 1)))
+    o_t, s_t = _tl(x, **kw)
+    o_f, s_f = _fl(x, **kw)
+    np.testing.assert_allclose(s_t, s_f, rtol=0, atol=1e-12)
+    qp = x["q"][0, :, 0, :] @ x["wq"][0]
+    vp = x["v"][0, :, 0, :] @ x["wv"][0]
+    u = vp - k[0, :, 0, :] @ x["S"][0, 0]
+    b = x["beta"][0, 0]
+    for i in range(5):
+        extra = sum(b[j] * (qp[i] @ k[0, j, 0]) * u[j] for j in range(i)) if i else 0.0
+        np.testing.assert_allclose(o_t[0, i, 0] - o_f[0, i, 0], extra, rtol=0, atol=1e-12)
+
+
+def test_token_level_reads_ignore_later_tokens():
+    # the inter-frame part of token i (token-level minus frame-level output,
+    # whose intra parts agree) depends on no token after i
+    _, x = _pass_inputs(54)
+    base = _tl(x)[0] - _fl(x)[0]
+    v2 = x["v"].copy()
+    v2[:, -1] += 5.0
+    pert = _tl(x, v=v2)[0] - _fl(x, v=v2)[0]
+    np.testing.assert_allclose(pert[:, :-1], base[:, :-1], rtol=0, atol=1e-12)
+    assert np.abs(pert[:, -1] - base[:, -1]).max() < 1e-12  # its own read precedes its write
+
+
+def test_token_level_noisy_pass_keeps_the_state():
+    _, x = _pass_inputs(55)
+    o_noisy, s_noisy = _tl(x, clean=False)
+    o_clean, _ = _tl(x, clean=True)
+    assert np.array_equal(s_noisy, x["S"])
+    assert np.array_equal(o_noisy, o_clean)
+
+
+def test_token_level_gate_acts_once_per_frame():
+    # beta = 0: the only change is the gate with token 0's update, so tokens
+    # after the first read alpha S_{N-1} and the frame ends in alpha S_{N-1}
+    # (not alpha^L S_{N-1})
+    _, x = _pass_inputs(56)
+    kw = dict(beta=np.zeros_like(x["beta"]))
+    o_t, s_t = _tl(x, **kw)
+    np.testing.assert_allclose(s_t, x["alpha"][:, :, None, None] * x["S"], rtol=0, atol=1e-12)
+    o_f, _ = _fl(x, **kw)
+    o_g, _ = _fl(x, S=x["alpha"][:, :, None, None] * x["S"], **kw)
+    np.testing.assert_allclose(o_t[:, 0], o_f[:, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o_t[:, 1:], o_g[:, 1:], rtol=0, atol=1e-12)
