@@ -72,6 +72,12 @@ def measured_traffic() -> int | None:
         return None
 
 
+def fp32_simt_tflops() -> float:
+    """Peak fp32 FMA throughput from the unit counts and the clock: 148 SMs x
+    128 FP32 lanes x 2 flop per FMA x 1965 MHz (B200)."""
+    return 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def load_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -289,6 +295,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--gating", default="headwise", choices=["headwise", "elementwise"],
                     help="forget gate per head (the pages' form) or per key feature")
+    ap.add_argument("--access", default="frame", choices=["frame", "token"],
+                    help="frame-level state access (the method) or token-level (the ablation)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-passes", type=int, default=0,
                     help="profiling case: run this many read-only passes over a ring of inputs "
@@ -312,7 +320,7 @@ def main():
     stream_idx = rank  # each rank: its own independent stream (replica)
     wq, wk, wv = workloads.phi_weights(w, 0)
     lay = Arl2Layer(w.batch, w.heads, w.head_dim, w.tokens, wq.cuda(), wk.cuda(), wv.cuda(),
-                    dtype=w.torch_dtype, host_staging=True, gating=args.gating)
+                    dtype=w.torch_dtype, host_staging=True, gating=args.gating, access=args.access)
     gate_draw = workloads.frame_gates_elementwise if args.gating == "elementwise" else workloads.frame_gates
     # all inputs of the stream, resident in HBM before timing
     ins, gates = [], []
@@ -443,13 +451,28 @@ def main():
 
     peaks = load_peaks()
     k_ms = float(np.mean(kernel_ms))
-    achieved = attn_flops(w) / (k_ms / 1e3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": measured_traffic(), "kernel": "attn_tc_kernel",
-                "kernel_ms": k_ms, "flops_per_launch": attn_flops(w),
-                "peak_kind": f"bf16 sustained ({peaks['source']})",
-                "frac_of_burst": achieved / peaks["bf16_tflops"]}
+    if args.access == "token":
+        # the ablation's read-only pass: the fused kernel for the intra-frame
+        # term, then fp32 SIMT phi maps and the chunked sequential scan; its
+        # algorithmic work is the intra term plus, per token, the three phi
+        # maps and the sequential read, residual and update (6 d^2 per head)
+        L, d, H, B = w.tokens, w.head_dim, w.heads, w.batch
+        flops = (4.0 * L * L * d * H + 6.0 * L * d * d * H + 6.0 * L * d * d * H) * B
+        achieved = flops / (k_ms / 1e3) / 1e12
+        peak = fp32_simt_tflops()
+        roofline = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "kernel": "token-level pass (attn_tc_kernel, phi_simt x3, tl_prep, tl_scan)",
+                    "kernel_ms": k_ms, "flops_per_launch": flops,
+                    "peak_kind": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1965 MHz (unit counts x clock)"}
+    else:
+        achieved = attn_flops(w) / (k_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": measured_traffic(), "kernel": "attn_tc_kernel",
+                    "kernel_ms": k_ms, "flops_per_launch": attn_flops(w),
+                    "peak_kind": f"bf16 sustained ({peaks['source']})",
+                    "frac_of_burst": achieved / peaks["bf16_tflops"]}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -465,7 +488,7 @@ def main():
         "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
                    "tokens_per_frame": w.tokens, "frames_per_step": w.frames, "passes": w.passes,
                    "parallelism": f"replicas{ws}", "l2": "inputs larger than L2 (1.2 GB ring)",
-                   "gating": args.gating},
+                   "gating": args.gating, "access": args.access},
         "tokens_per_s": value * w.tokens,
         "tflops_per_frame_algorithmic": frame_flops(w) / 1e12,
         "roofline": roofline, "clocks": clk,

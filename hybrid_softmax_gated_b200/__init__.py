@@ -28,6 +28,7 @@ ARL2_ERR_TIMEOUT = -6
 ARL2_BF16, ARL2_FP32 = 0, 1
 ARL2_IMPL_AUTO, ARL2_IMPL_SIMT = 0, 1
 ARL2_GATE_HEADWISE, ARL2_GATE_ELEMENTWISE = 0, 1
+ARL2_ACCESS_FRAME, ARL2_ACCESS_TOKEN = 0, 1
 
 EXPORTED = (
     "arl2_create", "arl2_frame_forward", "arl2_frame_forward_host", "arl2_state_reset",
@@ -44,7 +45,7 @@ class Arl2Config(ctypes.Structure):
         ("tokens_per_frame", ctypes.c_int), ("dtype", ctypes.c_int),
         ("w_q", ctypes.c_void_p), ("w_k", ctypes.c_void_p), ("w_v", ctypes.c_void_p),
         ("softmax_scale", ctypes.c_float), ("host_staging", ctypes.c_int), ("impl", ctypes.c_int),
-        ("max_ctas", ctypes.c_int), ("gating", ctypes.c_int),
+        ("max_ctas", ctypes.c_int), ("gating", ctypes.c_int), ("access", ctypes.c_int),
     ]
 
 
@@ -131,7 +132,7 @@ class Arl2Layer:
     def __init__(self, batch: int, heads: int, head_dim: int, tokens: int, w_q, w_k, w_v, *,
                  dtype: torch.dtype = torch.bfloat16, softmax_scale: float = 0.0,
                  host_staging: bool = False, impl: str = "auto", max_ctas: int = 0,
-                 gating: str = "headwise", stream=None):
+                 gating: str = "headwise", access: str = "frame", stream=None):
         if dtype not in (torch.bfloat16, torch.float32):
             raise ValueError("dtype must be torch.bfloat16 or torch.float32")
         for w in (w_q, w_k, w_v):
@@ -147,7 +148,9 @@ class Arl2Layer:
                          w_q.data_ptr(), w_k.data_ptr(), w_v.data_ptr(), float(softmax_scale),
                          1 if host_staging else 0,
                          {"auto": ARL2_IMPL_AUTO, "simt": ARL2_IMPL_SIMT}[impl], int(max_ctas),
-                         {"headwise": ARL2_GATE_HEADWISE, "elementwise": ARL2_GATE_ELEMENTWISE}[gating])
+                         {"headwise": ARL2_GATE_HEADWISE, "elementwise": ARL2_GATE_ELEMENTWISE}[gating],
+                         {"frame": ARL2_ACCESS_FRAME, "token": ARL2_ACCESS_TOKEN}[access])
+        self.token_level = access == "token"
         self.alpha_shape = lambda B, H: (B, H, head_dim) if gating == "elementwise" else (B, H)
         h = ctypes.c_void_p()
         with torch.cuda.device(self.device):
@@ -179,9 +182,10 @@ class Arl2Layer:
             out = torch.empty_like(q)
         self._tok(out, "out")
         B, L, H, _ = self.shape
-        if clean_pass:
+        gates = clean_pass or self.token_level  # token-level access reads the gates on every pass
+        if gates:
             if alpha is None or beta is None:
-                raise ValueError("the clean pass needs alpha and beta")
+                raise ValueError("this pass needs alpha and beta")
             if not (alpha.is_cuda and alpha.dtype == torch.float32 and alpha.is_contiguous()
                     and tuple(alpha.shape) == self.alpha_shape(B, H)):
                 raise ValueError(f"alpha must be a contiguous fp32 CUDA tensor {list(self.alpha_shape(B, H))}")
@@ -189,8 +193,8 @@ class Arl2Layer:
                     and tuple(beta.shape) == (B, H, L)):
                 raise ValueError("beta must be a contiguous fp32 CUDA tensor [B, H, L]")
         _check(_lib.arl2_frame_forward(self.handle, _ptr(q), _ptr(k), _ptr(v),
-                                       _ptr(alpha) if clean_pass else None,
-                                       _ptr(beta) if clean_pass else None,
+                                       _ptr(alpha) if gates else None,
+                                       _ptr(beta) if gates else None,
                                        1 if clean_pass else 0, _ptr(out), _stream(stream)),
                "arl2_frame_forward")
         return out
@@ -200,11 +204,12 @@ class Arl2Layer:
         for t in (q, k, v, out):
             if t.is_cuda or not t.is_contiguous() or tuple(t.shape) != self.shape or t.dtype != self.dtype:
                 raise ValueError("host token tensors must be contiguous CPU tensors of the layer shape")
-        if clean_pass and (alpha is None or beta is None or alpha.is_cuda or beta.is_cuda):
-            raise ValueError("the clean pass needs host alpha and beta")
+        gates = clean_pass or self.token_level
+        if gates and (alpha is None or beta is None or alpha.is_cuda or beta.is_cuda):
+            raise ValueError("this pass needs host alpha and beta")
         _check(_lib.arl2_frame_forward_host(self.handle, _ptr(q), _ptr(k), _ptr(v),
-                                            _ptr(alpha) if clean_pass else None,
-                                            _ptr(beta) if clean_pass else None,
+                                            _ptr(alpha) if gates else None,
+                                            _ptr(beta) if gates else None,
                                             1 if clean_pass else 0, _ptr(out), _stream(stream)),
                "arl2_frame_forward_host")
         return out

@@ -59,6 +59,10 @@ struct arl2_handle {
     float* stage_alpha = nullptr;
     float* stage_beta = nullptr;
     int alpha_per_key = 0;    // elementwise gating: alpha [B][H][d] instead of [B][H]
+    int token_level = 0;      // token-level (sequential) access instead of frame-level
+    float* tl_ws = nullptr;   // token-level chunk workspace
+    void* zero_read = nullptr;  // zero state for the intra-only attention launch
+                                // (bf16 Mt on the tensor-core path, fp32 S on SIMT)
     int* err = nullptr;       // device error word
     unsigned long long launches = 0;  // kernels enqueued by this handle
 };
@@ -97,7 +101,7 @@ void release(arl2_handle* h) {
     delete h->maps;
     void* ptrs[] = {h->w_all, h->S, h->Mt, h->Sb, h->part_s, h->attn_ws, h->qp, h->kp,
                     h->vp, h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], h->stage_tok[3],
-                    h->stage_alpha, h->stage_beta, h->err};
+                    h->stage_alpha, h->stage_beta, h->err, h->tl_ws, h->zero_read};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     delete h;
@@ -173,6 +177,7 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
     if (cfg->max_ctas < 0) return ARL2_ERR_INVALID_ARG;
     if (cfg->gating != ARL2_GATE_HEADWISE && cfg->gating != ARL2_GATE_ELEMENTWISE)
         return ARL2_ERR_INVALID_ARG;
+    if (cfg->access != ARL2_ACCESS_FRAME && cfg->access != ARL2_ACCESS_TOKEN) return ARL2_ERR_INVALID_ARG;
     if (!aligned16(cfg->w_q) || !aligned16(cfg->w_k) || !aligned16(cfg->w_v)) return ARL2_ERR_ALIGN;
     const bool use_tc = cfg->impl == ARL2_IMPL_AUTO && cfg->dtype == ARL2_BF16;
     if (use_tc && cfg->head_dim != 128) return ARL2_ERR_UNSUPPORTED;
@@ -188,6 +193,7 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
     h->impl = cfg->impl;
     h->use_tc = use_tc;
     h->alpha_per_key = cfg->gating == ARL2_GATE_ELEMENTWISE ? 1 : 0;
+    h->token_level = cfg->access == ARL2_ACCESS_TOKEN ? 1 : 0;
     h->scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->head_dim);
     h->esz = cfg->dtype == ARL2_BF16 ? 2 : 4;
     const Dims& dm = h->dm;
@@ -207,10 +213,16 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
         if (s == ARL2_OK) s = dalloc(h, &h->Sb, h->n_state * 2);
         if (s == ARL2_OK) s = dalloc(h, &h->part_s, parts * sizeof(float));
         if (s == ARL2_OK) s = dalloc(h, &h->attn_ws, arl2::attn_tc_workspace_bytes(dm));
-    } else {
+    }
+    if (!use_tc || h->token_level) {
         if (s == ARL2_OK) s = dalloc(h, &h->qp, h->n_tok * sizeof(float));
         if (s == ARL2_OK) s = dalloc(h, &h->kp, h->n_tok * sizeof(float));
         if (s == ARL2_OK) s = dalloc(h, &h->vp, h->n_tok * sizeof(float));
+    }
+    if (h->token_level) {
+        if (s == ARL2_OK) s = dalloc(h, &h->tl_ws, arl2::tl_workspace_floats(dm) * sizeof(float));
+        if (s == ARL2_OK) s = dalloc(h, &h->zero_read, h->n_state * (use_tc ? 2 : sizeof(float)));
+        if (s == ARL2_OK && arl2::tl_init() != cudaSuccess) s = ARL2_ERR_CUDA;
     }
     if (s == ARL2_OK && cfg->host_staging) {
         for (int i = 0; i < 4 && s == ARL2_OK; ++i) s = dalloc(h, &h->stage_tok[i], h->n_tok * h->esz);
@@ -240,6 +252,9 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
     if (s == ARL2_OK && use_tc &&
         cudaMemsetAsync(h->attn_ws, 0, arl2::attn_tc_workspace_bytes(dm), stream) != cudaSuccess)
         s = ARL2_ERR_CUDA;
+    if (s == ARL2_OK && h->token_level &&
+        cudaMemsetAsync(h->zero_read, 0, h->n_state * (use_tc ? 2 : sizeof(float)), stream) != cudaSuccess)
+        s = ARL2_ERR_CUDA;
     if (s != ARL2_OK) {
         cudaStreamSynchronize(stream);
         release(h);
@@ -249,16 +264,52 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
     return ARL2_OK;
 }
 
+// Token-level access: the intra-frame term through the usual attention
+// kernel reading a zero state, the phi maps in fp32, then the chunked
+// sequential read/update (token_level.cu), which adds q'_i S^(i) to out and
+// keeps S^(L) on the clean pass.
+static arl2_status token_level_pass(arl2_handle* h, const void* q, const void* k, const void* v,
+                                    const float* alpha, const float* beta, bool clean, void* out,
+                                    cudaStream_t st) {
+    const bool bf16 = h->dtype == ARL2_BF16;
+    const Dims& dm = h->dm;
+    if (h->use_tc) {
+        ++h->launches;
+        if (arl2::attn_tc_launch(h->tc, *h->maps, q, k, v, h->zero_read, out, h->scale, h->err, st) !=
+                cudaSuccess ||
+            arl2::launch_phi_simt(bf16, q, h->w[0], false, h->qp, nullptr, dm, st) != cudaSuccess)
+            return ARL2_ERR_CUDA;
+        ++h->launches;
+    } else {
+        h->launches += 2;
+        if (arl2::launch_phi_simt(bf16, q, h->w[0], false, h->qp, nullptr, dm, st) != cudaSuccess ||
+            arl2::launch_attn_simt(bf16, q, k, v, h->qp, static_cast<const float*>(h->zero_read), out,
+                                   h->scale, dm, st) != cudaSuccess)
+            return ARL2_ERR_CUDA;
+    }
+    h->launches += 4;
+    if (arl2::launch_phi_simt(bf16, k, h->w[1], true, h->kp, nullptr, dm, st) != cudaSuccess ||
+        arl2::launch_phi_simt(bf16, v, h->w[2], false, h->vp, nullptr, dm, st) != cudaSuccess ||
+        arl2::launch_tl(h->qp, h->kp, h->vp, alpha, h->alpha_per_key, beta, h->tl_ws, h->S, out, bf16,
+                        clean, dm, st) != cudaSuccess)
+        return ARL2_ERR_CUDA;
+    // the tensor-core copies of the state follow S (checkpoint consistency)
+    if (clean) return refresh_derived(h, st);
+    return ARL2_OK;
+}
+
 arl2_status arl2_frame_forward(arl2_handle* h, const void* q, const void* k, const void* v,
                                const float* alpha, const float* beta, int clean_pass, void* out,
                                cudaStream_t stream) {
     if (!h || !q || !k || !v || !out) return ARL2_ERR_INVALID_ARG;
-    if (clean_pass && (!alpha || !beta)) return ARL2_ERR_INVALID_ARG;
+    // token-level access reads through the gates on every pass
+    if ((clean_pass || h->token_level) && (!alpha || !beta)) return ARL2_ERR_INVALID_ARG;
     if (out == q || out == k || out == v) return ARL2_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ARL2_ERR_ALIGN;
     arl2_status s = check_device(h);
     if (s != ARL2_OK) return s;
     const bool bf16 = h->dtype == ARL2_BF16;
+    if (h->token_level) return token_level_pass(h, q, k, v, alpha, beta, clean_pass != 0, out, stream);
     if (h->use_tc) {
         ++h->launches;
         if (arl2::attn_tc_launch(h->tc, *h->maps, q, k, v, h->Mt, out, h->scale, h->err, stream) !=
@@ -280,7 +331,8 @@ arl2_status arl2_frame_forward_host(arl2_handle* h, const void* q, const void* k
                                     void* out, cudaStream_t stream) {
     if (!h || !q || !k || !v || !out) return ARL2_ERR_INVALID_ARG;
     if (!h->stage_tok[0]) return ARL2_ERR_INVALID_ARG;
-    if (clean_pass && (!alpha || !beta)) return ARL2_ERR_INVALID_ARG;
+    const bool gates = clean_pass || h->token_level;  // the passes that read alpha and beta
+    if (gates && (!alpha || !beta)) return ARL2_ERR_INVALID_ARG;
     arl2_status s = check_device(h);
     if (s != ARL2_OK) return s;
     const size_t tb = h->n_tok * h->esz;
@@ -290,7 +342,7 @@ arl2_status arl2_frame_forward_host(arl2_handle* h, const void* q, const void* k
             return ARL2_ERR_CUDA;
     const float* a_dev = nullptr;
     const float* b_dev = nullptr;
-    if (clean_pass) {
+    if (gates) {
         const Dims& dm = h->dm;
         if (cudaMemcpyAsync(h->stage_alpha, alpha, (size_t)dm.B * dm.H * (h->alpha_per_key ? dm.d : 1) * sizeof(float),
                             cudaMemcpyHostToDevice, stream) != cudaSuccess ||

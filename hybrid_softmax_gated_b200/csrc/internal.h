@@ -51,4 +51,16 @@ cudaError_t launch_accum_simt(const float* kp, const float* r, const float* alph
 cudaError_t launch_fold_state(const void* wq_bf16, const float* S, void* Mt, void* Sb, Dims dm,
                               cudaStream_t st);
 
+// ---- token-level (sequential) access, fp32 (token_level.cu) ------------
+// Chunks of the frame and the fp32 workspace of one pass.
+int tl_chunks(const Dims& dm);
+size_t tl_workspace_floats(const Dims& dm);
+cudaError_t tl_init();  // kernel attributes, once (arl2_create)
+// Adds q'_i S^(i) to out for every token (out already holds the intra-frame
+// term) and, when clean, stores S^(L) in S.  qp, kp (row-normalised), vp:
+// fp32 [B][L][H][d]; alpha [B][H] or [B][H][d]; beta [B][H][L].
+cudaError_t launch_tl(const float* qp, const float* kp, const float* vp, const float* alpha,
+                      int alpha_per_key, const float* beta, float* ws, float* S, void* out, bool bf16,
+                      bool clean, Dims dm, cudaStream_t st);
+
 }  // namespace arl2

@@ -73,6 +73,18 @@ typedef enum { ARL2_IMPL_AUTO = 0, ARL2_IMPL_SIMT = 1 } arl2_impl;
 /* Granularity of the forget gate alpha (see the conventions above). */
 typedef enum { ARL2_GATE_HEADWISE = 0, ARL2_GATE_ELEMENTWISE = 1 } arl2_gating;
 
+/* How the frame's tokens reach the state.  FRAME (the method, technical
+ * summary §2.2 "Frame-Level Access"): every token reads S_{N-1} and the
+ * clean pass updates once.  TOKEN (the ablation the pages compare with it):
+ * token i reads the state left by tokens 0..i-1 of the pass and then updates
+ * it with the delta rule, S <- G_i S + beta_i k'_i^T (v'_i - k'_i S), the
+ * forget gate acting once with token 0 (G_0 = alpha, G_i = 1); every pass
+ * reads through its own sequential states, so alpha and beta are required on
+ * every pass, and only the clean pass keeps the final state.  TOKEN runs on
+ * fp32 SIMT kernels for the sequential part (bf16 inputs are widened); with
+ * bf16 its output is rounded twice (the intra-frame term, then the sum). */
+typedef enum { ARL2_ACCESS_FRAME = 0, ARL2_ACCESS_TOKEN = 1 } arl2_access;
+
 typedef struct arl2_handle arl2_handle;
 
 typedef struct {
@@ -92,6 +104,7 @@ typedef struct {
                               SM; > 0 caps its persistent grid (co-scheduling
                               with other work, tests of the split schedule)   */
     arl2_gating gating;    /* HEADWISE: alpha [B][H]; ELEMENTWISE: [B][H][d]  */
+    arl2_access access;    /* FRAME (the method) or TOKEN (the ablation)      */
 } arl2_config;
 
 /* Create a layer on the current device.  Validates cfg, allocates the zeroed
@@ -104,7 +117,8 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
 /* One denoising pass of one latent frame (technical summary §2.1, §2.2).
  * Writes out = O_intra + O_inter for every token, reading S_{N-1}.  When
  * clean_pass is nonzero, then also updates the state in place to S_N; alpha
- * and beta are read only in that case and may be NULL otherwise.
+ * and beta are read only in that case and may be NULL otherwise (with
+ * access = ARL2_ACCESS_TOKEN they are read on every pass, see above).
  * q, k, v, out: device [B][L][H][d] dtype, 16-byte aligned; out must not
  * alias q, k or v.  alpha: device fp32 [B][H] ([B][H][d] with elementwise
  * gating); beta: device fp32 [B][H][L]. */

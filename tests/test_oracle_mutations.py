@@ -45,7 +45,8 @@ MUTATIONS = {
         "S[(size_t)c * d + n] = a * S[(size_t)c * d + n] + dS[(size_t)c * d + n];",
         "S[(size_t)c * d + n] = (alpha_per_key ? alpha[((size_t)b * H + h) * d + n] : a)"
         " * S[(size_t)c * d + n] + dS[(size_t)c * d + n];"),
-    "elementwise_gate_one_value": ("alpha[((size_t)b * H + h) * d + c]", "alpha[((size_t)b * H + h) * d]"),
+    "elementwise_gate_one_value": ("const double a = alpha_per_key ? alpha[((size_t)b * H + h) * d + c]",
+                                   "const double a = alpha_per_key ? alpha[((size_t)b * H + h) * d]"),
     "token_level_reads_frame_state": (
         "for (int c = 0; c < d; ++c) acc += qp[(size_t)i * d + c] * St[(size_t)c * d + n];",
         "for (int c = 0; c < d; ++c) acc += qp[(size_t)i * d + c] * S[(size_t)c * d + n];"),
