@@ -28,52 +28,100 @@ __device__ __forceinline__ size_t tok(int b, int t, int h, int c, const Dims& dm
 }
 
 // ---------------------------------------------------------------- phi ----
-constexpr int kPhiRows = 32;
+// One CTA: 128 tokens of one (b, h); 256 threads, thread (rg, cg) computes
+// rows 8 rg .. 8 rg + 7 and columns 8 cg .. 8 cg + 7 of x W[h] from W and
+// the token rows staged in shared memory (fp32), then the optional row
+// L2 norm (the 16 threads of a row group hold a whole row: half a warp).
+constexpr int kPhiRows = 128;
+constexpr int kPhiThreads = 256;
 
 template <typename T>
-__global__ void __launch_bounds__(128) phi_simt_kernel(const T* __restrict__ x,
-                                                       const T* __restrict__ w, int l2norm,
-                                                       float* __restrict__ out_f,
-                                                       T* __restrict__ out_t, Dims dm) {
+__device__ __forceinline__ void store8(T* p, const float* y, bool full, int n);
+template <>
+__device__ __forceinline__ void store8<float>(float* p, const float* y, bool full, int n) {
+    if (full) {
+        reinterpret_cast<float4*>(p)[0] = make_float4(y[0], y[1], y[2], y[3]);
+        reinterpret_cast<float4*>(p)[1] = make_float4(y[4], y[5], y[6], y[7]);
+    } else {
+        for (int e = 0; e < n; ++e) p[e] = y[e];
+    }
+}
+template <>
+__device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16* p, const float* y, bool full, int n) {
+    if (full) {
+        uint4 u;
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]), h1 = __floats2bfloat162_rn(y[2], y[3]);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4], y[5]), h3 = __floats2bfloat162_rn(y[6], y[7]);
+        u.x = *reinterpret_cast<uint32_t*>(&h0);
+        u.y = *reinterpret_cast<uint32_t*>(&h1);
+        u.z = *reinterpret_cast<uint32_t*>(&h2);
+        u.w = *reinterpret_cast<uint32_t*>(&h3);
+        *reinterpret_cast<uint4*>(p) = u;
+    } else {
+        for (int e = 0; e < n; ++e) p[e] = __float2bfloat16_rn(y[e]);
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kPhiThreads) phi_simt_kernel(const T* __restrict__ x,
+                                                               const T* __restrict__ w, int l2norm,
+                                                               float* __restrict__ out_f,
+                                                               T* __restrict__ out_t, Dims dm) {
     extern __shared__ float sm[];
     const int d = dm.d;
-    float* Ws = sm;                 // [d][d]
-    float* Xs = Ws + d * d;         // [kPhiRows][d]
-    float* Ys = Xs + kPhiRows * d;  // [kPhiRows][d]
-    __shared__ float inv[kPhiRows];
+    float* Ws = sm;                 // [d][128]
+    float* Xs = Ws + d * 128;       // [kPhiRows][d]
     const int h = blockIdx.y, b = blockIdx.z;
     const int t0 = blockIdx.x * kPhiRows;
     const int nt = min(kPhiRows, dm.L - t0);
-    for (int i = threadIdx.x; i < d * d; i += blockDim.x) Ws[i] = to_f(w[(size_t)h * d * d + i]);
-    for (int i = threadIdx.x; i < nt * d; i += blockDim.x) {
+    for (int i = threadIdx.x; i < d * 128; i += blockDim.x) {
+        const int a = i >> 7, c = i & 127;
+        Ws[i] = c < d ? to_f(w[((size_t)h * d + a) * d + c]) : 0.f;
+    }
+    for (int i = threadIdx.x; i < kPhiRows * d; i += blockDim.x) {
         const int r = i / d, c = i - r * d;
-        Xs[i] = to_f(x[tok(b, t0 + r, h, c, dm)]);
+        Xs[i] = r < nt ? to_f(x[tok(b, t0 + r, h, c, dm)]) : 0.f;
     }
     __syncthreads();
-    const int c = threadIdx.x;
-    if (c < d) {
-        for (int r = 0; r < nt; ++r) {
-            float acc = 0.f;
-            for (int a = 0; a < d; ++a) acc = fmaf(Xs[r * d + a], Ws[a * d + c], acc);
-            Ys[r * d + c] = acc;
+    const int rg = threadIdx.x >> 4, cg = threadIdx.x & 15;
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
+    for (int a = 0; a < d; ++a) {
+        float xr[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xr[i] = Xs[(rg * 8 + i) * d + a];
+        const float4 w0 = *reinterpret_cast<const float4*>(Ws + a * 128 + cg * 8);
+        const float4 w1 = *reinterpret_cast<const float4*>(Ws + a * 128 + cg * 8 + 4);
+        const float wc[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) acc[i][jj] = fmaf(xr[i], wc[jj], acc[i][jj]);
+    }
+    const int c0 = cg * 8;
+    const int ncol = max(0, min(8, d - c0));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float inv = 1.f;
+        if (l2norm) {
+            float ss = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) ss = fmaf(acc[i][jj], acc[i][jj], ss);
+            for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            inv = 1.f / fmaxf(sqrtf(ss), 1e-6f);
         }
-    }
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int r = warp; r < nt; r += blockDim.x >> 5) {
-        float ss = 0.f;
-        if (l2norm)
-            for (int cc = lane; cc < d; cc += 32) ss = fmaf(Ys[r * d + cc], Ys[r * d + cc], ss);
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (lane == 0) inv[r] = l2norm ? 1.f / fmaxf(sqrtf(ss), 1e-6f) : 1.f;
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < nt * d; i += blockDim.x) {
-        const int r = i / d, cc = i - r * d;
-        const float y = Ys[i] * inv[r];
-        const size_t o = tok(b, t0 + r, h, cc, dm);
-        if (out_f) out_f[o] = y;
-        else out_t[o] = from_f<T>(y);
+        const int r = rg * 8 + i;
+        if (r >= nt || ncol == 0) continue;
+        float y[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) y[jj] = acc[i][jj] * inv;
+        const size_t o = tok(b, t0 + r, h, c0, dm);
+        const bool full = ncol == 8 && (d & 7) == 0;
+        if (out_f) store8<float>(out_f + o, y, full, ncol);
+        else store8<T>(out_t + o, y, full, ncol);
     }
 }
 
@@ -249,7 +297,7 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 }
 
 // Dynamic shared memory of each kernel at the largest head_dim (128).
-constexpr size_t kPhiSmemMax = sizeof(float) * (128 * 128 + 2 * kPhiRows * 128);
+constexpr size_t kPhiSmemMax = sizeof(float) * (128 * 128 + kPhiRows * 128);
 constexpr size_t kAttnSmemMax =
     sizeof(float) * (kAQ * 128 + kAK * 129 + kAK * 128 + kAQ * (kAK + 1) + 128 * 128);
 constexpr size_t kResidualSmemMax = sizeof(float) * (128 * 128 + kRRows * 128);
@@ -267,13 +315,13 @@ cudaError_t simt_init() {
 
 cudaError_t launch_phi_simt(bool bf16, const void* x, const void* w, bool l2norm, float* out_f,
                             void* out_t, Dims dm, cudaStream_t st) {
-    const size_t smem = sizeof(float) * ((size_t)dm.d * dm.d + 2 * kPhiRows * dm.d);
+    const size_t smem = sizeof(float) * ((size_t)dm.d * 128 + (size_t)kPhiRows * dm.d);
     const dim3 grid((dm.L + kPhiRows - 1) / kPhiRows, dm.H, dm.B);
     if (bf16) {
-        phi_simt_kernel<__nv_bfloat16><<<grid, 128, smem, st>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)w, l2norm,
+        phi_simt_kernel<__nv_bfloat16><<<grid, kPhiThreads, smem, st>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)w, l2norm,
                                      out_f, (__nv_bfloat16*)out_t, dm);
     } else {
-        phi_simt_kernel<float><<<grid, 128, smem, st>>>((const float*)x, (const float*)w, l2norm, out_f,
+        phi_simt_kernel<float><<<grid, kPhiThreads, smem, st>>>((const float*)x, (const float*)w, l2norm, out_f,
                                      (float*)out_t, dm);
     }
     return cudaGetLastError();

@@ -18,8 +18,8 @@
 //   k~_j = k'_j G (j >= 1, chunk 0), k~_j = k'_j otherwise,
 //   o_j  += q~_j S_0 + sum_{i<j} P[j][i] u_i,  P[j][i] = beta_i q'_j . k'_i,
 //   S_C  = G S_0 + (diag(beta) K')^T U.
-// tl_prep_kernel forms, for every chunk independently, T = (I + A)^{-1},
-// T K~, T V', Q~, diag(beta) K' and P; tl_scan_kernel then runs the chunks
+// tl_prep_kernel forms, for every chunk independently, T K~ and T V' with
+// T = (I + A)^{-1} (by forward substitution), Q~, diag(beta) K' and P; tl_scan_kernel then runs the chunks
 // in order for a slice of value features (the columns of S evolve
 // independently), adding the reads into out and, on the clean pass, storing
 // the final state.
@@ -32,6 +32,10 @@ constexpr int kTlChunk = 64;     // C
 constexpr int kTlCols = 16;      // value features per scan CTA
 constexpr int kTlThreads = 256;
 constexpr int kPad = 4;          // row padding of [C][d] staging (bank spread)
+
+// Row stride of [C][d] staging in shared memory: a multiple of 4 floats (for
+// float4 access) plus kPad (bank spread).
+__host__ __device__ inline int padded(int d) { return ((d + 3) & ~3) + kPad; }
 
 __device__ __forceinline__ size_t tokidx(int b, int t, int h, int c, const Dims& dm) {
     return (((size_t)b * dm.L + t) * dm.H + h) * dm.d + c;
@@ -52,7 +56,7 @@ __global__ void __launch_bounds__(kTlThreads) tl_prep_kernel(const float* __rest
                                                             float* __restrict__ ws, Dims dm,
                                                             int n_chunks) {
     extern __shared__ float sm[];
-    const int d = dm.d, dp = d + kPad;
+    const int d = dm.d, dp = padded(d), d4 = (d + 3) / 4;
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t0 = c * kTlChunk;
     float* Ks = sm;                       // [C][dp] k'
@@ -60,16 +64,15 @@ __global__ void __launch_bounds__(kTlThreads) tl_prep_kernel(const float* __rest
     float* Vs = Qs + kTlChunk * dp;       // [C][dp] v'
     float* A = Vs + kTlChunk * dp;        // [C][C]
     float* P = A + kTlChunk * kTlChunk;   // [C][C]
-    float* T = P + kTlChunk * kTlChunk;   // [C][C]
-    float* bs = T + kTlChunk * kTlChunk;  // [C] beta
+    float* bs = P + kTlChunk * kTlChunk;  // [C] beta
     float* gs = bs + kTlChunk;            // [d] gate of chunk 0 per key feature
     const size_t bh = (size_t)b * dm.H + h;
-    for (int i = threadIdx.x; i < kTlChunk * d; i += blockDim.x) {
-        const int j = i / d, e = i - j * d, t = t0 + j;
-        const bool ok = t < dm.L;
-        Ks[j * dp + e] = ok ? kp[tokidx(b, t, h, e, dm)] : 0.f;
-        Qs[j * dp + e] = ok ? qp[tokidx(b, t, h, e, dm)] : 0.f;
-        Vs[j * dp + e] = ok ? vp[tokidx(b, t, h, e, dm)] : 0.f;
+    for (int i = threadIdx.x; i < kTlChunk * dp; i += blockDim.x) {
+        const int j = i / dp, e = i - j * dp, t = t0 + j;
+        const bool ok = t < dm.L && e < d;  // (the row padding is zero: float4 dots)
+        Ks[i] = ok ? kp[tokidx(b, t, h, e, dm)] : 0.f;
+        Qs[i] = ok ? qp[tokidx(b, t, h, e, dm)] : 0.f;
+        Vs[i] = ok ? vp[tokidx(b, t, h, e, dm)] : 0.f;
     }
     for (int j = threadIdx.x; j < kTlChunk; j += blockDim.x)
         bs[j] = t0 + j < dm.L ? beta[bh * dm.L + t0 + j] : 0.f;
@@ -81,9 +84,13 @@ __global__ void __launch_bounds__(kTlThreads) tl_prep_kernel(const float* __rest
         const int j = p / kTlChunk, i = p - j * kTlChunk;
         float a = 0.f, q = 0.f;
         if (i < j) {
-            for (int e = 0; e < d; ++e) {
-                a = fmaf(Ks[j * dp + e], Ks[i * dp + e], a);
-                q = fmaf(Qs[j * dp + e], Ks[i * dp + e], q);
+            const float4* kj = reinterpret_cast<const float4*>(Ks + j * dp);
+            const float4* ki = reinterpret_cast<const float4*>(Ks + i * dp);
+            const float4* qj = reinterpret_cast<const float4*>(Qs + j * dp);
+            for (int e4 = 0; e4 < d4; ++e4) {
+                const float4 x = kj[e4], y = ki[e4], z = qj[e4];
+                a = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, a))));
+                q = fmaf(z.x, y.x, fmaf(z.y, y.y, fmaf(z.z, y.z, fmaf(z.w, y.w, q))));
             }
             a *= bs[i];
             q *= bs[i];
@@ -92,36 +99,35 @@ __global__ void __launch_bounds__(kTlThreads) tl_prep_kernel(const float* __rest
         P[p] = q;
     }
     __syncthreads();
-    // T = (I + A)^{-1}, unit lower triangular: row j = e_j - sum_{i<j} A[j][i] T[i]
-    // (each thread one column m, rows in order)
-    for (int m = threadIdx.x; m < kTlChunk; m += blockDim.x) {
-        for (int j = 0; j < kTlChunk; ++j) {
-            float t = j == m ? 1.f : 0.f;
-            for (int i = m; i < j; ++i) t = fmaf(-A[j * kTlChunk + i], T[i * kTlChunk + m], t);
-            T[j * kTlChunk + m] = j < m ? 0.f : t;
-        }
-    }
-    __syncthreads();
     float* out = ws + (bh * n_chunks + c) * tl_chunk_floats(d);
     float* TK = out;
     float* TV = TK + (size_t)kTlChunk * d;
     float* QG = TV + (size_t)kTlChunk * d;
     float* BK = QG + (size_t)kTlChunk * d;
     float* Pg = BK + (size_t)kTlChunk * d;
-    // T K~ and T V' (k~_i = k'_i G for i >= 1 in chunk 0), Q~, diag(beta) K'
+    // T K~ and T V' with T = (I + A)^{-1}: forward substitution, one
+    // right-hand-side column per thread (K~'s columns, then V''s), rows in
+    // order: x_j = r_j - sum_{i<j} A[j][i] x_i.  k~_i = k'_i G for i >= 1 in
+    // chunk 0.  The solutions overwrite Ks / Vs in place.
+    for (int col = threadIdx.x; col < 2 * d; col += blockDim.x) {
+        const bool is_k = col < d;
+        const int e = is_k ? col : col - d;
+        float* X = is_k ? Ks : Vs;
+        const float g = (is_k && c == 0) ? gs[e] : 1.f;
+        for (int j = 0; j < kTlChunk; ++j) {
+            float x = X[j * dp + e];
+            if (is_k && j >= 1) x *= g;
+            if (is_k) BK[j * d + e] = bs[j] * X[j * dp + e];  // diag(beta) K' (before overwrite)
+            for (int i = 0; i < j; ++i) x = fmaf(-A[j * kTlChunk + i], X[i * dp + e], x);
+            X[j * dp + e] = x;
+        }
+    }
+    __syncthreads();
     for (int p = threadIdx.x; p < kTlChunk * d; p += blockDim.x) {
         const int j = p / d, e = p - j * d;
-        float tk = 0.f, tv = 0.f;
-        for (int i = 0; i <= j; ++i) {
-            const float tji = T[j * kTlChunk + i];
-            const float ki = (c == 0 && i >= 1) ? Ks[i * dp + e] * gs[e] : Ks[i * dp + e];
-            tk = fmaf(tji, ki, tk);
-            tv = fmaf(tji, Vs[i * dp + e], tv);
-        }
-        TK[p] = tk;
-        TV[p] = tv;
+        TK[p] = Ks[j * dp + e];
+        TV[p] = Vs[j * dp + e];
         QG[p] = (c == 0 && j >= 1) ? Qs[j * dp + e] * gs[e] : Qs[j * dp + e];
-        BK[p] = bs[j] * Ks[j * dp + e];
     }
     for (int p = threadIdx.x; p < kTlChunk * kTlChunk; p += blockDim.x) Pg[p] = P[p];
 }
@@ -150,7 +156,7 @@ __global__ void __launch_bounds__(kTlThreads) tl_scan_kernel(const float* __rest
                                                             int alpha_per_key, int clean, Dims dm,
                                                             int n_chunks) {
     extern __shared__ float sm[];
-    const int d = dm.d, dp = d + kPad;
+    const int d = dm.d, dp = padded(d);
     const int n0 = blockIdx.x * kTlCols, h = blockIdx.y, b = blockIdx.z;
     const size_t bh = (size_t)b * dm.H + h;
     float* Ss = sm;                          // [d][16] state slice
@@ -176,11 +182,26 @@ __global__ void __launch_bounds__(kTlThreads) tl_scan_kernel(const float* __rest
         const float* BK = QG + (size_t)kTlChunk * d;
         const float* P = BK + (size_t)kTlChunk * d;
         __syncthreads();  // the previous chunk is done with the staging buffers
-        for (int i = threadIdx.x; i < kTlChunk * d; i += blockDim.x) {
-            const int r = i / d, e = i - r * d;
-            TKs[r * dp + e] = __ldg(TK + i);
-            QGs[r * dp + e] = __ldg(QG + i);
-            BKs[r * dp + e] = __ldg(BK + i);
+        if ((d & 3) == 0) {
+            // float4 loads, many in flight (the chunk's inputs come from L2)
+            const int d4 = d >> 2, n4 = kTlChunk * d4;
+#pragma unroll 4
+            for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+                const int r = i / d4, e = (i - r * d4) * 4;
+                const float4 x = __ldg(reinterpret_cast<const float4*>(TK) + i);
+                const float4 y = __ldg(reinterpret_cast<const float4*>(QG) + i);
+                const float4 z = __ldg(reinterpret_cast<const float4*>(BK) + i);
+                *reinterpret_cast<float4*>(TKs + r * dp + e) = x;
+                *reinterpret_cast<float4*>(QGs + r * dp + e) = y;
+                *reinterpret_cast<float4*>(BKs + r * dp + e) = z;
+            }
+        } else {
+            for (int i = threadIdx.x; i < kTlChunk * d; i += blockDim.x) {
+                const int r = i / d, e = i - r * d;
+                TKs[r * dp + e] = __ldg(TK + i);
+                QGs[r * dp + e] = __ldg(QG + i);
+                BKs[r * dp + e] = __ldg(BK + i);
+            }
         }
         for (int i = threadIdx.x; i < kTlChunk * kTlChunk; i += blockDim.x) Ps[i] = __ldg(P + i);
         for (int i = threadIdx.x; i < kTlChunk * kTlCols; i += blockDim.x) {
@@ -259,10 +280,10 @@ __global__ void __launch_bounds__(kTlThreads) tl_scan_kernel(const float* __rest
 }
 
 size_t prep_smem(int d) {
-    return sizeof(float) * ((size_t)3 * kTlChunk * (d + kPad) + 3 * kTlChunk * kTlChunk + kTlChunk + d);
+    return sizeof(float) * ((size_t)3 * kTlChunk * padded(d) + 2 * kTlChunk * kTlChunk + kTlChunk + d);
 }
 size_t scan_smem(int d) {
-    return sizeof(float) * ((size_t)d * kTlCols + kTlChunk * kTlCols + 3 * (size_t)kTlChunk * (d + kPad) +
+    return sizeof(float) * ((size_t)d * kTlCols + kTlChunk * kTlCols + 3 * (size_t)kTlChunk * padded(d) +
                             kTlChunk * kTlChunk + kTlChunk * kTlCols);
 }
 
