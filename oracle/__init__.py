@@ -11,7 +11,9 @@ the values given to the GPU (bf16- or fp32-rounded).
 
 Method source: "Attend Locally, Remember Linearly" technical summary,
 section 2.1 (hybrid decomposition, phi maps, state update, inter read) and
-section 2.2 (frame-level access, clean-pass updates).
+section 2.2 (frame-level access, clean-pass updates).  The softmax teacher
+layer with a KV cache (teacher_pass) follows section 1 ("KV Cache Growth")
+and section 4 ("Efficiency"): the attention the hybrid layer replaces.
 """
 from __future__ import annotations
 
@@ -55,9 +57,12 @@ def _load():
             lib.arl2_oracle_phi.argtypes = [I, I, I, I, P, P, I, P]
             lib.arl2_oracle_pass_token_level.argtypes = [I, I, I, I, D, P, P, P, P, P, P, P, I, P, I,
                                                          P, P]
+            lib.arl2_oracle_teacher_pass.argtypes = [I, I, I, I, I, D, P, P, P, P, P, P]
+            lib.arl2_oracle_teacher_rows.argtypes = [I, I, I, I, I, D, P, P, P, P, P, I, P, P, P]
             for f in (lib.arl2_oracle_pass, lib.arl2_oracle_rows,
                       lib.arl2_oracle_state_update, lib.arl2_oracle_state_update_gated,
-                      lib.arl2_oracle_phi, lib.arl2_oracle_pass_token_level):
+                      lib.arl2_oracle_phi, lib.arl2_oracle_pass_token_level,
+                      lib.arl2_oracle_teacher_pass, lib.arl2_oracle_teacher_rows):
                 f.restype = I
             _lib = lib
     return _lib
@@ -177,6 +182,61 @@ def phi(x, w, l2norm: bool):
     if rc != 0:
         raise RuntimeError("arl2_oracle_phi failed")
     return out
+
+
+def _cache(cache_k, cache_v, B, H, d):
+    if cache_k is None:
+        return np.zeros((B, 0, H, d)), np.zeros((B, 0, H, d))
+    kc, vc = f64(cache_k), f64(cache_v)
+    if kc.shape != vc.shape or kc.shape[0] != B or kc.shape[2:] != (H, d):
+        raise ValueError(f"cache shape {kc.shape} / {vc.shape}")
+    return kc, vc
+
+
+def teacher_pass(q, k, v, cache_k=None, cache_v=None, scale=None):
+    """Softmax teacher layer with a KV cache, one pass of one frame:
+    O = softmax([Q Kc^T, Q K^T] scale) [Vc; V], the frame's queries attending
+    to the clean keys/values of every earlier frame (cache_k, cache_v
+    [B, Lc, H, d], frames in order; None for the first frame) and,
+    bidirectionally, to their own.  Returns out [B, L, H, d].  The caller
+    appends a clean pass's k, v to the cache (teacher_append)."""
+    q, k, v = f64(q), f64(k), f64(v)
+    B, H, d, L = _dims(q)
+    kc, vc = _cache(cache_k, cache_v, B, H, d)
+    Lc = int(kc.shape[1])
+    out = np.zeros_like(q)
+    sc = default_scale(d) if scale is None else float(scale)
+    rc = _load().arl2_oracle_teacher_pass(B, H, d, L, Lc, sc, _p(q), _p(k), _p(v), _p(kc), _p(vc),
+                                          _p(out))
+    if rc != 0:
+        raise RuntimeError("arl2_oracle_teacher_pass failed")
+    return out
+
+
+def teacher_rows(q, k, v, cache_k, cache_v, rows_b, rows_t, scale=None):
+    """teacher_pass for selected token rows only: returns [nrows, H, d]."""
+    q, k, v = f64(q), f64(k), f64(v)
+    B, H, d, L = _dims(q)
+    kc, vc = _cache(cache_k, cache_v, B, H, d)
+    Lc = int(kc.shape[1])
+    rb = np.ascontiguousarray(np.asarray(rows_b, dtype=np.int32))
+    rt = np.ascontiguousarray(np.asarray(rows_t, dtype=np.int32))
+    n = int(rb.shape[0])
+    out = np.zeros((n, H, d))
+    sc = default_scale(d) if scale is None else float(scale)
+    rc = _load().arl2_oracle_teacher_rows(B, H, d, L, Lc, sc, _p(q), _p(k), _p(v), _p(kc), _p(vc),
+                                          n, _p(rb), _p(rt), _p(out))
+    if rc != 0:
+        raise RuntimeError("arl2_oracle_teacher_rows failed")
+    return out
+
+
+def teacher_append(cache_k, cache_v, k, v):
+    """The cache after a clean pass: (cache_k; k), (cache_v; v) along tokens."""
+    k, v = f64(k), f64(v)
+    if cache_k is None:
+        return k.copy(), v.copy()
+    return np.concatenate([f64(cache_k), k], axis=1), np.concatenate([f64(cache_v), v], axis=1)
 
 
 def zero_state(B: int, H: int, d: int) -> np.ndarray:

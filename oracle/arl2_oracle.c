@@ -331,3 +331,99 @@ int arl2_oracle_pass_token_level(int B, int H, int d, int L, double scale, const
                 err |= 1;
     return err ? -1 : 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Softmax teacher layer with a KV cache: the attention the hybrid layer
+ * replaces, kept by the layers of the stack that stay softmax (technical
+ * summary section 1 "KV Cache Growth"; section 4 "Efficiency", where the
+ * speedup grows with video length as the cache comes to dominate).  The
+ * pages fix the cache's role, not its arithmetic; the reading taken here is
+ * chunk-causal attention at frame granularity:
+ *   O = softmax([Q Kc^T, Q K^T] * scale) [Vc; V]
+ * for the L query rows of frame N, where (Kc, Vc) hold, in frame order, the
+ * keys and values of the clean passes of frames 0..N-1 (the same passes
+ * that update the hybrid layer's state, section 2.2 "Clean-Pass Updates"),
+ * and (K, V) are the current pass's own, attended bidirectionally.  A clean
+ * pass then appends its K and V to the cache; the caller does that by
+ * concatenation, nothing here keeps state.
+ *
+ * kc, vc: [B][Lc][H][d] (Lc = N L; Lc = 0 for the first frame, when kc and
+ * vc may be NULL).  q, k, v, out: [B][L][H][d]. */
+
+/* One query row: cached keys j < Lc first, then the frame's own keys. */
+static void teacher_row(int H, int d, int L, int Lc, int b, int h, int i, double scale,
+                        const double* q, const double* k, const double* v, const double* kc,
+                        const double* vc, double* s /* [Lc + L] */, double* o /* [d] */) {
+    const double* qi = q + IDX4(b, i, h, 0, L, H, d);
+    const int n = Lc + L;
+    double m = -INFINITY;
+    for (int j = 0; j < n; ++j) {
+        const double* kj = j < Lc ? kc + IDX4(b, j, h, 0, Lc, H, d)
+                                  : k + IDX4(b, j - Lc, h, 0, L, H, d);
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) dot += qi[c] * kj[c];
+        s[j] = dot * scale;
+        if (s[j] > m) m = s[j];
+    }
+    double l = 0.0;
+    for (int j = 0; j < n; ++j) {
+        s[j] = exp(s[j] - m);
+        l += s[j];
+    }
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    for (int j = 0; j < n; ++j) {
+        const double* vj = j < Lc ? vc + IDX4(b, j, h, 0, Lc, H, d)
+                                  : v + IDX4(b, j - Lc, h, 0, L, H, d);
+        for (int c = 0; c < d; ++c) o[c] += s[j] * vj[c];
+    }
+    for (int c = 0; c < d; ++c) o[c] = o[c] / l;
+}
+
+static int teacher_args_bad(int B, int H, int d, int L, int Lc, const double* q, const double* k,
+                            const double* v, const double* kc, const double* vc) {
+    if (bad_dims(B, H, d, L) || Lc < 0 || !q || !k || !v) return 1;
+    return Lc > 0 && (!kc || !vc);
+}
+
+/* Every row of the frame. */
+int arl2_oracle_teacher_pass(int B, int H, int d, int L, int Lc, double scale, const double* q,
+                             const double* k, const double* v, const double* kc, const double* vc,
+                             double* out) {
+    if (teacher_args_bad(B, H, d, L, Lc, q, k, v, kc, vc) || !out) return -1;
+    int err = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : err)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            double* s = (double*)malloc(sizeof(double) * ((size_t)Lc + L));
+            if (!s) { err |= 1; continue; }
+            for (int i = 0; i < L; ++i)
+                teacher_row(H, d, L, Lc, b, h, i, scale, q, k, v, kc, vc, s,
+                            out + IDX4(b, i, h, 0, L, H, d));
+            free(s);
+        }
+    }
+    return err ? -1 : 0;
+}
+
+/* Selected rows only (row r: token rows_t[r] of stream rows_b[r]); out_rows
+ * is [nrows][H][d].  For long caches, where the whole frame is too slow. */
+int arl2_oracle_teacher_rows(int B, int H, int d, int L, int Lc, double scale, const double* q,
+                             const double* k, const double* v, const double* kc, const double* vc,
+                             int nrows, const int* rows_b, const int* rows_t, double* out_rows) {
+    if (teacher_args_bad(B, H, d, L, Lc, q, k, v, kc, vc) || nrows < 0 || !out_rows) return -1;
+    if (nrows > 0 && (!rows_b || !rows_t)) return -1;
+    for (int r = 0; r < nrows; ++r)
+        if (rows_b[r] < 0 || rows_b[r] >= B || rows_t[r] < 0 || rows_t[r] >= L) return -1;
+    int err = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : err)
+    for (int r = 0; r < nrows; ++r) {
+        for (int h = 0; h < H; ++h) {
+            double* s = (double*)malloc(sizeof(double) * ((size_t)Lc + L));
+            if (!s) { err |= 1; continue; }
+            teacher_row(H, d, L, Lc, rows_b[r], h, rows_t[r], scale, q, k, v, kc, vc, s,
+                        out_rows + ((size_t)r * H + h) * d);
+            free(s);
+        }
+    }
+    return err ? -1 : 0;
+}

@@ -54,6 +54,16 @@ MUTATIONS = {
         "for (int c = 0; c < d; ++c) acc += kp[(size_t)i * d + c] * St[(size_t)c * d + n];",
         "for (int c = 0; c < d; ++c) acc += kp[(size_t)i * d + c] * S[(size_t)c * d + n];"),
     "token_level_gate_every_token": ("if (i == 0) g = alpha_per_key", "if (1) g = alpha_per_key"),
+    "teacher_scale_dropped": ("s[j] = dot * scale;", "s[j] = dot;"),
+    "teacher_cached_values_from_keys": ("const double* vj = j < Lc ? vc + IDX4(b, j, h, 0, Lc, H, d)",
+                                        "const double* vj = j < Lc ? kc + IDX4(b, j, h, 0, Lc, H, d)"),
+    "teacher_cache_stride_of_a_frame": ("const double* kj = j < Lc ? kc + IDX4(b, j, h, 0, Lc, H, d)",
+                                        "const double* kj = j < Lc ? kc + IDX4(b, j, h, 0, L, H, d)"),
+    "teacher_frame_key_head_dropped": (": k + IDX4(b, j - Lc, h, 0, L, H, d);",
+                                       ": k + IDX4(b, j - Lc, 0, 0, L, H, d);"),
+    "teacher_normaliser_without_cache": (
+        "for (int j = 0; j < n; ++j) {\n        s[j] = exp(s[j] - m);\n        l += s[j];",
+        "for (int j = 0; j < n; ++j) {\n        s[j] = exp(s[j] - m);\n        l += j < Lc ? 0.0 : s[j];"),
 }
 
 

@@ -9,7 +9,8 @@ streams and heads, scale invariance of the k' normalisation).
 
 Method text: "Attend Locally, Remember Linearly", technical summary
 section 2.1 (branches, phi maps, state update, read) and section 2.2
-(frame-level access, clean-pass updates).
+(frame-level access, clean-pass updates); the softmax teacher layer with a
+KV cache from section 1 (KV Cache Growth) and section 4 (Efficiency).
 """
 import json
 import math
@@ -82,6 +83,11 @@ def test_hand_worked_case(case):
     q = as_blhd(case.get("q", zeros))
     k = as_blhd(case["k"])
     v = as_blhd(case["v"])
+    if case.get("layer") == "teacher":
+        out = oracle.teacher_pass(q, k, v, as_blhd(case["cache_k"]), as_blhd(case["cache_v"]),
+                                  scale=case.get("scale"))
+        np.testing.assert_allclose(out[0, :, 0, :], case["expected_out"], rtol=0, atol=1e-12)
+        return
     wq = w_from(case.get("w_q", "identity"), d)
     wk = w_from(case.get("w_k", "identity"), d)
     wv = w_from(case.get("w_v", "identity"), d)
@@ -479,3 +485,114 @@ def test_token_level_gate_acts_once_per_frame():
     o_g, _ = _fl(x, S=x["alpha"][:, :, None, None] * x["S"], **kw)
     np.testing.assert_allclose(o_t[:, 0], o_f[:, 0], rtol=0, atol=1e-12)
     np.testing.assert_allclose(o_t[:, 1:], o_g[:, 1:], rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Softmax teacher layer with a KV cache (technical summary section 1 "KV
+# Cache Growth", section 4 "Efficiency"): frame N attends to the clean keys
+# and values of frames 0..N-1 and, bidirectionally, to its own
+# --------------------------------------------------------------------------
+
+def _teacher_inputs(seed, B=2, H=3, d=8, L=5, frames=3):
+    rng = np.random.default_rng(seed)
+    q, k, v = (rnd(rng, B, L, H, d) for _ in range(3))
+    kc, vc = (rnd(rng, B, frames * L, H, d) for _ in range(2))
+    return q, k, v, kc, vc
+
+
+def _sdpa(q, k, v, scale=None):
+    """torch's scaled_dot_product_attention in float64, [B, L, H, d] layout."""
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).permute(0, 2, 1, 3)
+    o = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), scale=scale)
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+@pytest.mark.parametrize("frames", [0, 1, 3])
+def test_teacher_equals_library_sdpa_over_cache_then_frame(frames):
+    q, k, v, kc, vc = _teacher_inputs(21 + frames, frames=frames)
+    out = oracle.teacher_pass(q, k, v, kc if frames else None, vc if frames else None)
+    ref = _sdpa(q, np.concatenate([kc, k], axis=1), np.concatenate([vc, v], axis=1))
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_teacher_scale_is_used():
+    q, k, v, kc, vc = _teacher_inputs(30, frames=2)
+    out = oracle.teacher_pass(q, k, v, kc, vc, scale=0.9)
+    ref = _sdpa(q, np.concatenate([kc, k], axis=1), np.concatenate([vc, v], axis=1), scale=0.9)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_teacher_with_empty_cache_is_the_hybrid_intra_branch():
+    # the first frame has no cache: the teacher is then the hybrid layer's
+    # intra-frame softmax (with a zero state the inter read adds nothing)
+    q, k, v, _, _ = _teacher_inputs(31)
+    B, L, H, d = q.shape
+    eye = eye_w(H, d)
+    hybrid, _ = oracle.frame_pass(q, k, v, eye, eye, eye, None, None, oracle.zero_state(B, H, d), False)
+    np.testing.assert_allclose(oracle.teacher_pass(q, k, v), hybrid, rtol=0, atol=1e-13)
+
+
+def test_teacher_frame_duplicated_in_cache_changes_nothing():
+    # each key appearing twice doubles numerator and denominator alike
+    q, k, v, _, _ = _teacher_inputs(32)
+    alone = oracle.teacher_pass(q, k, v)
+    np.testing.assert_allclose(oracle.teacher_pass(q, k, v, k, v), alone, rtol=0, atol=1e-12)
+    kk, vv = np.concatenate([k, k], axis=1), np.concatenate([v, v], axis=1)
+    np.testing.assert_allclose(oracle.teacher_pass(q, k, v, kk, vv), alone, rtol=0, atol=1e-12)
+
+
+def test_teacher_cache_token_order_is_irrelevant():
+    q, k, v, kc, vc = _teacher_inputs(33, frames=4)
+    perm = np.random.default_rng(3).permutation(kc.shape[1])
+    a = oracle.teacher_pass(q, k, v, kc, vc)
+    b = oracle.teacher_pass(q, k, v, kc[:, perm], vc[:, perm])
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_teacher_dominant_cached_key_selects_its_value():
+    # one cached key aligned with every query at a large scale takes all the weight
+    q, k, v, kc, vc = _teacher_inputs(34, B=1, H=1, d=4, L=3, frames=2)
+    q = np.abs(q) + 0.5
+    kc[0, 4, 0] = 60.0 * np.ones(4)
+    out = oracle.teacher_pass(q, k, v, kc, vc)
+    for i in range(3):
+        np.testing.assert_allclose(out[0, i, 0], vc[0, 4, 0], rtol=0, atol=1e-9)
+
+
+def test_teacher_streams_and_heads_read_their_own_cache():
+    q, k, v, kc, vc = _teacher_inputs(35, frames=2)
+    base = oracle.teacher_pass(q, k, v, kc, vc)
+    kc2, vc2 = kc.copy(), vc.copy()
+    kc2[1] += 1.0
+    vc2[1] -= 2.0
+    kc2[:, :, 2] *= 3.0
+    out = oracle.teacher_pass(q, k, v, kc2, vc2)
+    np.testing.assert_array_equal(out[0, :, :2], base[0, :, :2])  # stream 0, heads 0-1 untouched
+    assert np.abs(out[1] - base[1]).max() > 1e-3
+    assert np.abs(out[0, :, 2] - base[0, :, 2]).max() > 1e-3
+
+
+def test_teacher_rows_match_the_full_pass():
+    q, k, v, kc, vc = _teacher_inputs(36, frames=2)
+    full = oracle.teacher_pass(q, k, v, kc, vc)
+    rb, rt = [1, 0, 1, 0], [4, 0, 2, 3]
+    np.testing.assert_array_equal(oracle.teacher_rows(q, k, v, kc, vc, rb, rt), full[rb, rt])
+
+
+def test_teacher_append_is_concatenation_in_frame_order():
+    q, k, v, kc, vc = _teacher_inputs(37, frames=1)
+    k2, v2 = oracle.teacher_append(kc, vc, k, v)
+    np.testing.assert_array_equal(k2[:, :kc.shape[1]], kc)
+    np.testing.assert_array_equal(v2[:, kc.shape[1]:], v)
+    k0, v0 = oracle.teacher_append(None, None, k, v)
+    np.testing.assert_array_equal(k0, k)
+
+
+def test_teacher_rejects_bad_arguments():
+    q, k, v, kc, vc = _teacher_inputs(38, frames=1)
+    with pytest.raises(ValueError):
+        oracle.teacher_pass(q, k, v, kc[:, :, :2], vc[:, :, :2])
+    with pytest.raises(ValueError):
+        oracle.teacher_pass(q, k, v, kc, vc[:, :3])
+    with pytest.raises(RuntimeError):
+        oracle.teacher_rows(q, k, v, kc, vc, [2], [0])
