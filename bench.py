@@ -92,15 +92,19 @@ def load_peaks() -> dict:
 
 # ---------------------------------------------------------------- clocks --
 class ClockSampler:
-    """nvidia-smi clock and throttle-reason samples during the timed region."""
+    """nvidia-smi clock and throttle-reason samples (every 50 ms) around the
+    timed region; mark(start, stop) keeps the samples taken inside it (or,
+    for a region shorter than the sampling interval, the nearest ones)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 50
 
     def __init__(self, device: int):
         self.proc = None
         self.path = None
+        self.region = None
         try:
             uuid = str(torch.cuda.get_device_properties(device).uuid)
             ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
@@ -108,13 +112,32 @@ class ClockSampler:
             self.path = os.path.join(out_dir, f"clocks_{os.getpid()}.csv")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", ident, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", str(self.INTERVAL_MS)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            # the timed region starts once the sampler is producing samples
+            t_end = time.time() + 10.0
+            while time.time() < t_end and self.proc.poll() is None:
+                if os.path.getsize(self.path) > 0:
+                    break
+                time.sleep(0.01)
         except Exception:
             self.proc = None
+
+    def mark(self, t0: float, t1: float) -> None:
+        """Host wall-clock bounds of the timed region (time.time())."""
+        self.region = (t0, t1)
+
+    @staticmethod
+    def _when(stamp: str):
+        import datetime
+        try:
+            return datetime.datetime.strptime(stamp.strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
 
     def stop(self) -> dict | None:
         if self.proc is None:
             return None
+        time.sleep(2.0 * self.INTERVAL_MS / 1000.0)  # one sample after the region
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -124,25 +147,33 @@ class ClockSampler:
             rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
         except Exception:
             return None
-        sm, mx, reasons = [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        parsed = []
         for r in rows:
             r = [x.strip() for x in r]
-            if len(r) < 9:
+            if len(r) < 10:
                 continue
             try:
-                sm.append(float(r[1]))
-                mx = max(mx, float(r[2]))
+                parsed.append((self._when(r[0]), float(r[2]), float(r[3]),
+                               {n for n, v in zip(names, r[6:10]) if v.lower() in ("active", "0x1") or v == "1"}))
             except ValueError:
                 continue
-            for n, v in zip(names, r[5:9]):
-                if v.lower() in ("active", "0x1") or v == "1":
-                    reasons.add(n)
-        if not sm:
+        if not parsed:
             return None
-        loaded = [s for s in sm if s > 0.5 * mx] or sm
+        inside = parsed
+        if self.region is not None and all(p[0] is not None for p in parsed):
+            t0, t1 = self.region
+            inside = [p for p in parsed if t0 <= p[0] <= t1]
+            if not inside:  # region shorter than the interval: the samples around it
+                before = [p for p in parsed if p[0] < t0]
+                after = [p for p in parsed if p[0] > t1]
+                inside = before[-1:] + after[:1]
+        sm = [p[1] for p in inside]
+        mx = max(p[2] for p in parsed)
+        reasons = set().union(*(p[3] for p in inside))
+        loaded = [v for v in sm if v > 0.5 * mx] or sm
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(inside)}
 
 
 # ------------------------------------------------------------ distributed --
@@ -285,6 +316,127 @@ def profile_case(args, w: workloads.Workload) -> int:
     return 0 if st == 0 else 1
 
 
+def teacher_flops(w: workloads.Workload, cached_frames: int) -> float:
+    """Algorithmic FLOPs of one teacher-layer pass with `cached_frames`
+    frames in the KV cache: 4 L (N L + L) d H per stream."""
+    L, d, H, B = w.tokens, w.head_dim, w.heads, w.batch
+    return 4.0 * L * (cached_frames + 1) * L * d * H * B
+
+
+def stack_curve(args, w: workloads.Workload) -> int:
+    """Softmax teacher layer (KV cache) against the hybrid layer over one long
+    stream: per-frame attention time and memory as the video grows, and the
+    30-layer stacks with 0, 50, 75 and 100 % of the layers replaced
+    (technical summary section 4 "Efficiency": the speedup and the memory
+    saving grow with video length as the KV cache comes to dominate).
+
+    Each layer kind runs the whole stream of `--curve-frames` frames once
+    untimed, then once timed with an event pair around every frame (all of
+    its passes, the clean pass's cache append or state update included); each
+    frame is one CUDA graph.  Inputs cycle through a ring of pass inputs
+    larger than L2.  A stack's attention time is the sum over its layers
+    (the layers are independent work of identical cost per kind); its memory
+    is the sum of the teacher layers' KV caches and the hybrid layers' state
+    copies and workspaces.  Attention only: the pages' figures are whole-model.
+    """
+    from hybrid_softmax_gated_b200 import Arl2Layer, TeacherLayer
+    F = args.curve_frames
+    B, L, H, d = w.batch, w.tokens, w.heads, w.head_dim
+    esz = 2 if w.dtype == "bf16" else 4
+    per_set = 3 * B * L * H * d * esz
+    ring = max(2, (160 << 20) // per_set + 1)
+    ins = [workloads.pass_inputs(w, 0, 0, i, device="cuda") for i in range(ring)]
+    a, b = (t.cuda() for t in workloads.frame_gates(w, 0, 0))
+    out = torch.empty_like(ins[0][0])
+    st = torch.cuda.current_stream()
+    cap_stream = torch.cuda.Stream()
+    wq, wk, wv = workloads.phi_weights(w, 0)
+    hyb = Arl2Layer(B, H, d, L, wq.cuda(), wk.cuda(), wv.cuda(), dtype=w.torch_dtype)
+    tea = TeacherLayer(B, H, d, L, F, dtype=w.torch_dtype)
+
+    def frame_call(kind, f):
+        for p in range(w.passes):
+            q, k, v = ins[(f * w.passes + p) % ring]
+            clean = workloads.is_clean(w, p)
+            if kind == "teacher":
+                tea.forward(q, k, v, clean_pass=clean, out=out)
+            else:
+                hyb.forward(q, k, v, a, b, clean_pass=clean, out=out)
+
+    def run(kind):
+        graphs = []
+        for f in range(F):  # the teacher's graphs keep the cache length each frame saw
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap_stream):
+                frame_call(kind, f)
+            graphs.append(g)
+        for g in graphs:  # upload and warm up: the whole stream once, untimed
+            g.replay()
+        torch.cuda.synchronize()
+        if kind == "hybrid":
+            hyb.state_reset()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(F + 1)]
+        evs[0].record(st)
+        for f, g in enumerate(graphs):
+            g.replay()
+            evs[f + 1].record(st)
+        torch.cuda.synchronize()
+        ms = [evs[f].elapsed_time(evs[f + 1]) for f in range(F)]
+        del graphs
+        return ms
+
+    t_tea = run("teacher")
+    t_hyb = run("hybrid")
+    bad = (tea.device_status(), hyb.device_status())
+    if bad != (0, 0):
+        raise SystemExit(f"device status {bad}")
+    frame_b = B * L * H * d * esz
+    hyb_bytes = hyb.device_bytes()
+    marks = sorted({m for m in (1, 21, 81, 231, F) if m <= F})
+    peaks = load_peaks()
+    n_layers = 30
+    curve = []
+    for m in marks:
+        T_t, T_h = sum(t_tea[:m]), sum(t_hyb[:m])
+        cache = 2 * m * frame_b
+        row = {"frames": m, "video_frames": 4 * (m - 1) + 1,
+               "teacher_ms_frame": t_tea[m - 1], "hybrid_ms_frame": t_hyb[m - 1],
+               "teacher_ms_video": T_t, "hybrid_ms_video": T_h,
+               "teacher_cache_bytes": cache, "hybrid_state_bytes": hyb_bytes,
+               "teacher_tflops_last_frame": w.passes * teacher_flops(w, m - 1) / (t_tea[m - 1] * 1e-3) / 1e12}
+        stacks = {}
+        for r in (0.0, 0.5, 0.75, 1.0):
+            n_h = int(round(n_layers * r))
+            n_t = n_layers - n_h
+            t = n_t * T_t + n_h * T_h
+            mem = n_t * cache + n_h * hyb_bytes
+            stacks[f"{int(r * 100)}%"] = {"attn_ms_video": t, "attn_bytes": mem}
+        base = stacks["0%"]
+        for v in stacks.values():
+            v["speedup_vs_all_softmax"] = base["attn_ms_video"] / v["attn_ms_video"]
+            v["memory_vs_all_softmax"] = v["attn_bytes"] / base["attn_bytes"]
+        row["stack30"] = stacks
+        curve.append(row)
+    last = curve[-1]
+    line = {
+        "metric": "attention per video: softmax KV-cache teacher vs ARL2 hybrid layer (480p, 30-layer stacks)",
+        "unit": "ms", "data": "synthetic", "dtype": w.dtype, "n_gpus": 1,
+        "config": {"workload": w.name, "batch": B, "heads": H, "head_dim": d, "tokens_per_frame": L,
+                   "passes": w.passes, "frames": F, "layers": n_layers,
+                   "l2": f"inputs larger than L2 ({ring} input sets)"},
+        "curve": curve,
+        "roofline": {"kernel": "attn_tc_kernel (teacher, longest cache)", "bound": "tensor",
+                     "achieved": last["teacher_tflops_last_frame"], "peak": peaks["bf16_tflops_sustained"],
+                     "unit": "TFLOP/s", "frac": last["teacher_tflops_last_frame"] / peaks["bf16_tflops_sustained"],
+                     "note": "whole frame (4 passes and the append) timed; peak: bf16 sustained "
+                             f"({peaks['source']})"},
+    }
+    tea.close()
+    hyb.close()
+    print(json.dumps(line))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -298,6 +450,11 @@ def main():
     ap.add_argument("--access", default="frame", choices=["frame", "token"],
                     help="frame-level state access (the method) or token-level (the ablation)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stack-curve", action="store_true",
+                    help="softmax KV-cache teacher vs hybrid layer over one long stream, and the "
+                         "30-layer stacks built from them (one JSON line, not the headline)")
+    ap.add_argument("--curve-frames", type=int, default=231,
+                    help="latent frames of the stack-curve stream (231: 921 video frames)")
     ap.add_argument("--profile-passes", type=int, default=0,
                     help="profiling case: run this many read-only passes over a ring of inputs "
                          "larger than L2 and exit (no timing, no JSON line)")
@@ -312,6 +469,8 @@ def main():
     torch.cuda.set_device(local)
     if args.profile_passes > 0:
         return profile_case(args, w)
+    if args.stack_curve:
+        return stack_curve(args, w)
     if ws > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
@@ -386,13 +545,16 @@ def main():
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(ws)
     torch.cuda.synchronize()
+    t_wall0 = time.time()
     start.record(st)
     for g in graphs:
         g.replay()
     stop.record(st)
     torch.cuda.synchronize()
+    t_wall1 = time.time()
     barrier(ws)
     elapsed_ms = start.elapsed_time(stop)
+    clocks.mark(t_wall0, t_wall1)
     clk = clocks.stop()
     status = lay.device_status()
     if status != 0:

@@ -12,6 +12,10 @@ The layer ("Attend Locally, Remember Linearly", technical summary §2.1 and
     clean pass only, after the read:
     S_N = alpha S_{N-1} + K'^T diag(beta) (V' - K' S_{N-1}),
     K' = rownorm(K W_k[h]), V' = V W_v[h]
+
+and the softmax teacher layer it replaces (TeacherLayer, technical summary
+§1 "KV Cache Growth"): frame N attends to the clean keys/values of frames
+0..N-1, kept in a KV cache, and bidirectionally to its own.
 """
 from __future__ import annotations
 
@@ -35,6 +39,9 @@ EXPORTED = (
     "arl2_state_get", "arl2_state_set", "arl2_phi_apply", "arl2_device_status",
     "arl2_device_bytes", "arl2_kernel_launches", "arl2_state_update_noalloc", "arl2_destroy",
     "arl2_status_string", "arl2_version",
+    "arl2_kv_create", "arl2_kv_frame_forward", "arl2_kv_frame_forward_host", "arl2_kv_reset",
+    "arl2_kv_frames", "arl2_kv_cache_get", "arl2_kv_device_status", "arl2_kv_device_bytes",
+    "arl2_kv_cache_bytes", "arl2_kv_kernel_launches", "arl2_kv_destroy",
 )
 NOALLOC_MAX_ELEMENTS = 1 << 22
 
@@ -46,6 +53,15 @@ class Arl2Config(ctypes.Structure):
         ("w_q", ctypes.c_void_p), ("w_k", ctypes.c_void_p), ("w_v", ctypes.c_void_p),
         ("softmax_scale", ctypes.c_float), ("host_staging", ctypes.c_int), ("impl", ctypes.c_int),
         ("max_ctas", ctypes.c_int), ("gating", ctypes.c_int), ("access", ctypes.c_int),
+    ]
+
+
+class Arl2KvConfig(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int), ("heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+        ("tokens_per_frame", ctypes.c_int), ("max_frames", ctypes.c_int), ("dtype", ctypes.c_int),
+        ("softmax_scale", ctypes.c_float), ("host_staging", ctypes.c_int), ("impl", ctypes.c_int),
+        ("max_ctas", ctypes.c_int),
     ]
 
 
@@ -71,6 +87,17 @@ def _load() -> ctypes.CDLL:
         "arl2_destroy": ([H], None),
         "arl2_status_string": ([I], ctypes.c_char_p),
         "arl2_version": ([], I),
+        "arl2_kv_create": ([ctypes.POINTER(Arl2KvConfig), P, ctypes.POINTER(H)], I),
+        "arl2_kv_frame_forward": ([H, P, P, P, I, P, P], I),
+        "arl2_kv_frame_forward_host": ([H, P, P, P, I, P, P], I),
+        "arl2_kv_reset": ([H], I),
+        "arl2_kv_frames": ([H], I),
+        "arl2_kv_cache_get": ([H, P, P, P], I),
+        "arl2_kv_device_status": ([H, P], I),
+        "arl2_kv_device_bytes": ([H], S),
+        "arl2_kv_cache_bytes": ([H], S),
+        "arl2_kv_kernel_launches": ([H], ctypes.c_ulonglong),
+        "arl2_kv_destroy": ([H], None),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -255,6 +282,110 @@ class Arl2Layer:
     def close(self) -> None:
         if getattr(self, "_h", None) is not None:
             _lib.arl2_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+
+class TeacherLayer:
+    """The softmax teacher layer with a KV cache (arl2_kv_* in the C ABI).
+
+    One pass of frame N: out = softmax([Q Kc^T, Q K^T] scale) [Vc; V], where
+    (Kc, Vc) are the clean keys/values of frames 0..N-1 (the cache) and
+    (K, V) the pass's own; a clean pass appends its k, v.  The cache holds up
+    to max_frames frames, allocated at creation.
+    """
+
+    def __init__(self, batch: int, heads: int, head_dim: int, tokens: int, max_frames: int, *,
+                 dtype: torch.dtype = torch.bfloat16, softmax_scale: float = 0.0,
+                 host_staging: bool = False, impl: str = "auto", max_ctas: int = 0,
+                 device=None, stream=None):
+        if dtype not in (torch.bfloat16, torch.float32):
+            raise ValueError("dtype must be torch.bfloat16 or torch.float32")
+        self.shape = (batch, tokens, heads, head_dim)
+        self.dtype = dtype
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        cfg = Arl2KvConfig(batch, heads, head_dim, tokens, max_frames,
+                           ARL2_BF16 if dtype == torch.bfloat16 else ARL2_FP32, float(softmax_scale),
+                           1 if host_staging else 0,
+                           {"auto": ARL2_IMPL_AUTO, "simt": ARL2_IMPL_SIMT}[impl], int(max_ctas))
+        h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            _check(_lib.arl2_kv_create(ctypes.byref(cfg), _stream(stream), ctypes.byref(h)), "arl2_kv_create")
+        self._h = h
+
+    def _tok(self, t, name):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == self.dtype):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor of the layer dtype")
+        if tuple(t.shape) != self.shape:
+            raise ValueError(f"{name} must have shape {self.shape}")
+        return t
+
+    @property
+    def handle(self):
+        if self._h is None:
+            raise RuntimeError("layer is closed")
+        return self._h
+
+    def forward(self, q, k, v, clean_pass: bool = False, out=None, stream=None):
+        """One pass of the current frame; returns out [B, L, H, d]."""
+        self._tok(q, "q"), self._tok(k, "k"), self._tok(v, "v")
+        if out is None:
+            out = torch.empty_like(q)
+        self._tok(out, "out")
+        _check(_lib.arl2_kv_frame_forward(self.handle, _ptr(q), _ptr(k), _ptr(v), 1 if clean_pass else 0,
+                                          _ptr(out), _stream(stream)), "arl2_kv_frame_forward")
+        return out
+
+    def forward_host(self, q, k, v, clean_pass: bool, out, stream=None):
+        """arl2_kv_frame_forward_host: q, k, v, out are host (pinned) tensors."""
+        for t in (q, k, v, out):
+            if t.is_cuda or not t.is_contiguous() or tuple(t.shape) != self.shape or t.dtype != self.dtype:
+                raise ValueError("host token tensors must be contiguous CPU tensors of the layer shape")
+        _check(_lib.arl2_kv_frame_forward_host(self.handle, _ptr(q), _ptr(k), _ptr(v), 1 if clean_pass else 0,
+                                               _ptr(out), _stream(stream)), "arl2_kv_frame_forward_host")
+        return out
+
+    def reset(self) -> None:
+        _check(_lib.arl2_kv_reset(self.handle), "arl2_kv_reset")
+
+    def frames(self) -> int:
+        return int(_lib.arl2_kv_frames(self.handle))
+
+    def cache_get(self, stream=None):
+        """(k, v) in the cache: [B, frames * L, H, d] each."""
+        B, L, H, d = self.shape
+        n = self.frames() * L
+        kc = torch.empty(B, n, H, d, dtype=self.dtype, device=self.device)
+        vc = torch.empty_like(kc)
+        _check(_lib.arl2_kv_cache_get(self.handle, _ptr(kc), _ptr(vc), _stream(stream)), "arl2_kv_cache_get")
+        return kc, vc
+
+    def device_status(self, stream=None) -> int:
+        return _lib.arl2_kv_device_status(self.handle, _stream(stream))
+
+    def device_bytes(self) -> int:
+        return int(_lib.arl2_kv_device_bytes(self.handle))
+
+    def cache_bytes(self) -> int:
+        return int(_lib.arl2_kv_cache_bytes(self.handle))
+
+    def kernel_launches(self) -> int:
+        return int(_lib.arl2_kv_kernel_launches(self.handle))
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None:
+            _lib.arl2_kv_destroy(self._h)
             self._h = None
 
     def __del__(self):

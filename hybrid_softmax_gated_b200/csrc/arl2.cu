@@ -147,7 +147,7 @@ arl2_status clean_update(arl2_handle* h, const void* k, const void* v, const flo
 
 extern "C" {
 
-int arl2_version(void) { return 10100; }
+int arl2_version(void) { return 10200; }
 
 const char* arl2_status_string(arl2_status s) {
     switch (s) {

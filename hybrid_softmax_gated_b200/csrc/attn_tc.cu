@@ -105,6 +105,7 @@ struct Seg {
 // Unit schedule shared by every role of every CTA.
 struct Sched {
     int n_q, n_kv, T;  // tiles per (stream, head), key blocks, tiles in total
+    int n_c;           // leading key blocks read from the KV cache (0: none)
     int G;             // CTAs
     int split;         // 1: persistent unit ranges, 0: one tile per CTA
     long long U;       // units
@@ -182,16 +183,36 @@ __device__ __forceinline__ int valid_keys(int L, int kv) {
     return v < kBN ? v : kBN;
 }
 
+// Keys of block kv: the first nc blocks cover the Lc cached keys, the rest
+// the frame's own L keys; each run ends in its own ragged block.
+__device__ __forceinline__ int block_keys(int nc, int L, int Lc, int kv) {
+    return kv < nc ? valid_keys(Lc, kv) : valid_keys(L, kv - nc);
+}
+
+// K-ring items of a segment: its key blocks, then (with the inter-frame
+// read, for a segment that finishes its tile) the (W_q S)^T tile.
+template <bool kInter>
+__device__ __forceinline__ int seg_items(const Seg& sg) {
+    return sg.kv1 - sg.kv0 + (kInter && sg.kind != kHead ? 1 : 0);
+}
+
+// kInter: add the inter-frame read Q (W_q S) (the hybrid layer); without
+// it, plain softmax attention whose first Lc keys come from a KV cache
+// (tm_kc, tm_vc) and the rest from the frame (tm_k, tm_v).
+template <bool kInter>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_m,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
+                   const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_m,
                    const __grid_constant__ CUtensorMap tm_o, float* __restrict__ part_o,
-                   float* __restrict__ part_ml, int* __restrict__ flags, int L, int H, Sched sch,
+                   float* __restrict__ part_ml, int* __restrict__ flags, int L, int Lc, int H, Sched sch,
                    float scale_log2, int* err) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                         ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // key blocks from the KV cache (the hybrid layer has none: a constant 0)
+    const int nc = kInter ? 0 : sch.n_c;
     volatile int* abort = &sm.abort;
     const int no_abort = 0;
     const CtaRange rng = cta_range(sch, blockIdx.x);
@@ -249,7 +270,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tma_prefetch_desc(&tm_q);
         ptx::tma_prefetch_desc(&tm_k);
         ptx::tma_prefetch_desc(&tm_v);
-        ptx::tma_prefetch_desc(&tm_m);
+        if (nc > 0) {
+            ptx::tma_prefetch_desc(&tm_kc);
+            ptx::tma_prefetch_desc(&tm_vc);
+        }
+        if (kInter) ptx::tma_prefetch_desc(&tm_m);
         int kc = 0, vc = 0;  // ring counters (same sequence as the UMMA issuer)
         // A K slot is free again once its previous item is consumed: a key
         // block is released by the softmax warpgroup that saw its S (k_empty,
@@ -279,8 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t bar = ptx::smem_u32(&sm.k_full[s]), dst = ptx::smem_u32(sm.k[s]);
             ptx::mbar_arrive_expect_tx_w(bar, kTileBytes);
             if (kv >= 0) {
-                ptx::tma_load_4d_w(dst, &tm_k, 0, h, kv * kBN, b, bar);
-                ptx::tma_load_4d_w(dst + kHalfBytes, &tm_k, 64, h, kv * kBN, b, bar);
+                const CUtensorMap* tm = kv < nc ? &tm_kc : &tm_k;
+                const int row = (kv < nc ? kv : kv - nc) * kBN;
+                ptx::tma_load_4d_w(dst, tm, 0, h, row, b, bar);
+                ptx::tma_load_4d_w(dst + kHalfBytes, tm, 64, h, row, b, bar);
             } else {
                 ptx::tma_load_4d_w(dst, &tm_m, 0, 0, b * H + h, 0, bar);
                 ptx::tma_load_4d_w(dst + kHalfBytes, &tm_m, 64, 0, b * H + h, 0, bar);
@@ -293,8 +320,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (vc >= 2 && !wwait(&sm.v_empty[s], ((vc >> 1) - 1) & 1)) return false;
             const uint32_t bar = ptx::smem_u32(&sm.v_full[s]), dst = ptx::smem_u32(sm.v[s]);
             ptx::mbar_arrive_expect_tx_w(bar, kTileBytes);
-            ptx::tma_load_4d_w(dst, &tm_v, 0, h, kv * kBN, b, bar);
-            ptx::tma_load_4d_w(dst + kHalfBytes, &tm_v, 64, h, kv * kBN, b, bar);
+            const CUtensorMap* tm = kv < nc ? &tm_vc : &tm_v;
+            const int row = (kv < nc ? kv : kv - nc) * kBN;
+            ptx::tma_load_4d_w(dst, tm, 0, h, row, b, bar);
+            ptx::tma_load_4d_w(dst + kHalfBytes, tm, 64, h, row, b, bar);
             ++vc;
             return true;
         };
@@ -317,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // segment is a head piece) the (W_q S)^T tile; the issuer takes
             // items 0 and 1 first and item j + 2 after the P V of block j.
             const int n = sg.kv1 - sg.kv0;
-            const int nk = n + (sg.kind != kHead ? 1 : 0);
+            const int nk = seg_items<kInter>(sg);
             auto load_item = [&](int i) { return load_k(b, h, i < n ? sg.kv0 + i : -1); };
             for (int i = 0; ok && i < 2 && i < nk; ++i) ok = load_item(i);
             for (int j = 0; ok && j < n; ++j) {
@@ -349,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Seg sg = seg_at(sch, rng, si);
             const int qs = si & 1;
             const int n = sg.kv1 - sg.kv0;
-            const int nk = n + (sg.kind != kHead ? 1 : 0);
+            const int nk = seg_items<kInter>(sg);
             if (!wwait(&sm.q_full[qs], (si >> 1) & 1)) {
                 ok = false;
                 break;
@@ -374,12 +403,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t k_s = ptx::smem_u32(sm.k[s]);
                 const uint32_t d = tmem + kColS + (uint32_t)buf * kBN;
                 if (i < n) {
-                    const int valid = valid_keys(L, sg.kv0 + i);
+                    const int valid = block_keys(nc, L, Lc, sg.kv0 + i);
                     const uint32_t idesc = ptx::idesc_bf16_f32(kBM, (valid + 15) & ~15, false, false);
                     ptx::umma_ss8_kk(d, kmajor_desc(q_s, 0), kmajor_desc(k_s, 0), idesc, 0u);
                     ptx::umma_commit_w(ptx::smem_u32(&sm.s_full[buf]));
-                    // a head piece's last use of Q (once per CTA at most)
-                    if (sg.kind == kHead && i == n - 1) ptx::umma_commit_w(ptx::smem_u32(&sm.q_empty[qs]));
+                    // the last use of Q: a head piece's (once per CTA at most), or
+                    // every segment's without the inter-frame read
+                    if ((!kInter || sg.kind == kHead) && i == n - 1)
+                        ptx::umma_commit_w(ptx::smem_u32(&sm.q_empty[qs]));
                 } else {
                     // O_inter: the last use of Q and of the (W_q S)^T tile
                     ptx::umma_ss8_kk(d, kmajor_desc(q_s, 0), kmajor_desc(k_s, 0), idesc_qm, 0u);
@@ -397,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 p_par ^= 1u << buf;
                 if (!ok) break;
                 ptx::tc_fence_after();
-                const int ksteps = (valid_keys(L, sg.kv0 + j) + 15) >> 4;
+                const int ksteps = (block_keys(nc, L, Lc, sg.kv0 + j) + 15) >> 4;
                 const uint32_t p_t = tmem + kColS + (uint32_t)buf * kBN;
                 const uint32_t o_t = tmem + kColO + (uint32_t)buf * kD;
                 const uint32_t v_s = ptx::smem_u32(sm.v[vs]);
@@ -417,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (j + 2 < nk) ok = issue_item(j + 2);
             }
             if (!ok) break;
-            prev_oi_buf = sg.kind != kHead ? (vb + n) & 1 : -1;
+            prev_oi_buf = kInter && sg.kind != kHead ? (vb + n) & 1 : -1;
             vb += nk;
         }
         if (!ok) {
@@ -438,9 +469,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int b = bh / H, h = bh - b * H;
             for (int half = 0; half < 2; ++half) {
                 ptx::tma_prefetch_l2_4d(&tm_q, half * 64, h, qt * kBM, b);
-                ptx::tma_prefetch_l2_4d(&tm_v, half * 64, h, sg.kv0 * kBN, b);
-                for (int i = 0; i < 2 && sg.kv0 + i < sg.kv1; ++i)
-                    ptx::tma_prefetch_l2_4d(&tm_k, half * 64, h, (sg.kv0 + i) * kBN, b);
+                for (int i = 0; i < 2 && sg.kv0 + i < sg.kv1; ++i) {
+                    const int kv = sg.kv0 + i;
+                    const int row = (kv < nc ? kv : kv - nc) * kBN;
+                    ptx::tma_prefetch_l2_4d(kv < nc ? &tm_kc : &tm_k, half * 64, h, row, b);
+                    if (i == 0) ptx::tma_prefetch_l2_4d(kv < nc ? &tm_vc : &tm_v, half * 64, h, row, b);
+                }
             }
         }
         __syncwarp();
@@ -533,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float x[128];
 #pragma unroll
                 for (int i = 0; i < 128; ++i) x[i] = __uint_as_float(raw[i >> 5][i & 31]);
-                const int valid = valid_keys(L, sg.kv0 + j);
+                const int valid = block_keys(nc, L, Lc, sg.kv0 + j);
                 if (valid < kBN) {
 #pragma unroll
                     for (int i = 0; i < 128; ++i)
@@ -676,7 +710,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < 2; ++c) {
                     float acc[32];
                     uint32_t oi[32];
-                    load_acc(c, acc, std::true_type{}, oi_col, oi);
+                    load_acc(c, acc, std::bool_constant<kInter>{}, oi_col, oi);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) acc[i] *= a_t;
                     if (sg.kind == kTail) {
@@ -696,8 +730,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int i = gq * 8 + e * 2;
-                            w[e] = ptx::pack_bf16x2(fmaf(acc[i], inv_l, __uint_as_float(oi[i])),
-                                                    fmaf(acc[i + 1], inv_l, __uint_as_float(oi[i + 1])));
+                            const float i0 = kInter ? __uint_as_float(oi[i]) : 0.f;
+                            const float i1 = kInter ? __uint_as_float(oi[i + 1]) : 0.f;
+                            w[e] = ptx::pack_bf16x2(fmaf(acc[i], inv_l, i0), fmaf(acc[i + 1], inv_l, i1));
                         }
                         ptx::st_shared_v4(stage + ptx::tile_chunk_offset(row, wg * 8 + c * 4 + gq), w[0], w[1],
                                           w[2], w[3]);
@@ -709,8 +744,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ptx::tc_fence_before();
             warp_arrive(&sm.o_free);
-            vb += n + (sg.kind != kHead ? 1 : 0);
-            kc0 += n + (sg.kind != kHead ? 1 : 0);
+            vb += seg_items<kInter>(sg);
+            kc0 += seg_items<kInter>(sg);
             vc0 += n;
         }
         if (!ok) fail();
@@ -730,13 +765,70 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 struct AttnTc {
     Dims dm{};
+    int G = 0;  // CTAs the persistent grid may use
     const void* m_ptr = nullptr;
     CUtensorMap tm_m{};
-    Sched sch{};
+    Sched sch{};  // the schedule without cached keys
     float* part_o = nullptr;
     float* part_ml = nullptr;
     int* flags = nullptr;
 };
+
+namespace {
+
+// Tiles of 128 query rows against n_c + ceil(L / 128) key blocks.  The
+// split-tile workspace depends on the tiles only, so one workspace serves
+// every cache length.
+Sched make_sched(const Dims& dm, int Lc, int G) {
+    Sched s{};
+    s.n_q = (dm.L + kBM - 1) / kBM;
+    s.n_c = (Lc + kBN - 1) / kBN;
+    s.n_kv = s.n_c + (dm.L + kBN - 1) / kBN;
+    s.T = dm.B * dm.H * s.n_q;
+    s.U = (long long)s.T * s.n_kv;
+    s.split = s.T > G ? 1 : 0;
+    s.G = s.split ? G : s.T;
+    return s;
+}
+
+template <bool kInter>
+bool kernel_ready() {
+    if (cudaFuncSetAttribute(attn_tc_kernel<kInter>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    // the warpgroups' register split needs the launch count it was sized for
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, attn_tc_kernel<kInter>) != cudaSuccess || fa.numRegs != kRegsLaunch) {
+        cudaGetLastError();
+        return false;
+    }
+    return true;
+}
+
+template <bool kInter>
+cudaError_t launch(const AttnTc* t, const Sched& sch, const CUtensorMap& cq, const CUtensorMap& ck,
+                   const CUtensorMap& cv, const CUtensorMap& ckc, const CUtensorMap& cvc,
+                   const CUtensorMap& co, int Lc, float scale, int* err, cudaStream_t st) {
+    const float sl2 = scale * 1.4426950408889634f;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(sch.G, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    // Programmatic dependent launch: the CTAs start (set-up only) while the
+    // previous kernel drains.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, attn_tc_kernel<kInter>, cq, ck, cv, ckc, cvc, t->tm_m, co, t->part_o,
+                              t->part_ml, t->flags, t->dm.L, Lc, t->dm.H, sch, sl2, err);
+}
+
+}  // namespace
 
 size_t attn_tc_workspace_bytes(const Dims& dm) {
     const size_t tiles = (size_t)dm.B * dm.H * ((dm.L + kBM - 1) / kBM);
@@ -745,17 +837,7 @@ size_t attn_tc_workspace_bytes(const Dims& dm) {
 
 AttnTc* attn_tc_create(Dims dm, void* workspace, int max_ctas) {
     if (dm.d != kD || dm.L < 1 || dm.H < 1 || dm.B < 1 || !tma_available() || !workspace) return nullptr;
-    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes) != cudaSuccess) {
-        cudaGetLastError();
-        return nullptr;
-    }
-    // the warpgroups' register split needs the launch count it was sized for
-    cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, attn_tc_kernel) != cudaSuccess || fa.numRegs != kRegsLaunch) {
-        cudaGetLastError();
-        return nullptr;
-    }
+    if (!kernel_ready<true>() || !kernel_ready<false>()) return nullptr;
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
@@ -765,15 +847,9 @@ AttnTc* attn_tc_create(Dims dm, void* workspace, int max_ctas) {
     AttnTc* t = new (std::nothrow) AttnTc();
     if (!t) return nullptr;
     t->dm = dm;
-    Sched& s = t->sch;
-    s.n_q = (dm.L + kBM - 1) / kBM;
-    s.n_kv = (dm.L + kBN - 1) / kBN;
-    s.T = dm.B * dm.H * s.n_q;
-    s.U = (long long)s.T * s.n_kv;
-    const int G = max_ctas > 0 && max_ctas < sms ? max_ctas : sms;
-    s.split = s.T > G ? 1 : 0;
-    s.G = s.split ? G : s.T;
-    const size_t tiles = (size_t)s.T;
+    t->G = max_ctas > 0 && max_ctas < sms ? max_ctas : sms;
+    t->sch = make_sched(dm, 0, t->G);
+    const size_t tiles = (size_t)t->sch.T;
     char* w = static_cast<char*>(workspace);
     t->part_o = reinterpret_cast<float*>(w);
     t->part_ml = reinterpret_cast<float*>(w + tiles * kBM * kD * 4);
@@ -799,21 +875,18 @@ cudaError_t attn_tc_launch(AttnTc* t, TokenMapCache& maps, const void* q, const 
     CUtensorMap cq, ck, cv, co;
     if (!maps.get(q, &cq) || !maps.get(k, &ck) || !maps.get(v, &cv) || !maps.get(out, &co))
         return cudaErrorInvalidValue;
-    const float sl2 = scale * 1.4426950408889634f;
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(t->sch.G, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cfg.stream = st;
-    // Programmatic dependent launch: the CTAs start (set-up only) while the
-    // previous kernel drains.
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, attn_tc_kernel, cq, ck, cv, t->tm_m, co, t->part_o, t->part_ml,
-                              t->flags, dm.L, dm.H, t->sch, sl2, err);
+    return launch<true>(t, t->sch, cq, ck, cv, ck, cv, co, 0, scale, err, st);
+}
+
+cudaError_t attn_tc_launch_cached(AttnTc* t, TokenMapCache& maps, const void* q, const void* k,
+                                  const void* v, const CUtensorMap* kc, const CUtensorMap* vc, int Lc,
+                                  void* out, float scale, int* err, cudaStream_t st) {
+    if (Lc < 0 || (Lc > 0 && (!kc || !vc))) return cudaErrorInvalidValue;
+    CUtensorMap cq, ck, cv, co;
+    if (!maps.get(q, &cq) || !maps.get(k, &ck) || !maps.get(v, &cv) || !maps.get(out, &co))
+        return cudaErrorInvalidValue;
+    const Sched sch = Lc > 0 ? make_sched(t->dm, Lc, t->G) : t->sch;
+    return launch<false>(t, sch, cq, ck, cv, Lc > 0 ? *kc : ck, Lc > 0 ? *vc : cv, co, Lc, scale, err, st);
 }
 
 }  // namespace arl2

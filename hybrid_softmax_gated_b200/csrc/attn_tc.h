@@ -1,5 +1,7 @@
 // Tensor-core (tcgen05) kernel for the per-pass read of the ARL2 layer:
 //   out = softmax(Q K^T scale) V + Q (W_q S_{N-1})
+// and, without the state read, for the softmax teacher layer whose keys and
+// values run on from a KV cache into the frame's own.
 // bf16 in, fp32 accumulate in TMEM, bf16 out; head_dim 128.
 #pragma once
 
@@ -29,5 +31,14 @@ int* attn_tc_flags(AttnTc* t, size_t* count);
 cudaError_t attn_tc_launch(AttnTc* t, TokenMapCache& maps, const void* q, const void* k,
                            const void* v, const void* Mt, void* out, float scale, int* err,
                            cudaStream_t st);
+
+// Plain softmax attention of the frame's queries over Lc cached keys, then
+// the frame's own L keys (the softmax teacher layer with a KV cache):
+//   out = softmax([Q Kc^T, Q K^T] scale) [Vc; V]
+// kc, vc: maps of the cache's first Lc rows (tma_encode_token_rows); unused
+// (may be null) when Lc = 0.
+cudaError_t attn_tc_launch_cached(AttnTc* t, TokenMapCache& maps, const void* q, const void* k,
+                                  const void* v, const CUtensorMap* kc, const CUtensorMap* vc, int Lc,
+                                  void* out, float scale, int* err, cudaStream_t st);
 
 }  // namespace arl2

@@ -37,6 +37,19 @@ cudaError_t launch_attn_simt(bool bf16, const void* q, const void* k, const void
                              const float* qp, const float* S, void* out, float scale,
                              Dims dm, cudaStream_t st);
 
+// The same attention with Lc leading keys from a KV cache kc, vc
+// ([B][cap][H][d], element type of q); S == nullptr: no inter term (the
+// softmax teacher layer), qp unused then.
+cudaError_t launch_attn_simt_cached(bool bf16, const void* q, const void* k, const void* v,
+                                    const void* kc, const void* vc, int Lc, long long cap,
+                                    const float* qp, const float* S, void* out, float scale, Dims dm,
+                                    cudaStream_t st);
+
+// Copy a frame's k and v ([B][L][H][d], esz bytes per element) into frames
+// [slot, slot + 1) of the caches kc, vc ([B][cap_frames * L][H][d]).
+cudaError_t launch_kv_append(const void* k, const void* v, void* kc, void* vc, size_t esz, int slot,
+                             int cap_frames, Dims dm, cudaStream_t st);
+
 // r = vp - kp S, written over vp (fp32 [B][L][H][d]); S is the pre-update state.
 cudaError_t launch_residual_simt(const float* kp, float* vp_to_r, const float* S, Dims dm,
                                  cudaStream_t st);

@@ -128,12 +128,15 @@ __global__ void __launch_bounds__(kPhiThreads) phi_simt_kernel(const T* __restri
 // --------------------------------------------------------------- attn ----
 // One block: 32 query rows of one (b, h); 256 threads, thread (r, g) with
 // r = tid / 8 owns output columns g, g+8, g+16, ... of row r.  Keys stream
-// through shared memory 32 at a time with an online softmax.
+// through shared memory 32 at a time with an online softmax: first the Lc
+// keys of a KV cache (kc, vc: [B][cap][H][d], the softmax teacher layer),
+// then the frame's own L.  S == nullptr: no inter-frame read.
 constexpr int kAQ = 32, kAK = 32, kAThreads = 256, kAColsPerThread = 16;
 
 template <typename T>
 __global__ void __launch_bounds__(kAThreads) attn_simt_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+    const T* __restrict__ kc, const T* __restrict__ vc, int Lc, long long cap,
     const float* __restrict__ qp, const float* __restrict__ S, T* __restrict__ out,
     float scale_log2, Dims dm) {
     extern __shared__ float sm[];
@@ -157,14 +160,24 @@ __global__ void __launch_bounds__(kAThreads) attn_simt_kernel(
     for (int i = 0; i < kAColsPerThread; ++i) o[i] = 0.f;
     float m = -INFINITY, l = 0.f;
 
-    for (int k0 = 0; k0 < dm.L; k0 += kAK) {
-        const int nk = min(kAK, dm.L - k0);
+    const int Lk = Lc + dm.L;
+    for (int k0 = 0; k0 < Lk; k0 += kAK) {
+        const int nk = min(kAK, Lk - k0);
         __syncthreads();  // previous tile fully consumed (and Qs written)
         for (int i = tid; i < kAK * d; i += kAThreads) {
             const int j = i / d, c = i - j * d;
-            const bool ok = j < nk;
-            Ks[j * (d + 1) + c] = ok ? to_f(k[tok(b, k0 + j, h, c, dm)]) : 0.f;
-            Vs[j * d + c] = ok ? to_f(v[tok(b, k0 + j, h, c, dm)]) : 0.f;
+            const int t = k0 + j;
+            float kx = 0.f, vx = 0.f;
+            if (j < nk && t < Lc) {
+                const size_t o = (((size_t)b * cap + t) * dm.H + h) * d + c;
+                kx = to_f(kc[o]);
+                vx = to_f(vc[o]);
+            } else if (j < nk) {
+                kx = to_f(k[tok(b, t - Lc, h, c, dm)]);
+                vx = to_f(v[tok(b, t - Lc, h, c, dm)]);
+            }
+            Ks[j * (d + 1) + c] = kx;
+            Vs[j * d + c] = vx;
         }
         __syncthreads();
         float s[4];
@@ -204,6 +217,16 @@ __global__ void __launch_bounds__(kAThreads) attn_simt_kernel(
         }
     }
     const float inv_l = 1.f / l;
+    if (!S) {
+        if (r < nq) {
+#pragma unroll
+            for (int i = 0; i < kAColsPerThread; ++i) {
+                const int c = g + 8 * i;
+                if (c < d) out[tok(b, q0 + r, h, c, dm)] = from_f<T>(o[i] * inv_l);
+            }
+        }
+        return;
+    }
     __syncthreads();
     // inter-frame read: (q W_q) S with the pre-update state
     const float* Sbh = S + ((size_t)b * dm.H + h) * d * d;
@@ -327,23 +350,31 @@ cudaError_t launch_phi_simt(bool bf16, const void* x, const void* w, bool l2norm
     return cudaGetLastError();
 }
 
-cudaError_t launch_attn_simt(bool bf16, const void* q, const void* k, const void* v,
-                             const float* qp, const float* S, void* out, float scale, Dims dm,
-                             cudaStream_t st) {
+cudaError_t launch_attn_simt_cached(bool bf16, const void* q, const void* k, const void* v,
+                                    const void* kc, const void* vc, int Lc, long long cap,
+                                    const float* qp, const float* S, void* out, float scale, Dims dm,
+                                    cudaStream_t st) {
     const int d = dm.d;
     const size_t smem = sizeof(float) * ((size_t)kAQ * d + (size_t)kAK * (d + 1) +
                                          (size_t)kAK * d + (size_t)kAQ * (kAK + 1) + (size_t)d * d);
     const dim3 grid((dm.L + kAQ - 1) / kAQ, dm.H, dm.B);
     const float scale_log2 = scale * 1.4426950408889634f;
     if (bf16) {
-        attn_simt_kernel<__nv_bfloat16><<<grid, kAThreads, smem, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                           (const __nv_bfloat16*)v, qp, S, (__nv_bfloat16*)out,
-                                           scale_log2, dm);
+        attn_simt_kernel<__nv_bfloat16><<<grid, kAThreads, smem, st>>>(
+            (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, (const __nv_bfloat16*)kc,
+            (const __nv_bfloat16*)vc, Lc, cap, qp, S, (__nv_bfloat16*)out, scale_log2, dm);
     } else {
-        attn_simt_kernel<float><<<grid, kAThreads, smem, st>>>((const float*)q, (const float*)k, (const float*)v, qp, S,
-                                           (float*)out, scale_log2, dm);
+        attn_simt_kernel<float><<<grid, kAThreads, smem, st>>>((const float*)q, (const float*)k, (const float*)v,
+                                                               (const float*)kc, (const float*)vc, Lc, cap, qp, S,
+                                                               (float*)out, scale_log2, dm);
     }
     return cudaGetLastError();
+}
+
+cudaError_t launch_attn_simt(bool bf16, const void* q, const void* k, const void* v,
+                             const float* qp, const float* S, void* out, float scale, Dims dm,
+                             cudaStream_t st) {
+    return launch_attn_simt_cached(bf16, q, k, v, nullptr, nullptr, 0, 0, qp, S, out, scale, dm, st);
 }
 
 cudaError_t launch_residual_simt(const float* kp, float* vp_to_r, const float* S, Dims dm,

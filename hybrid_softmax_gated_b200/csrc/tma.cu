@@ -49,6 +49,14 @@ bool tma_encode_tokens(CUtensorMap* m, const void* p, const Dims& dm) {
     return encode4(m, p, dims, strides, box);
 }
 
+bool tma_encode_token_rows(CUtensorMap* m, const void* p, int B, int H, int rows, long long capacity) {
+    if (rows < 1 || rows > capacity) return false;
+    const cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {128 * 2, (cuuint64_t)H * 128 * 2, (cuuint64_t)capacity * H * 128 * 2};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    return encode4(m, p, dims, strides, box);
+}
+
 bool tma_encode_tiles(CUtensorMap* m, const void* p, int outer) {
     const cuuint64_t dims[4] = {128, 128, (cuuint64_t)outer, 1};
     const cuuint64_t strides[3] = {128 * 2, 128 * 128 * 2, (cuuint64_t)outer * 128 * 128 * 2};

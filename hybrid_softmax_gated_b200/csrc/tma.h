@@ -17,6 +17,11 @@ bool tma_available();
 // Token tensor [B][L][H][128] bf16: dims {128, H, L, B}; box {64, 1, 128, 1}.
 bool tma_encode_tokens(CUtensorMap* m, const void* p, const Dims& dm);
 
+// The first `rows` token rows of a [B][capacity][H][128] bf16 buffer (a KV
+// cache): dims {128, H, rows, B}, batch stride capacity rows; rows past
+// `rows` read as zeros.
+bool tma_encode_token_rows(CUtensorMap* m, const void* p, int B, int H, int rows, long long capacity);
+
 // Square bf16 tiles [outer][128][128] (outer = H or B*H flattened, the
 // innermost dimension contiguous): dims {128, 128, outer}; box {64, 128, 1}.
 bool tma_encode_tiles(CUtensorMap* m, const void* p, int outer);

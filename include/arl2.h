@@ -205,6 +205,88 @@ arl2_status arl2_state_update_noalloc(int batch, int heads, int head_dim, int to
  * NULL is ignored. */
 void arl2_destroy(arl2_handle* h);
 
+/* ------------------------------------------------------------------------
+ * Softmax teacher layer with a KV cache.
+ *
+ * The attention the hybrid layer replaces, kept by the layers of a stack
+ * that stay softmax: technical summary §1 ("KV Cache Growth": the cache of
+ * keys and values grows with every generated frame) and §4 ("Efficiency":
+ * the speedup of the hybrid stack grows with video length as that cache
+ * comes to dominate).  The pages fix the cache's role, not its arithmetic;
+ * this layer reads it as chunk-causal attention at frame granularity.  For
+ * one pass of frame N (N = arl2_kv_frames before the call):
+ *   O = softmax([Q Kc^T, Q K^T] * scale) [Vc; V]
+ * where (Kc, Vc) hold the keys and values of the clean passes of frames
+ * 0..N-1 in frame order, and (K, V) are this pass's own, attended
+ * bidirectionally.  A clean pass then appends its k and v to the cache (the
+ * same passes that update the hybrid layer's state, §2.2 "Clean-Pass
+ * Updates"); other passes leave the cache alone.
+ *
+ * The cache holds max_frames frames and is allocated by arl2_kv_create; no
+ * later call allocates.  Device memory held: 2 B max_frames L H d elements
+ * of dtype plus workspaces; the part in use grows by 2 B L H d elements per
+ * frame (arl2_kv_cache_bytes). */
+typedef struct arl2_kv_handle arl2_kv_handle;
+
+typedef struct {
+    int batch;             /* B >= 1                                          */
+    int heads;             /* H >= 1                                          */
+    int head_dim;          /* d: 128 for the bf16 tensor-core kernel; 1..128 SIMT */
+    int tokens_per_frame;  /* L >= 1                                          */
+    int max_frames;        /* cache capacity in frames, >= 1; max_frames * L
+                              <= 2^26                                         */
+    arl2_dtype dtype;      /* dtype of q, k, v, out and the cache             */
+    float softmax_scale;   /* 0 selects 1/sqrt(d)                             */
+    int host_staging;      /* nonzero: staging buffers for
+                              arl2_kv_frame_forward_host                      */
+    arl2_impl impl;
+    int max_ctas;          /* as in arl2_config                               */
+} arl2_kv_config;
+
+/* Create a teacher layer with an empty cache on the current device.
+ * Errors: INVALID_ARG, SHAPE, UNSUPPORTED (dtype/head_dim), OOM, CUDA. */
+arl2_status arl2_kv_create(const arl2_kv_config* cfg, cudaStream_t stream, arl2_kv_handle** out);
+
+/* One pass of one frame: out = the attention above over the cached frames
+ * and this pass's k, v; with clean_pass nonzero, then appends k and v to the
+ * cache.  q, k, v, out: device [B][L][H][d] dtype, 16-byte aligned; out must
+ * not alias q, k or v.  SHAPE (nothing enqueued) for a clean pass when the
+ * cache already holds max_frames frames.  The frame count lives on the host:
+ * a call recorded into a CUDA graph keeps the cache length it saw. */
+arl2_status arl2_kv_frame_forward(arl2_kv_handle* h, const void* q, const void* k, const void* v,
+                                  int clean_pass, void* out, cudaStream_t stream);
+
+/* arl2_kv_frame_forward on HOST buffers (pinned for asynchronous copies):
+ * q, k, v are copied into the handle's staging buffers, and out back, all
+ * stream-ordered.  Needs host_staging != 0 (INVALID_ARG otherwise). */
+arl2_status arl2_kv_frame_forward_host(arl2_kv_handle* h, const void* q, const void* k, const void* v,
+                                       int clean_pass, void* out, cudaStream_t stream);
+
+/* Empty the cache (the start of a new video stream).  Host-side only. */
+arl2_status arl2_kv_reset(arl2_kv_handle* h);
+
+/* Frames in the cache; -1 for NULL. */
+int arl2_kv_frames(const arl2_kv_handle* h);
+
+/* Copy the cached keys and values to device buffers k_dst, v_dst, each
+ * [B][frames * L][H][d] dtype (dense).  Nothing is copied while empty. */
+arl2_status arl2_kv_cache_get(arl2_kv_handle* h, void* k_dst, void* v_dst, cudaStream_t stream);
+
+/* As arl2_device_status, for the teacher layer's kernels. */
+arl2_status arl2_kv_device_status(arl2_kv_handle* h, cudaStream_t stream);
+
+/* Device bytes the handle holds (the whole cache capacity included). */
+size_t arl2_kv_device_bytes(const arl2_kv_handle* h);
+
+/* Bytes of the cache in use: 2 B frames L H d elements of dtype. */
+size_t arl2_kv_cache_bytes(const arl2_kv_handle* h);
+
+/* Kernels this handle has enqueued since creation. */
+unsigned long long arl2_kv_kernel_launches(const arl2_kv_handle* h);
+
+/* Release the handle (synchronises the device first); NULL is ignored. */
+void arl2_kv_destroy(arl2_kv_handle* h);
+
 /* Static string for a status code. */
 const char* arl2_status_string(arl2_status s);
 

@@ -39,7 +39,7 @@ def test_binding_covers_every_export():
 
 
 def test_version_and_status_strings():
-    assert arl2.version() == 10100
+    assert arl2.version() == 10200
     for code in range(0, -8, -1):
         s = arl2._lib.arl2_status_string(code).decode()
         assert s and s != "unknown status"
@@ -89,3 +89,34 @@ def test_gating_mode_is_validated_before_cuda():
     assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1
     cfg = arl2.Arl2Config(1, 1, 16, 16, 1, fake, fake, fake, 0.0, 0, 0, -1, arl2.ARL2_GATE_ELEMENTWISE)
     assert lib.arl2_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1  # (max_ctas < 0)
+
+
+def test_teacher_layer_arguments_are_validated_before_cuda():
+    lib = arl2._lib
+    h = ctypes.c_void_p()
+    K = arl2.Arl2KvConfig
+    assert lib.arl2_kv_create(None, None, ctypes.byref(h)) == -1
+    cfg = K(1, 1, 16, 16, 4, arl2.ARL2_FP32, 0.0, 0, 0, 0)
+    assert lib.arl2_kv_create(ctypes.byref(cfg), None, None) == -1
+    for bad in [(0, 1, 16, 16, 4), (1, 0, 16, 16, 4), (1, 1, 0, 16, 4), (1, 1, 129, 16, 4),
+                (1, 1, 16, 0, 4), (1, 1, 16, 16, 0), (1, 1, 16, 1 << 20, 1 << 7)]:
+        cfg = K(*bad, arl2.ARL2_FP32, 0.0, 0, 0, 0)
+        assert lib.arl2_kv_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -2, bad
+    cfg = K(1, 1, 64, 16, 4, arl2.ARL2_BF16, 0.0, 0, 0, 0)  # tensor cores need d = 128
+    assert lib.arl2_kv_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -7
+    cfg = K(1, 1, 16, 16, 4, 9, 0.0, 0, 0, 0)  # no such dtype
+    assert lib.arl2_kv_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1
+    cfg = K(1, 1, 16, 16, 4, arl2.ARL2_FP32, -0.5, 0, 0, 0)  # bad scale
+    assert lib.arl2_kv_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1
+    cfg = K(1, 1, 16, 16, 4, arl2.ARL2_FP32, 0.0, 0, 3, 0)  # no such impl
+    assert lib.arl2_kv_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1
+    assert lib.arl2_kv_frame_forward(None, None, None, None, 0, None, None) == -1
+    assert lib.arl2_kv_frame_forward_host(None, None, None, None, 0, None, None) == -1
+    assert lib.arl2_kv_reset(None) == -1
+    assert lib.arl2_kv_frames(None) == -1
+    assert lib.arl2_kv_cache_get(None, None, None, None) == -1
+    assert lib.arl2_kv_device_status(None, None) == -1
+    assert lib.arl2_kv_device_bytes(None) == 0
+    assert lib.arl2_kv_cache_bytes(None) == 0
+    assert lib.arl2_kv_kernel_launches(None) == 0
+    lib.arl2_kv_destroy(None)
