@@ -292,6 +292,32 @@ def run_reference(args, w: workloads.Workload):
 
 
 # -------------------------------------------------------------- GPU side --
+def profile_teacher_case(args, w: workloads.Workload) -> int:
+    """Profiling case of the teacher layer: a cache of --profile-teacher
+    frames loaded directly (cache_set, no attention launches), then
+    --profile-passes passes over a ring of inputs, the last one clean."""
+    from hybrid_softmax_gated_b200 import TeacherLayer
+    n = args.profile_teacher
+    B, L, H, d = w.batch, w.tokens, w.heads, w.head_dim
+    tea = TeacherLayer(B, H, d, L, n + 1, dtype=w.torch_dtype)
+    g = torch.Generator(device="cuda").manual_seed(workloads.subseed(workloads.SEED_BASE, 7, n))
+    kc = torch.randn(B, n * L, H, d, generator=g, device="cuda").to(w.torch_dtype)
+    vc = torch.randn(B, n * L, H, d, generator=g, device="cuda").to(w.torch_dtype)
+    tea.cache_set(kc, vc)
+    ring = 4
+    ins = [workloads.pass_inputs(w, 0, 0, i, device="cuda") for i in range(ring)]
+    out = torch.empty_like(ins[0][0])
+    passes = max(1, args.profile_passes)
+    for i in range(passes):  # the last pass is clean: it appends to the cache
+        tea.forward(*ins[i % ring], clean_pass=i == passes - 1, out=out)
+    torch.cuda.synchronize()
+    st = tea.device_status()
+    tea.close()
+    print(f"teacher profile case {w.name}: {n} cached frames ({n * L} keys), "
+          f"{passes} passes (the last one clean), status {st}")
+    return 0 if st == 0 else 1
+
+
 def profile_case(args, w: workloads.Workload) -> int:
     """A small case for ncu: one clean pass (non-zero state), then
     --profile-passes read-only passes cycling through a ring of input sets
@@ -453,6 +479,9 @@ def main():
     ap.add_argument("--stack-curve", action="store_true",
                     help="softmax KV-cache teacher vs hybrid layer over one long stream, and the "
                          "30-layer stacks built from them (one JSON line, not the headline)")
+    ap.add_argument("--profile-teacher", type=int, default=0,
+                    help="profiling case of the teacher layer with this many cached frames "
+                         "(read-only passes as --profile-passes; no timing, no JSON line)")
     ap.add_argument("--curve-frames", type=int, default=231,
                     help="latent frames of the stack-curve stream (231: 921 video frames)")
     ap.add_argument("--profile-passes", type=int, default=0,
@@ -467,6 +496,8 @@ def main():
 
     ws, rank, local = dist_env()
     torch.cuda.set_device(local)
+    if args.profile_teacher > 0:
+        return profile_teacher_case(args, w)
     if args.profile_passes > 0:
         return profile_case(args, w)
     if args.stack_curve:

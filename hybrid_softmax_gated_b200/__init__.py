@@ -40,7 +40,7 @@ EXPORTED = (
     "arl2_device_bytes", "arl2_kernel_launches", "arl2_state_update_noalloc", "arl2_destroy",
     "arl2_status_string", "arl2_version",
     "arl2_kv_create", "arl2_kv_frame_forward", "arl2_kv_frame_forward_host", "arl2_kv_reset",
-    "arl2_kv_frames", "arl2_kv_cache_get", "arl2_kv_device_status", "arl2_kv_device_bytes",
+    "arl2_kv_frames", "arl2_kv_cache_get", "arl2_kv_cache_set", "arl2_kv_device_status", "arl2_kv_device_bytes",
     "arl2_kv_cache_bytes", "arl2_kv_kernel_launches", "arl2_kv_destroy",
 )
 NOALLOC_MAX_ELEMENTS = 1 << 22
@@ -93,6 +93,7 @@ def _load() -> ctypes.CDLL:
         "arl2_kv_reset": ([H], I),
         "arl2_kv_frames": ([H], I),
         "arl2_kv_cache_get": ([H, P, P, P], I),
+        "arl2_kv_cache_set": ([H, P, P, I, P], I),
         "arl2_kv_device_status": ([H, P], I),
         "arl2_kv_device_bytes": ([H], S),
         "arl2_kv_cache_bytes": ([H], S),
@@ -370,6 +371,18 @@ class TeacherLayer:
         vc = torch.empty_like(kc)
         _check(_lib.arl2_kv_cache_get(self.handle, _ptr(kc), _ptr(vc), _stream(stream)), "arl2_kv_cache_get")
         return kc, vc
+
+    def cache_set(self, k, v, stream=None) -> None:
+        """Load the cache from (k, v), [B, n * L, H, d] each (n whole frames)."""
+        B, L, H, d = self.shape
+        for t in (k, v):
+            if not (t.is_cuda and t.is_contiguous() and t.dtype == self.dtype and t.dim() == 4
+                    and t.shape[0] == B and t.shape[2:] == (H, d) and t.shape[1] % L == 0):
+                raise ValueError("cache tensors must be contiguous CUDA tensors [B, n * L, H, d]")
+        if k.shape != v.shape:
+            raise ValueError("k and v must have the same shape")
+        _check(_lib.arl2_kv_cache_set(self.handle, _ptr(k), _ptr(v), k.shape[1] // L, _stream(stream)),
+               "arl2_kv_cache_set")
 
     def device_status(self, stream=None) -> int:
         return _lib.arl2_kv_device_status(self.handle, _stream(stream))

@@ -289,6 +289,25 @@ arl2_status arl2_kv_cache_get(arl2_kv_handle* h, void* k_dst, void* v_dst, cudaS
     return ARL2_OK;
 }
 
+arl2_status arl2_kv_cache_set(arl2_kv_handle* h, const void* k_src, const void* v_src, int frames,
+                              cudaStream_t stream) {
+    if (!h || frames < 0 || (frames > 0 && (!k_src || !v_src))) return ARL2_ERR_INVALID_ARG;
+    if (frames > h->cap_frames) return ARL2_ERR_SHAPE;
+    arl2_status s = check_device(h);
+    if (s != ARL2_OK) return s;
+    if (frames > 0) {
+        const size_t frame_b = (size_t)h->dm.L * h->dm.H * h->dm.d * h->esz;
+        const size_t width = frame_b * frames, pitch = frame_b * h->cap_frames;
+        if (cudaMemcpy2DAsync(h->kc, pitch, k_src, width, width, h->dm.B, cudaMemcpyDeviceToDevice, stream) !=
+                cudaSuccess ||
+            cudaMemcpy2DAsync(h->vc, pitch, v_src, width, width, h->dm.B, cudaMemcpyDeviceToDevice, stream) !=
+                cudaSuccess)
+            return ARL2_ERR_CUDA;
+    }
+    h->frames = frames;
+    return ARL2_OK;
+}
+
 arl2_status arl2_kv_device_status(arl2_kv_handle* h, cudaStream_t stream) {
     if (!h) return ARL2_ERR_INVALID_ARG;
     arl2_status s = check_device(h);

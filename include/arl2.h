@@ -272,6 +272,13 @@ int arl2_kv_frames(const arl2_kv_handle* h);
  * [B][frames * L][H][d] dtype (dense).  Nothing is copied while empty. */
 arl2_status arl2_kv_cache_get(arl2_kv_handle* h, void* k_dst, void* v_dst, cudaStream_t stream);
 
+/* Replace the cache by `frames` frames from device buffers k_src, v_src,
+ * each [B][frames * L][H][d] dtype (dense): resume from a checkpoint taken
+ * with arl2_kv_cache_get.  frames = 0 empties the cache.  Errors:
+ * INVALID_ARG, SHAPE (frames > max_frames), CUDA. */
+arl2_status arl2_kv_cache_set(arl2_kv_handle* h, const void* k_src, const void* v_src, int frames,
+                              cudaStream_t stream);
+
 /* As arl2_device_status, for the teacher layer's kernels. */
 arl2_status arl2_kv_device_status(arl2_kv_handle* h, cudaStream_t stream);
 

@@ -115,6 +115,7 @@ def test_teacher_layer_arguments_are_validated_before_cuda():
     assert lib.arl2_kv_reset(None) == -1
     assert lib.arl2_kv_frames(None) == -1
     assert lib.arl2_kv_cache_get(None, None, None, None) == -1
+    assert lib.arl2_kv_cache_set(None, None, None, 0, None) == -1
     assert lib.arl2_kv_device_status(None, None) == -1
     assert lib.arl2_kv_device_bytes(None) == 0
     assert lib.arl2_kv_cache_bytes(None) == 0

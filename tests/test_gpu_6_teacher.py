@@ -177,3 +177,27 @@ def test_teacher_kernel_launch_count():
         assert lay.kernel_launches() == 3  # attention, then the append
     finally:
         lay.close()
+
+
+def test_teacher_cache_checkpoint_and_resume():
+    # a layer resumed from another's cache continues exactly as the original
+    w = small(130, frames=4)
+    a = make_teacher(w)
+    b = make_teacher(w)
+    try:
+        for f in range(2):
+            q, k, v = (t.cuda() for t in workloads.pass_inputs(w, 0, f, 1))
+            a.forward(q, k, v, clean_pass=True)
+        kc, vc = a.cache_get()
+        b.cache_set(kc, vc)
+        assert b.frames() == 2
+        for f in range(2, 4):
+            q, k, v = (t.cuda() for t in workloads.pass_inputs(w, 0, f, 1))
+            assert torch.equal(a.forward(q, k, v, clean_pass=True), b.forward(q, k, v, clean_pass=True))
+        with pytest.raises(Arl2Error):
+            b.cache_set(torch.cat([kc] * 3, 1), torch.cat([vc] * 3, 1))  # 6 frames > capacity 4
+        b.cache_set(kc[:, :0], vc[:, :0])
+        assert b.frames() == 0
+    finally:
+        a.close()
+        b.close()
