@@ -363,7 +363,10 @@ def stack_curve(args, w: workloads.Workload) -> int:
     larger than L2.  A stack's attention time is the sum over its layers
     (the layers are independent work of identical cost per kind); its memory
     is the sum of the teacher layers' KV caches and the hybrid layers' state
-    copies and workspaces.  Attention only: the pages' figures are whole-model.
+    copies and workspaces.  Real mixed stacks of 30 layers (50 % and 75 %
+    hybrid, spread evenly) then run the first --stack-frames frames, every
+    layer with its own handle, to check that sum.  Attention only: the pages'
+    figures are whole-model.
     """
     from hybrid_softmax_gated_b200 import Arl2Layer, TeacherLayer
     F = args.curve_frames
@@ -443,6 +446,66 @@ def stack_curve(args, w: workloads.Workload) -> int:
             v["memory_vs_all_softmax"] = v["attn_bytes"] / base["attn_bytes"]
         row["stack30"] = stacks
         curve.append(row)
+    # A real mixed stack: 30 layers (each its own handle and weights) run
+    # frame by frame, pass by pass, layer by layer over the first
+    # --stack-frames frames, against the sum of the single-layer times.
+    measured = []
+    Fs = min(args.stack_frames, F)
+    for r in (0.5, 0.75):
+        n_h = int(round(n_layers * r))
+        kinds = ["hybrid" if (i * n_h) // n_layers != ((i + 1) * n_h) // n_layers else "teacher"
+                 for i in range(n_layers)]
+        layers = []
+        for i, kind in enumerate(kinds):
+            if kind == "teacher":
+                layers.append(TeacherLayer(B, H, d, L, Fs, dtype=w.torch_dtype))
+            else:
+                wq_i, wk_i, wv_i = workloads.phi_weights(w, i)
+                layers.append(Arl2Layer(B, H, d, L, wq_i.cuda(), wk_i.cuda(), wv_i.cuda(), dtype=w.torch_dtype))
+        outs = [torch.empty_like(out) for _ in range(2)]
+
+        def stack_frame(f):
+            for p in range(w.passes):
+                clean = workloads.is_clean(w, p)
+                for i, lay in enumerate(layers):
+                    q, k, v = ins[(f * w.passes * n_layers + p * n_layers + i) % ring]
+                    if kinds[i] == "teacher":
+                        lay.forward(q, k, v, clean_pass=clean, out=outs[i & 1])
+                    else:
+                        lay.forward(q, k, v, a, b, clean_pass=clean, out=outs[i & 1])
+
+        graphs = []
+        for f in range(Fs):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap_stream):
+                stack_frame(f)
+            graphs.append(g)
+        for g in graphs:
+            g.replay()
+        torch.cuda.synchronize()
+        for kind, lay in zip(kinds, layers):
+            if kind == "hybrid":
+                lay.state_reset()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for g in graphs:
+            g.replay()
+        e1.record(st)
+        torch.cuda.synchronize()
+        t_meas = e0.elapsed_time(e1)
+        n_t = n_layers - n_h
+        t_model = n_t * sum(t_tea[:Fs]) + n_h * sum(t_hyb[:Fs])
+        mem = sum(lay.cache_bytes() if kind == "teacher" else lay.device_bytes()
+                  for kind, lay in zip(kinds, layers))
+        bad = [lay.device_status() for lay in layers]
+        del graphs
+        for lay in layers:
+            lay.close()
+        if any(bad):
+            raise SystemExit(f"device status {bad}")
+        measured.append({"hybrid_share": f"{int(r * 100)}%", "frames": Fs, "layers": n_layers,
+                         "hybrid_layers": n_h, "attn_ms_video_measured": t_meas,
+                         "attn_ms_video_sum_of_layers": t_model, "attn_bytes": mem})
     last = curve[-1]
     line = {
         "metric": "attention per video: softmax KV-cache teacher vs ARL2 hybrid layer (480p, 30-layer stacks)",
@@ -451,6 +514,7 @@ def stack_curve(args, w: workloads.Workload) -> int:
                    "passes": w.passes, "frames": F, "layers": n_layers,
                    "l2": f"inputs larger than L2 ({ring} input sets)"},
         "curve": curve,
+        "stack_measured": measured,
         "roofline": {"kernel": "attn_tc_kernel (teacher, longest cache)", "bound": "tensor",
                      "achieved": last["teacher_tflops_last_frame"], "peak": peaks["bf16_tflops_sustained"],
                      "unit": "TFLOP/s", "frac": last["teacher_tflops_last_frame"] / peaks["bf16_tflops_sustained"],
@@ -482,6 +546,8 @@ def main():
     ap.add_argument("--profile-teacher", type=int, default=0,
                     help="profiling case of the teacher layer with this many cached frames "
                          "(read-only passes as --profile-passes; no timing, no JSON line)")
+    ap.add_argument("--stack-frames", type=int, default=21,
+                    help="frames of the real mixed 30-layer stacks run by --stack-curve")
     ap.add_argument("--curve-frames", type=int, default=231,
                     help="latent frames of the stack-curve stream (231: 921 video frames)")
     ap.add_argument("--profile-passes", type=int, default=0,
