@@ -13,7 +13,8 @@ Method source: "Attend Locally, Remember Linearly" technical summary,
 section 2.1 (hybrid decomposition, phi maps, state update, inter read) and
 section 2.2 (frame-level access, clean-pass updates).  The softmax teacher
 layer with a KV cache (teacher_pass) follows section 1 ("KV Cache Growth")
-and section 4 ("Efficiency"): the attention the hybrid layer replaces.
+and section 4 ("Efficiency"): the attention the hybrid layer replaces.  The
+gate projections (gate_projection) follow section 2.1 ("State Update").
 """
 from __future__ import annotations
 
@@ -59,10 +60,12 @@ def _load():
                                                          P, P]
             lib.arl2_oracle_teacher_pass.argtypes = [I, I, I, I, I, D, P, P, P, P, P, P]
             lib.arl2_oracle_teacher_rows.argtypes = [I, I, I, I, I, D, P, P, P, P, P, I, P, P, P]
+            lib.arl2_oracle_gate_projection.argtypes = [I, I, I, I, P, P, P, P, P]
             for f in (lib.arl2_oracle_pass, lib.arl2_oracle_rows,
                       lib.arl2_oracle_state_update, lib.arl2_oracle_state_update_gated,
                       lib.arl2_oracle_phi, lib.arl2_oracle_pass_token_level,
-                      lib.arl2_oracle_teacher_pass, lib.arl2_oracle_teacher_rows):
+                      lib.arl2_oracle_teacher_pass, lib.arl2_oracle_teacher_rows,
+                      lib.arl2_oracle_gate_projection):
                 f.restype = I
             _lib = lib
     return _lib
@@ -237,6 +240,26 @@ def teacher_append(cache_k, cache_v, k, v):
     if cache_k is None:
         return k.copy(), v.copy()
     return np.concatenate([f64(cache_k), k], axis=1), np.concatenate([f64(cache_v), v], axis=1)
+
+
+def gate_projection(x, w, bias):
+    """Gates from the layer's hidden states (the reading of "learned per-token
+    projections", technical summary section 2.1): per token and head the
+    logits a = x w[:, h] + bias[h] and g = x w[:, H + h] + bias[H + h];
+    beta = sigmoid(g) per token, alpha = sigmoid(mean over the frame's tokens
+    of a).  x [B, L, D], w [D, 2H], bias [2H].  Returns (alpha [B, H],
+    beta [B, H, L])."""
+    x, w, bias = f64(x), f64(w), f64(bias)
+    B, L, D = x.shape
+    if w.ndim != 2 or w.shape[0] != D or w.shape[1] % 2 or bias.shape != (w.shape[1],):
+        raise ValueError(f"gate weights {w.shape} / bias {bias.shape} for hidden size {D}")
+    H = w.shape[1] // 2
+    alpha = np.zeros((B, H))
+    beta = np.zeros((B, H, L))
+    rc = _load().arl2_oracle_gate_projection(B, L, D, H, _p(x), _p(w), _p(bias), _p(alpha), _p(beta))
+    if rc != 0:
+        raise RuntimeError("arl2_oracle_gate_projection failed")
+    return alpha, beta
 
 
 def zero_state(B: int, H: int, d: int) -> np.ndarray:

@@ -427,3 +427,42 @@ int arl2_oracle_teacher_rows(int B, int H, int d, int L, int Lc, double scale, c
     }
     return err ? -1 : 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Gate projections.  The technical summary (section 2.1 "State Update")
+ * calls alpha (forget gate) and beta (learning rate) learned per-token
+ * projections and gives no form; the reading taken here:
+ *   per token i and head h, two logits from the token's hidden state x_i:
+ *     a_ih = x_i . w[:, h]     + bias[h]
+ *     g_ih = x_i . w[:, H + h] + bias[H + h]
+ *   beta_ih = sigmoid(g_ih)                 (one rate per token)
+ *   alpha_h = sigmoid((1/L) sum_i a_ih)     (one forget gate per frame and
+ *             head: the frame updates the state once, section 2.2
+ *             "Frame-Level Access", and headwise gating is the form the
+ *             ablations adopt, section 4)
+ * x: [B][L][D] (the layer's input hidden states); w: [D][2H]; bias: [2H];
+ * alpha: [B][H]; beta: [B][H][L]. */
+static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
+
+int arl2_oracle_gate_projection(int B, int L, int D, int H, const double* x, const double* w,
+                                const double* bias, double* alpha, double* beta) {
+    if (B < 1 || L < 1 || D < 1 || H < 1 || !x || !w || !bias || !alpha || !beta) return -1;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            double a_sum = 0.0;
+            for (int i = 0; i < L; ++i) {
+                const double* xi = x + ((size_t)b * L + i) * D;
+                double a = bias[h], g = bias[H + h];
+                for (int e = 0; e < D; ++e) {
+                    a += xi[e] * w[(size_t)e * 2 * H + h];
+                    g += xi[e] * w[(size_t)e * 2 * H + H + h];
+                }
+                beta[((size_t)b * H + h) * L + i] = sigmoid(g);
+                a_sum += a;
+            }
+            alpha[(size_t)b * H + h] = sigmoid(a_sum / L);
+        }
+    }
+    return 0;
+}

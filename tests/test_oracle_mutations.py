@@ -54,6 +54,14 @@ MUTATIONS = {
         "for (int c = 0; c < d; ++c) acc += kp[(size_t)i * d + c] * St[(size_t)c * d + n];",
         "for (int c = 0; c < d; ++c) acc += kp[(size_t)i * d + c] * S[(size_t)c * d + n];"),
     "token_level_gate_every_token": ("if (i == 0) g = alpha_per_key", "if (1) g = alpha_per_key"),
+    "gate_alpha_mean_of_sigmoids": ("a_sum += a;", "a_sum += sigmoid(a) - 0.5;"),
+    "gate_alpha_sum_not_mean": ("alpha[(size_t)b * H + h] = sigmoid(a_sum / L);",
+                                "alpha[(size_t)b * H + h] = sigmoid(a_sum);"),
+    "gate_weight_transposed": ("a += xi[e] * w[(size_t)e * 2 * H + h];",
+                               "a += xi[e] * w[(size_t)h * D + e];"),
+    "gate_beta_bias_dropped": ("double a = bias[h], g = bias[H + h];", "double a = bias[h], g = 0.0;"),
+    "gate_alpha_from_beta_column": ("a += xi[e] * w[(size_t)e * 2 * H + h];",
+                                    "a += xi[e] * w[(size_t)e * 2 * H + H + h];"),
     "teacher_scale_dropped": ("s[j] = dot * scale;", "s[j] = dot;"),
     "teacher_cached_values_from_keys": ("const double* vj = j < Lc ? vc + IDX4(b, j, h, 0, Lc, H, d)",
                                         "const double* vj = j < Lc ? kc + IDX4(b, j, h, 0, Lc, H, d)"),

@@ -10,7 +10,8 @@ streams and heads, scale invariance of the k' normalisation).
 Method text: "Attend Locally, Remember Linearly", technical summary
 section 2.1 (branches, phi maps, state update, read) and section 2.2
 (frame-level access, clean-pass updates); the softmax teacher layer with a
-KV cache from section 1 (KV Cache Growth) and section 4 (Efficiency).
+KV cache from section 1 (KV Cache Growth) and section 4 (Efficiency); the
+gate projections from section 2.1 (State Update).
 """
 import json
 import math
@@ -78,6 +79,13 @@ def golden_cases():
 
 @pytest.mark.parametrize("case", golden_cases(), ids=lambda c: c["name"])
 def test_hand_worked_case(case):
+    if case.get("layer") == "gates":
+        alpha, beta = oracle.gate_projection(np.asarray(case["x"], dtype=np.float64)[None],
+                                             np.asarray(case["w"], dtype=np.float64),
+                                             np.asarray(case["bias"], dtype=np.float64))
+        np.testing.assert_allclose(alpha[0, 0], case["expected_alpha"], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(beta[0, 0], case["expected_beta"], rtol=0, atol=1e-12)
+        return
     d, L = case["d"], case["L"]
     zeros = np.zeros((L, d))
     q = as_blhd(case.get("q", zeros))
@@ -596,3 +604,101 @@ def test_teacher_rejects_bad_arguments():
         oracle.teacher_pass(q, k, v, kc, vc[:, :3])
     with pytest.raises(RuntimeError):
         oracle.teacher_rows(q, k, v, kc, vc, [2], [0])
+
+
+# --------------------------------------------------------------------------
+# Gate projections (technical summary section 2.1 "State Update": alpha and
+# beta are learned per-token projections; reading: linear logits per token,
+# beta = sigmoid(g_i), alpha = sigmoid(mean_i a_i))
+# --------------------------------------------------------------------------
+
+def _gate_inputs(seed, B=2, L=9, D=12, H=3):
+    rng = np.random.default_rng(seed)
+    x = rnd(rng, B, L, D)
+    w = rnd(rng, D, 2 * H, scale=1.0 / np.sqrt(D))
+    bias = rnd(rng, 2 * H)
+    return x, w, bias
+
+
+def _logit(p):
+    return np.log(p) - np.log1p(-p)
+
+
+def test_gates_of_zero_hidden_states_are_the_bias_sigmoids():
+    x, w, bias = _gate_inputs(40)
+    a, b = oracle.gate_projection(np.zeros_like(x), w, bias)
+    H = w.shape[1] // 2
+    np.testing.assert_allclose(a, np.broadcast_to(1 / (1 + np.exp(-bias[:H])), a.shape), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(b, np.broadcast_to((1 / (1 + np.exp(-bias[H:])))[None, :, None], b.shape),
+                               rtol=0, atol=1e-15)
+
+
+def test_gate_logits_are_affine_in_the_hidden_state():
+    # logit(beta(x + y)) = logit(beta(x)) + logit(beta(y)) - bias, and the
+    # frame gate's logit (a mean of affine logits) obeys the same identity
+    x, w, bias = _gate_inputs(41)
+    y, _, _ = _gate_inputs(42)
+    H = w.shape[1] // 2
+    ax, bx = oracle.gate_projection(x, w, bias)
+    ay, by = oracle.gate_projection(y, w, bias)
+    axy, bxy = oracle.gate_projection(x + y, w, bias)
+    np.testing.assert_allclose(_logit(bxy), _logit(bx) + _logit(by) - bias[H:][None, :, None], rtol=0, atol=1e-9)
+    np.testing.assert_allclose(_logit(axy), _logit(ax) + _logit(ay) - bias[:H][None], rtol=0, atol=1e-9)
+
+
+def test_frame_gate_of_repeated_tokens_is_the_token_gate():
+    # L copies of one token: the mean logit is that token's logit
+    x, w, bias = _gate_inputs(43, L=1)
+    a1, _ = oracle.gate_projection(x, w, bias)
+    aL, bL = oracle.gate_projection(np.repeat(x, 7, axis=1), w, bias)
+    np.testing.assert_allclose(aL, a1, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(bL, np.repeat(bL[:, :, :1], 7, axis=2), rtol=0, atol=0)
+
+
+def test_frame_gate_is_the_sigmoid_of_the_mean_logit_not_the_mean_sigmoid():
+    # two single-token frames and their union: the union's logit is the mean
+    x, w, bias = _gate_inputs(44, L=2)
+    a0, b0 = oracle.gate_projection(x[:, :1], w, bias)
+    a1, b1 = oracle.gate_projection(x[:, 1:], w, bias)
+    a, b = oracle.gate_projection(x, w, bias)
+    np.testing.assert_allclose(_logit(a), (_logit(a0) + _logit(a1)) / 2, rtol=0, atol=1e-9)
+    np.testing.assert_allclose(b, np.concatenate([b0, b1], axis=2), rtol=0, atol=0)
+    assert np.abs(a - (a0 + a1) / 2).max() > 1e-4
+
+
+def test_gate_token_permutation():
+    x, w, bias = _gate_inputs(45)
+    perm = np.random.default_rng(4).permutation(x.shape[1])
+    a, b = oracle.gate_projection(x, w, bias)
+    ap, bp = oracle.gate_projection(x[:, perm], w, bias)
+    np.testing.assert_allclose(ap, a, rtol=0, atol=1e-14)
+    np.testing.assert_array_equal(bp, b[:, :, perm])
+
+
+def test_gate_heads_read_their_own_columns():
+    x, w, bias = _gate_inputs(46)
+    H = w.shape[1] // 2
+    a, b = oracle.gate_projection(x, w, bias)
+    w2, bias2 = w.copy(), bias.copy()
+    w2[:, 1] += 1.0          # head 1's alpha column
+    bias2[H + 2] -= 3.0      # head 2's beta bias
+    a2, b2 = oracle.gate_projection(x, w2, bias2)
+    np.testing.assert_array_equal(a2[:, [0, 2]], a[:, [0, 2]])
+    np.testing.assert_array_equal(b2[:, :2], b[:, :2])
+    assert np.abs(a2[:, 1] - a[:, 1]).max() > 1e-3 and np.abs(b2[:, 2] - b[:, 2]).max() > 1e-3
+    # and streams only their own hidden states
+    x2 = x.copy()
+    x2[1] += 1.0
+    a3, b3 = oracle.gate_projection(x2, w, bias)
+    np.testing.assert_array_equal(a3[0], a[0])
+    np.testing.assert_array_equal(b3[0], b[0])
+
+
+def test_gate_projection_rejects_bad_shapes():
+    x, w, bias = _gate_inputs(47)
+    with pytest.raises(ValueError):
+        oracle.gate_projection(x, w[:-1], bias)
+    with pytest.raises(ValueError):
+        oracle.gate_projection(x, w, bias[:-1])
+    with pytest.raises(ValueError):
+        oracle.gate_projection(x, w[:, :-1], bias[:-1])
