@@ -318,6 +318,25 @@ def profile_teacher_case(args, w: workloads.Workload) -> int:
     return 0 if st == 0 else 1
 
 
+def profile_gates_case(args, w: workloads.Workload) -> int:
+    """Profiling case of the gate projection: --profile-gates launches of
+    arl2_gates_apply over a ring of frames' hidden states."""
+    from hybrid_softmax_gated_b200 import Arl2Layer
+    wq, wk, wv = workloads.phi_weights(w, 0)
+    wg, bg = workloads.gate_projection_weights(w, 0)
+    lay = Arl2Layer(w.batch, w.heads, w.head_dim, w.tokens, wq.cuda(), wk.cuda(), wv.cuda(),
+                    dtype=w.torch_dtype, gate_weights=(wg.cuda(), bg.cuda()))
+    ring = 8
+    xs = [workloads.hidden_states(w, 0, f, device="cuda") for f in range(ring)]
+    for i in range(args.profile_gates):
+        lay.gates_apply(xs[i % ring])
+    torch.cuda.synchronize()
+    st = lay.device_status()
+    lay.close()
+    print(f"gate profile case {w.name}: {args.profile_gates} launches, status {st}")
+    return 0 if st == 0 else 1
+
+
 def profile_case(args, w: workloads.Workload) -> int:
     """A small case for ncu: one clean pass (non-zero state), then
     --profile-passes read-only passes cycling through a ring of input sets
@@ -539,10 +558,14 @@ def main():
                     help="forget gate per head (the pages' form) or per key feature")
     ap.add_argument("--access", default="frame", choices=["frame", "token"],
                     help="frame-level state access (the method) or token-level (the ablation)")
+    ap.add_argument("--gates", default="given", choices=["given", "projected"],
+                    help="alpha and beta as inputs, or projected in-kernel from the hidden states")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stack-curve", action="store_true",
                     help="softmax KV-cache teacher vs hybrid layer over one long stream, and the "
                          "30-layer stacks built from them (one JSON line, not the headline)")
+    ap.add_argument("--profile-gates", type=int, default=0,
+                    help="profiling case of the gate projection: this many launches (no timing)")
     ap.add_argument("--profile-teacher", type=int, default=0,
                     help="profiling case of the teacher layer with this many cached frames "
                          "(read-only passes as --profile-passes; no timing, no JSON line)")
@@ -564,6 +587,8 @@ def main():
     torch.cuda.set_device(local)
     if args.profile_teacher > 0:
         return profile_teacher_case(args, w)
+    if args.profile_gates > 0:
+        return profile_gates_case(args, w)
     if args.profile_passes > 0:
         return profile_case(args, w)
     if args.stack_curve:
@@ -575,14 +600,27 @@ def main():
 
     stream_idx = rank  # each rank: its own independent stream (replica)
     wq, wk, wv = workloads.phi_weights(w, 0)
+    projected = args.gates == "projected"
+    if projected and args.gating != "headwise":
+        raise SystemExit("--gates projected makes headwise gates")
+    gate_w = None
+    if projected:
+        wg, bg = workloads.gate_projection_weights(w, 0)
+        gate_w = (wg.cuda(), bg.cuda())
     lay = Arl2Layer(w.batch, w.heads, w.head_dim, w.tokens, wq.cuda(), wk.cuda(), wv.cuda(),
-                    dtype=w.torch_dtype, host_staging=True, gating=args.gating, access=args.access)
+                    dtype=w.torch_dtype, host_staging=True, gating=args.gating, access=args.access,
+                    gate_weights=gate_w)
     gate_draw = workloads.frame_gates_elementwise if args.gating == "elementwise" else workloads.frame_gates
-    # all inputs of the stream, resident in HBM before timing
-    ins, gates = [], []
+    # all inputs of the stream, resident in HBM before timing; with projected
+    # gates, the frame's hidden states instead of its alpha and beta
+    ins, gates, hidden = [], [], []
     for f in range(w.frames):
-        a, b = gate_draw(w, stream_idx, f)
-        gates.append((a.cuda(), b.cuda()))
+        if projected:
+            hidden.append(workloads.hidden_states(w, stream_idx, f, device="cuda"))
+            gates.append((None, None))
+        else:
+            a, b = gate_draw(w, stream_idx, f)
+            gates.append((a.cuda(), b.cuda()))
         for p in range(w.passes):
             ins.append(workloads.pass_inputs(w, stream_idx, f, p, device="cuda"))
     out = torch.empty_like(ins[0][0])
@@ -602,7 +640,11 @@ def main():
                 clean = workloads.is_clean(w, p)
                 if evs is not None and p == 0:
                     evs[f][0].record()
-                lay.forward(q, k, v, a, b, clean_pass=clean, out=out)
+                if projected:
+                    needs_x = clean or lay.token_level
+                    lay.forward_hidden(q, k, v, hidden[f] if needs_x else None, clean_pass=clean, out=out)
+                else:
+                    lay.forward(q, k, v, a, b, clean_pass=clean, out=out)
                 if evs is not None and p == w.passes - 2:
                     evs[f][1].record()
 
@@ -674,25 +716,61 @@ def main():
     if lay.device_status() != 0:
         raise SystemExit("device status not ok after the kernel timing")
 
+    gate_kernel = None
+    if projected:
+        # the gate projection alone: back-to-back launches over the frames'
+        # hidden states, one CUDA graph, an event pair around it
+        n_g = 4 * w.frames
+        lay.gates_apply(hidden[0])
+        gg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gg, stream=cap):
+            for i in range(n_g):
+                lay.gates_apply(hidden[i % w.frames])
+        gg.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(st)
+        gg.replay()
+        g1.record(st)
+        torch.cuda.synchronize()
+        g_ms = g0.elapsed_time(g1) / n_g
+        del gg
+        D = workloads.hidden_dim(w)
+        g_bytes = w.batch * w.tokens * D * 2 + D * 2 * w.heads * 2 + w.batch * w.heads * (w.tokens + 1) * 4
+        g_flops = 2.0 * w.batch * w.tokens * D * 2 * w.heads
+        gate_kernel = {"kernel": "gate_proj_kernel", "kernel_ms": g_ms, "bytes_per_launch": g_bytes,
+                       "achieved_gbs": g_bytes / (g_ms / 1e3) / 1e9, "hbm_peak_gbs": load_peaks()["hbm_gbs"],
+                       "achieved_tflops": g_flops / (g_ms / 1e3) / 1e12,
+                       "fp32_fma_peak_tflops": fp32_simt_tflops()}
+
     # end to end: host (pinned) buffers through arl2_frame_forward_host
     ring = 8
     host_in = [tuple(t.cpu().pin_memory() for t in ins[i]) for i in range(ring)]
-    host_gates = [tuple(t.cpu().pin_memory() for t in gates[f]) for f in range(min(ring, w.frames))]
+    if projected:
+        host_gates = [(hidden[f].cpu().pin_memory(),) for f in range(min(ring, w.frames))]
+    else:
+        host_gates = [tuple(t.cpu().pin_memory() for t in gates[f]) for f in range(min(ring, w.frames))]
     host_out = torch.empty(ins[0][0].shape, dtype=ins[0][0].dtype).pin_memory()
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     h2d = d2h = 0
     tok_bytes = ins[0][0].numel() * ins[0][0].element_size()
-    gate_bytes = (gates[0][0].numel() + gates[0][1].numel()) * 4
+    gate_bytes = (hidden[0].numel() * hidden[0].element_size() if projected
+                  else (gates[0][0].numel() + gates[0][1].numel()) * 4)
 
     def e2e_step():
         lay.state_reset()
         i = 0
         for f in range(w.frames):
-            a, b = host_gates[f % len(host_gates)]
+            g = host_gates[f % len(host_gates)]
             for p in range(w.passes):
                 q, k, v = host_in[i % ring]
                 i += 1
-                lay.forward_host(q, k, v, a, b, workloads.is_clean(w, p), host_out)
+                clean = workloads.is_clean(w, p)
+                if projected:
+                    needs_x = clean or lay.token_level
+                    lay.forward_hidden_host(q, k, v, g[0] if needs_x else None, clean, host_out)
+                else:
+                    lay.forward_host(q, k, v, g[0], g[1], clean, host_out)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -704,7 +782,8 @@ def main():
     e_stop.synchronize()
     barrier(ws)
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_stop), ws)
-    h2d = w.frames * (w.passes * 3 * tok_bytes + gate_bytes)
+    gate_passes = w.passes if args.access == "token" else 1  # the passes that carry gate inputs
+    h2d = w.frames * (w.passes * 3 * tok_bytes + gate_passes * gate_bytes)
     d2h = w.frames * w.passes * tok_bytes
     e2e_value = args.e2e_steps * w.frames * w.batch * ws / (e2e_ms / 1e3)
 
@@ -747,7 +826,7 @@ def main():
         "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
                    "tokens_per_frame": w.tokens, "frames_per_step": w.frames, "passes": w.passes,
                    "parallelism": f"replicas{ws}", "l2": "inputs larger than L2 (1.2 GB ring)",
-                   "gating": args.gating, "access": args.access},
+                   "gating": args.gating, "access": args.access, "gates": args.gates},
         "tokens_per_s": value * w.tokens,
         "tflops_per_frame_algorithmic": frame_flops(w) / 1e12,
         "roofline": roofline, "clocks": clk,
@@ -757,6 +836,8 @@ def main():
         "cpu_baseline": cpu,
         "peak_device_bytes": torch.cuda.max_memory_allocated() + lay.device_bytes(),
     }
+    if gate_kernel is not None:
+        line["gate_kernel"] = gate_kernel
     if rank == 0:
         print(json.dumps(line), flush=True)
     lay.close()

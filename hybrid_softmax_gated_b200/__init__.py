@@ -38,7 +38,8 @@ EXPORTED = (
     "arl2_create", "arl2_frame_forward", "arl2_frame_forward_host", "arl2_state_reset",
     "arl2_state_get", "arl2_state_set", "arl2_phi_apply", "arl2_device_status",
     "arl2_device_bytes", "arl2_kernel_launches", "arl2_state_update_noalloc", "arl2_destroy",
-    "arl2_status_string", "arl2_version",
+    "arl2_status_string", "arl2_version", "arl2_gates_apply", "arl2_frame_forward_hidden",
+    "arl2_frame_forward_hidden_host",
     "arl2_kv_create", "arl2_kv_frame_forward", "arl2_kv_frame_forward_host", "arl2_kv_reset",
     "arl2_kv_frames", "arl2_kv_cache_get", "arl2_kv_cache_set", "arl2_kv_device_status", "arl2_kv_device_bytes",
     "arl2_kv_cache_bytes", "arl2_kv_kernel_launches", "arl2_kv_destroy",
@@ -53,6 +54,7 @@ class Arl2Config(ctypes.Structure):
         ("w_q", ctypes.c_void_p), ("w_k", ctypes.c_void_p), ("w_v", ctypes.c_void_p),
         ("softmax_scale", ctypes.c_float), ("host_staging", ctypes.c_int), ("impl", ctypes.c_int),
         ("max_ctas", ctypes.c_int), ("gating", ctypes.c_int), ("access", ctypes.c_int),
+        ("hidden_dim", ctypes.c_int), ("w_gate", ctypes.c_void_p), ("b_gate", ctypes.c_void_p),
     ]
 
 
@@ -87,6 +89,9 @@ def _load() -> ctypes.CDLL:
         "arl2_destroy": ([H], None),
         "arl2_status_string": ([I], ctypes.c_char_p),
         "arl2_version": ([], I),
+        "arl2_gates_apply": ([H, P, P, P, P], I),
+        "arl2_frame_forward_hidden": ([H, P, P, P, P, I, P, P], I),
+        "arl2_frame_forward_hidden_host": ([H, P, P, P, P, I, P, P], I),
         "arl2_kv_create": ([ctypes.POINTER(Arl2KvConfig), P, ctypes.POINTER(H)], I),
         "arl2_kv_frame_forward": ([H, P, P, P, I, P, P], I),
         "arl2_kv_frame_forward_host": ([H, P, P, P, I, P, P], I),
@@ -160,7 +165,7 @@ class Arl2Layer:
     def __init__(self, batch: int, heads: int, head_dim: int, tokens: int, w_q, w_k, w_v, *,
                  dtype: torch.dtype = torch.bfloat16, softmax_scale: float = 0.0,
                  host_staging: bool = False, impl: str = "auto", max_ctas: int = 0,
-                 gating: str = "headwise", access: str = "frame", stream=None):
+                 gating: str = "headwise", access: str = "frame", gate_weights=None, stream=None):
         if dtype not in (torch.bfloat16, torch.float32):
             raise ValueError("dtype must be torch.bfloat16 or torch.float32")
         for w in (w_q, w_k, w_v):
@@ -171,13 +176,26 @@ class Arl2Layer:
         self.shape = (batch, tokens, heads, head_dim)
         self.dtype = dtype
         self.device = w_q.device
+        self.hidden_dim = 0
+        w_gate = b_gate = None
+        if gate_weights is not None:
+            w_gate, b_gate = gate_weights
+            if not (w_gate.is_cuda and w_gate.is_contiguous() and w_gate.dtype == dtype and w_gate.dim() == 2
+                    and w_gate.shape[1] == 2 * heads):
+                raise ValueError("gate weights must be a contiguous CUDA tensor [D, 2H] of the layer dtype")
+            if not (b_gate.is_cuda and b_gate.is_contiguous() and b_gate.dtype == torch.float32
+                    and tuple(b_gate.shape) == (2 * heads,)):
+                raise ValueError("gate bias must be a contiguous fp32 CUDA tensor [2H]")
+            self.hidden_dim = int(w_gate.shape[0])
         cfg = Arl2Config(batch, heads, head_dim, tokens,
                          ARL2_BF16 if dtype == torch.bfloat16 else ARL2_FP32,
                          w_q.data_ptr(), w_k.data_ptr(), w_v.data_ptr(), float(softmax_scale),
                          1 if host_staging else 0,
                          {"auto": ARL2_IMPL_AUTO, "simt": ARL2_IMPL_SIMT}[impl], int(max_ctas),
                          {"headwise": ARL2_GATE_HEADWISE, "elementwise": ARL2_GATE_ELEMENTWISE}[gating],
-                         {"frame": ARL2_ACCESS_FRAME, "token": ARL2_ACCESS_TOKEN}[access])
+                         {"frame": ARL2_ACCESS_FRAME, "token": ARL2_ACCESS_TOKEN}[access],
+                         self.hidden_dim, None if w_gate is None else w_gate.data_ptr(),
+                         None if b_gate is None else b_gate.data_ptr())
         self.token_level = access == "token"
         self.alpha_shape = lambda B, H: (B, H, head_dim) if gating == "elementwise" else (B, H)
         h = ctypes.c_void_p()
@@ -240,6 +258,54 @@ class Arl2Layer:
                                             _ptr(beta) if gates else None,
                                             1 if clean_pass else 0, _ptr(out), _stream(stream)),
                "arl2_frame_forward_host")
+        return out
+
+    def _hidden(self, x):
+        B, L, _, _ = self.shape
+        if not (x.is_cuda and x.is_contiguous() and x.dtype == self.dtype
+                and tuple(x.shape) == (B, L, self.hidden_dim)):
+            raise ValueError(f"x must be a contiguous CUDA tensor [B, L, D] = {[B, L, self.hidden_dim]}")
+        return x
+
+    def gates_apply(self, x, stream=None):
+        """arl2_gates_apply: (alpha [B, H], beta [B, H, L]) projected from the
+        hidden states x [B, L, D]."""
+        B, L, H, _ = self.shape
+        self._hidden(x)
+        alpha = torch.empty(B, H, dtype=torch.float32, device=self.device)
+        beta = torch.empty(B, H, L, dtype=torch.float32, device=self.device)
+        _check(_lib.arl2_gates_apply(self.handle, _ptr(x), _ptr(alpha), _ptr(beta), _stream(stream)),
+               "arl2_gates_apply")
+        return alpha, beta
+
+    def forward_hidden(self, q, k, v, x=None, clean_pass: bool = False, out=None, stream=None):
+        """One pass with the gates projected from x [B, L, D] (needed on the
+        clean pass, and on every pass with token-level access)."""
+        self._tok(q, "q"), self._tok(k, "k"), self._tok(v, "v")
+        if out is None:
+            out = torch.empty_like(q)
+        self._tok(out, "out")
+        if x is not None:
+            self._hidden(x)
+        elif clean_pass or self.token_level:
+            raise ValueError("this pass needs the hidden states x")
+        _check(_lib.arl2_frame_forward_hidden(self.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(x),
+                                              1 if clean_pass else 0, _ptr(out), _stream(stream)),
+               "arl2_frame_forward_hidden")
+        return out
+
+    def forward_hidden_host(self, q, k, v, x, clean_pass: bool, out, stream=None):
+        """arl2_frame_forward_hidden_host: q, k, v, x, out are host (pinned) tensors."""
+        B, L, _, _ = self.shape
+        for t in (q, k, v, out):
+            if t.is_cuda or not t.is_contiguous() or tuple(t.shape) != self.shape or t.dtype != self.dtype:
+                raise ValueError("host token tensors must be contiguous CPU tensors of the layer shape")
+        if x is not None and (x.is_cuda or not x.is_contiguous() or x.dtype != self.dtype
+                              or tuple(x.shape) != (B, L, self.hidden_dim)):
+            raise ValueError("x must be a contiguous CPU tensor [B, L, D] of the layer dtype")
+        _check(_lib.arl2_frame_forward_hidden_host(self.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(x),
+                                                   1 if clean_pass else 0, _ptr(out), _stream(stream)),
+               "arl2_frame_forward_hidden_host")
         return out
 
     def state_reset(self, stream=None) -> None:

@@ -63,6 +63,15 @@ struct arl2_handle {
     float* tl_ws = nullptr;   // token-level chunk workspace
     void* zero_read = nullptr;  // zero state for the intra-only attention launch
                                 // (bf16 Mt on the tensor-core path, fp32 S on SIMT)
+    // gate projections (optional): weights, and the gates they produce
+    int hidden = 0;             // D, 0 without projections
+    void* w_gate = nullptr;     // transposed: [gate_padded_outputs(H)][D] in dtype
+    float* b_gate = nullptr;    // [2H]
+    float* g_alpha = nullptr;   // [B][H]
+    float* g_beta = nullptr;    // [B][H][L]
+    float* g_part = nullptr;    // [B][gate_tiles(L)][H]
+    unsigned* g_count = nullptr;  // [B], zero between launches
+    void* stage_x = nullptr;    // host entry: staging of x [B][L][D]
     int* err = nullptr;       // device error word
     unsigned long long launches = 0;  // kernels enqueued by this handle
 };
@@ -101,7 +110,8 @@ void release(arl2_handle* h) {
     delete h->maps;
     void* ptrs[] = {h->w_all, h->S, h->Mt, h->Sb, h->part_s, h->attn_ws, h->qp, h->kp,
                     h->vp, h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], h->stage_tok[3],
-                    h->stage_alpha, h->stage_beta, h->err, h->tl_ws, h->zero_read};
+                    h->stage_alpha, h->stage_beta, h->err, h->tl_ws, h->zero_read,
+                    h->w_gate, h->b_gate, h->g_alpha, h->g_beta, h->g_part, h->g_count, h->stage_x};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     delete h;
@@ -147,7 +157,7 @@ arl2_status clean_update(arl2_handle* h, const void* k, const void* v, const flo
 
 extern "C" {
 
-int arl2_version(void) { return 10200; }
+int arl2_version(void) { return 10300; }
 
 const char* arl2_status_string(arl2_status s) {
     switch (s) {
@@ -181,6 +191,12 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
     if (!aligned16(cfg->w_q) || !aligned16(cfg->w_k) || !aligned16(cfg->w_v)) return ARL2_ERR_ALIGN;
     const bool use_tc = cfg->impl == ARL2_IMPL_AUTO && cfg->dtype == ARL2_BF16;
     if (use_tc && cfg->head_dim != 128) return ARL2_ERR_UNSUPPORTED;
+    if (cfg->w_gate) {
+        if (!cfg->b_gate) return ARL2_ERR_INVALID_ARG;
+        if (!arl2::gate_shape_ok(cfg->hidden_dim, cfg->heads)) return ARL2_ERR_SHAPE;
+        if (!aligned16(cfg->w_gate) || !aligned16(cfg->b_gate)) return ARL2_ERR_ALIGN;
+        if (cfg->gating != ARL2_GATE_HEADWISE) return ARL2_ERR_UNSUPPORTED;  // one alpha per head
+    }
 
     arl2_handle* h = new (std::nothrow) arl2_handle();
     if (!h) return ARL2_ERR_OOM;
@@ -230,7 +246,22 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
             s = dalloc(h, &h->stage_alpha, (size_t)dm.B * dm.H * (h->alpha_per_key ? dm.d : 1) * sizeof(float));
         if (s == ARL2_OK) s = dalloc(h, &h->stage_beta, (size_t)dm.B * dm.H * dm.L * sizeof(float));
     }
+    const size_t gate_w_bytes =
+        cfg->w_gate ? (size_t)cfg->hidden_dim * arl2::gate_padded_outputs(dm.H) * h->esz : 0;
+    if (s == ARL2_OK && cfg->w_gate) {
+        h->hidden = cfg->hidden_dim;
+        s = dalloc(h, &h->w_gate, gate_w_bytes);
+        if (s == ARL2_OK) s = dalloc(h, &h->b_gate, 2 * (size_t)dm.H * sizeof(float));
+        if (s == ARL2_OK) s = dalloc(h, &h->g_alpha, (size_t)dm.B * dm.H * sizeof(float));
+        if (s == ARL2_OK) s = dalloc(h, &h->g_beta, (size_t)dm.B * dm.H * dm.L * sizeof(float));
+        if (s == ARL2_OK)
+            s = dalloc(h, &h->g_part, (size_t)dm.B * arl2::gate_tiles(dm.L) * dm.H * sizeof(float));
+        if (s == ARL2_OK) s = dalloc(h, &h->g_count, (size_t)dm.B * sizeof(unsigned));
+        if (s == ARL2_OK && cfg->host_staging)
+            s = dalloc(h, &h->stage_x, (size_t)dm.B * dm.L * h->hidden * h->esz);
+    }
     if (s == ARL2_OK && arl2::simt_init() != cudaSuccess) s = ARL2_ERR_CUDA;
+    if (s == ARL2_OK && h->w_gate && arl2::gate_init() != cudaSuccess) s = ARL2_ERR_CUDA;
     if (s == ARL2_OK && use_tc) {
         h->maps = new (std::nothrow) arl2::TokenMapCache(dm);
         h->tc = arl2::attn_tc_create(dm, h->attn_ws, cfg->max_ctas);
@@ -248,6 +279,13 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
             s = ARL2_ERR_CUDA;
     if (s == ARL2_OK) s = zero_state(h, stream);
     if (s == ARL2_OK && cudaMemsetAsync(h->err, 0, sizeof(int), stream) != cudaSuccess)
+        s = ARL2_ERR_CUDA;
+    if (s == ARL2_OK && h->w_gate &&
+        (arl2::launch_gate_transpose(h->dtype == ARL2_BF16, cfg->w_gate, h->w_gate, h->hidden, dm.H, stream) !=
+             cudaSuccess ||
+         cudaMemcpyAsync(h->b_gate, cfg->b_gate, 2 * (size_t)dm.H * sizeof(float), cudaMemcpyDeviceToDevice,
+                         stream) != cudaSuccess ||
+         cudaMemsetAsync(h->g_count, 0, (size_t)dm.B * sizeof(unsigned), stream) != cudaSuccess))
         s = ARL2_ERR_CUDA;
     if (s == ARL2_OK && use_tc &&
         cudaMemsetAsync(h->attn_ws, 0, arl2::attn_tc_workspace_bytes(dm), stream) != cudaSuccess)
@@ -354,6 +392,55 @@ arl2_status arl2_frame_forward_host(arl2_handle* h, const void* q, const void* k
     }
     s = arl2_frame_forward(h, h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], a_dev, b_dev,
                            clean_pass, h->stage_tok[3], stream);
+    if (s != ARL2_OK) return s;
+    if (cudaMemcpyAsync(out, h->stage_tok[3], tb, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return ARL2_ERR_CUDA;
+    return ARL2_OK;
+}
+
+arl2_status arl2_gates_apply(arl2_handle* h, const void* x, float* alpha, float* beta, cudaStream_t stream) {
+    if (!h || !x || !alpha || !beta) return ARL2_ERR_INVALID_ARG;
+    if (!h->w_gate) return ARL2_ERR_INVALID_ARG;
+    if (!aligned16(x)) return ARL2_ERR_ALIGN;
+    arl2_status s = check_device(h);
+    if (s != ARL2_OK) return s;
+    const Dims& dm = h->dm;
+    ++h->launches;
+    if (arl2::launch_gate_proj(h->dtype == ARL2_BF16, x, h->w_gate, h->b_gate, dm.B, dm.L, h->hidden, dm.H, beta,
+                               h->g_part, alpha, h->g_count, stream) != cudaSuccess)
+        return ARL2_ERR_CUDA;
+    return ARL2_OK;
+}
+
+arl2_status arl2_frame_forward_hidden(arl2_handle* h, const void* q, const void* k, const void* v,
+                                      const void* x, int clean_pass, void* out, cudaStream_t stream) {
+    if (!h || !q || !k || !v || !out) return ARL2_ERR_INVALID_ARG;
+    if (!h->w_gate) return ARL2_ERR_INVALID_ARG;
+    const bool gates = clean_pass || h->token_level;  // the passes that read alpha and beta
+    if (!gates) return arl2_frame_forward(h, q, k, v, nullptr, nullptr, 0, out, stream);
+    arl2_status s = arl2_gates_apply(h, x, h->g_alpha, h->g_beta, stream);
+    if (s != ARL2_OK) return s;
+    return arl2_frame_forward(h, q, k, v, h->g_alpha, h->g_beta, clean_pass, out, stream);
+}
+
+arl2_status arl2_frame_forward_hidden_host(arl2_handle* h, const void* q, const void* k, const void* v,
+                                           const void* x, int clean_pass, void* out, cudaStream_t stream) {
+    if (!h || !q || !k || !v || !out) return ARL2_ERR_INVALID_ARG;
+    if (!h->stage_tok[0] || !h->w_gate) return ARL2_ERR_INVALID_ARG;
+    const bool gates = clean_pass || h->token_level;
+    if (gates && !x) return ARL2_ERR_INVALID_ARG;
+    arl2_status s = check_device(h);
+    if (s != ARL2_OK) return s;
+    const size_t tb = h->n_tok * h->esz;
+    const void* src[3] = {q, k, v};
+    for (int i = 0; i < 3; ++i)
+        if (cudaMemcpyAsync(h->stage_tok[i], src[i], tb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+            return ARL2_ERR_CUDA;
+    if (gates && cudaMemcpyAsync(h->stage_x, x, (size_t)h->dm.B * h->dm.L * h->hidden * h->esz,
+                                 cudaMemcpyHostToDevice, stream) != cudaSuccess)
+        return ARL2_ERR_CUDA;
+    s = arl2_frame_forward_hidden(h, h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], gates ? h->stage_x : nullptr,
+                                  clean_pass, h->stage_tok[3], stream);
     if (s != ARL2_OK) return s;
     if (cudaMemcpyAsync(out, h->stage_tok[3], tb, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
         return ARL2_ERR_CUDA;

@@ -77,3 +77,21 @@ cudaError_t launch_tl(const float* qp, const float* kp, const float* vp, const f
                       bool clean, Dims dm, cudaStream_t st);
 
 }  // namespace arl2
+
+namespace arl2 {
+
+// ---- gate projections (gates.cu) ----------------------------------------
+// alpha [B][H] and beta [B][H][L] from hidden states x [B][L][D] and the
+// transposed weights wt [gate_padded_outputs(H)][D] (launch_gate_transpose
+// of w [D][2H]; x, w in the layer dtype), bias fp32 [2H].  part_a: fp32
+// [B][gate_tiles(L)][H] scratch; count: [B] zeroed words (left zeroed).
+int gate_tiles(int L);
+bool gate_shape_ok(int D, int H);
+int gate_padded_outputs(int H);
+cudaError_t gate_init();  // kernel attributes, once (arl2_create)
+cudaError_t launch_gate_transpose(bool bf16, const void* w, void* wt, int D, int H, cudaStream_t st);
+cudaError_t launch_gate_proj(bool bf16, const void* x, const void* wt, const float* bias, int B, int L, int D,
+                             int H, float* beta, float* part_a, float* alpha, unsigned* count,
+                             cudaStream_t st);
+
+}  // namespace arl2

@@ -105,13 +105,23 @@ typedef struct {
                               with other work, tests of the split schedule)   */
     arl2_gating gating;    /* HEADWISE: alpha [B][H]; ELEMENTWISE: [B][H][d]  */
     arl2_access access;    /* FRAME (the method) or TOKEN (the ablation)      */
+    /* Optional gate projections (see arl2_frame_forward_hidden).  NULL w_gate:
+     * none, and hidden_dim, b_gate are ignored. */
+    int hidden_dim;        /* D: width of the hidden states; a multiple of 8;
+                              needs 2 H <= 96                                 */
+    const void* w_gate;    /* device [D][2H] in dtype, 16-byte aligned; column
+                              h gives head h's alpha logit, column H + h its
+                              beta logit; copied at create                    */
+    const float* b_gate;   /* device fp32 [2H], 16-byte aligned; copied       */
 } arl2_config;
 
 /* Create a layer on the current device.  Validates cfg, allocates the zeroed
  * state S_0 = 0 and every workspace, and copies the three feature maps
  * (stream-ordered on `stream`).  On success *out receives the handle.
- * Errors: INVALID_ARG (null cfg/out/weights), SHAPE, ALIGN (weights),
- * UNSUPPORTED (dtype/head_dim the chosen kernels do not handle), OOM, CUDA. */
+ * Errors: INVALID_ARG (null cfg/out/weights, w_gate without b_gate), SHAPE
+ * (also hidden_dim with w_gate), ALIGN (weights), UNSUPPORTED (dtype/head_dim
+ * the chosen kernels do not handle; gate projections with elementwise
+ * gating), OOM, CUDA. */
 arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle** out);
 
 /* One denoising pass of one latent frame (technical summary §2.1, §2.2).
@@ -136,6 +146,31 @@ arl2_status arl2_frame_forward(arl2_handle* h, const void* q, const void* k, con
 arl2_status arl2_frame_forward_host(arl2_handle* h, const void* q, const void* k, const void* v,
                                     const float* alpha, const float* beta, int clean_pass,
                                     void* out, cudaStream_t stream);
+
+/* Gate projections (technical summary §2.1 "State Update": alpha and beta
+ * are learned per-token projections; the pages give no form, and this is
+ * the reading the library takes).  For hidden states x (device [B][L][D] in
+ * dtype, 16-byte aligned; the input of the layer's QKV projection):
+ *   a_ih = x_i . w_gate[:, h] + b_gate[h],  g_ih = x_i . w_gate[:, H+h] + b_gate[H+h]
+ *   beta[b][h][i] = sigmoid(g_ih)
+ *   alpha[b][h]   = sigmoid((1/L) sum_i a_ih)   (one forget gate per frame)
+ * Writes alpha (device fp32 [B][H]) and beta (device fp32 [B][H][L]).
+ * Needs a handle created with w_gate (INVALID_ARG otherwise); fp32
+ * accumulation; one kernel. */
+arl2_status arl2_gates_apply(arl2_handle* h, const void* x, float* alpha, float* beta, cudaStream_t stream);
+
+/* arl2_frame_forward with the gates projected from the hidden states x
+ * (arl2_gates_apply into the handle's own buffers) on the passes that read
+ * them: the clean pass (and, with token-level access, every pass).  x may be
+ * NULL on other passes.  Needs a handle created with w_gate. */
+arl2_status arl2_frame_forward_hidden(arl2_handle* h, const void* q, const void* k, const void* v,
+                                      const void* x, int clean_pass, void* out, cudaStream_t stream);
+
+/* arl2_frame_forward_hidden on HOST buffers (q, k, v, out [B][L][H][d] and x
+ * [B][L][D], pinned for asynchronous copies), stream-ordered like
+ * arl2_frame_forward_host.  Needs host_staging and w_gate at create. */
+arl2_status arl2_frame_forward_hidden_host(arl2_handle* h, const void* q, const void* k, const void* v,
+                                           const void* x, int clean_pass, void* out, cudaStream_t stream);
 
 /* S := 0 for every stream and head (the start of a new video stream). */
 arl2_status arl2_state_reset(arl2_handle* h, cudaStream_t stream);

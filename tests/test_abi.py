@@ -39,7 +39,7 @@ def test_binding_covers_every_export():
 
 
 def test_version_and_status_strings():
-    assert arl2.version() == 10200
+    assert arl2.version() == 10300
     for code in range(0, -8, -1):
         s = arl2._lib.arl2_status_string(code).decode()
         assert s and s != "unknown status"
@@ -121,3 +121,25 @@ def test_teacher_layer_arguments_are_validated_before_cuda():
     assert lib.arl2_kv_cache_bytes(None) == 0
     assert lib.arl2_kv_kernel_launches(None) == 0
     lib.arl2_kv_destroy(None)
+
+
+def test_gate_projection_config_is_validated_before_cuda():
+    lib = arl2._lib
+    h = ctypes.c_void_p()
+    fake = 0x1000
+
+    def cfg(hidden, w_gate, b_gate, gating=arl2.ARL2_GATE_HEADWISE, heads=2):
+        return arl2.Arl2Config(1, heads, 16, 16, arl2.ARL2_FP32, fake, fake, fake, 0.0, 0, 0, 0, gating,
+                               arl2.ARL2_ACCESS_FRAME, hidden, w_gate, b_gate)
+
+    assert lib.arl2_create(ctypes.byref(cfg(32, fake, None)), None, ctypes.byref(h)) == -1  # no bias
+    for hidden in (0, 7, 12):
+        assert lib.arl2_create(ctypes.byref(cfg(hidden, fake, fake)), None, ctypes.byref(h)) == -2
+    assert lib.arl2_create(ctypes.byref(cfg(32, fake, fake, heads=49)), None, ctypes.byref(h)) == -2
+    assert lib.arl2_create(ctypes.byref(cfg(32, fake + 8, fake)), None, ctypes.byref(h)) == -3
+    assert lib.arl2_create(ctypes.byref(cfg(32, fake, fake + 4)), None, ctypes.byref(h)) == -3
+    assert lib.arl2_create(ctypes.byref(cfg(32, fake, fake, gating=arl2.ARL2_GATE_ELEMENTWISE)), None,
+                           ctypes.byref(h)) == -7
+    assert lib.arl2_gates_apply(None, None, None, None, None) == -1
+    assert lib.arl2_frame_forward_hidden(None, None, None, None, None, 1, None, None) == -1
+    assert lib.arl2_frame_forward_hidden_host(None, None, None, None, None, 1, None, None) == -1

@@ -15,6 +15,8 @@ Value recipe (identical for every workload, per stream b and layer l):
   alpha         = sigmoid(N(2, 0.5)), shape [B, H], one per frame
                   (elementwise gating: shape [B, H, d], same distribution)
   beta          = sigmoid(N(0, 1)) / L, shape [B, H, L], one per frame
+  (gate projections: hidden states x ~ N(0, 1) [B, L, H d] per frame,
+   w_gate ~ N(0, 1/(H d)) [H d, 2H], bias 2 (alpha) and -ln L (beta))
 Every tensor is rounded to the run's dtype (q, k, v and W) or kept fp32
 (alpha, beta); the same rounded values go to the GPU and to the oracle.
 
@@ -82,7 +84,7 @@ def stream_base(layer: int, stream: int) -> int:
     return SEED_BASE + 1000 * layer + stream
 
 
-_TAG_QKV, _TAG_GATES, _TAG_W, _TAG_GATES_ELEM = 1, 2, 3, 4
+_TAG_QKV, _TAG_GATES, _TAG_W, _TAG_GATES_ELEM, _TAG_HIDDEN, _TAG_W_GATE = 1, 2, 3, 4, 5, 6
 
 
 def _gen(*parts: int, device: str = "cpu") -> torch.Generator:
@@ -147,6 +149,36 @@ def frame_gates_elementwise(w: Workload, layer: int, frame: int):
         g = _gen(stream_base(layer, b), _TAG_GATES_ELEM, frame)
         alpha[b] = torch.sigmoid(2.0 + 0.5 * torch.randn(H, d, generator=g))
     return alpha.contiguous(), beta
+
+
+def hidden_dim(w: Workload) -> int:
+    """Width D of the hidden states the gate projections read: H d (the DiT's
+    model width, 1536 for 12 heads of 128)."""
+    return w.heads * w.head_dim
+
+
+def hidden_states(w: Workload, layer: int, frame: int, device: str = "cpu"):
+    """x [B, L, D] ~ N(0, 1) in w's dtype: the layer input the gate
+    projections read (one draw per frame: the clean pass's)."""
+    B, L, D = w.batch, w.tokens, hidden_dim(w)
+    x = torch.empty(B, L, D, dtype=torch.float32, device=device)
+    for b in range(B):
+        g = _gen(stream_base(layer, b), _TAG_HIDDEN, frame, device=device)
+        x[b] = torch.randn(L, D, generator=g, device=device)
+    return x.to(w.torch_dtype).contiguous()
+
+
+def gate_projection_weights(w: Workload, layer: int = 0):
+    """w_gate [D, 2H] ~ N(0, 1/D) in w's dtype (logits of unit variance for
+    x ~ N(0, 1)) and bias [2H] fp32: 2 for the alpha columns (alpha near
+    sigmoid(2), as in frame_gates) and -ln(L) for the beta columns (beta
+    near e^{N(0,1)} / L, the scale of frame_gates' sigmoid(N(0,1)) / L)."""
+    import math
+    H, D, L = w.heads, hidden_dim(w), w.tokens
+    g = _gen(stream_base(layer, 0), _TAG_W_GATE)
+    wg = (torch.randn(D, 2 * H, generator=g) / math.sqrt(D)).to(w.torch_dtype).contiguous()
+    bias = torch.tensor([2.0] * H + [-math.log(L)] * H, dtype=torch.float32)
+    return wg, bias
 
 
 def is_clean(w: Workload, pass_idx: int) -> bool:
