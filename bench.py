@@ -325,7 +325,7 @@ def profile_gates_case(args, w: workloads.Workload) -> int:
     wq, wk, wv = workloads.phi_weights(w, 0)
     wg, bg = workloads.gate_projection_weights(w, 0)
     lay = Arl2Layer(w.batch, w.heads, w.head_dim, w.tokens, wq.cuda(), wk.cuda(), wv.cuda(),
-                    dtype=w.torch_dtype, gate_weights=(wg.cuda(), bg.cuda()))
+                    dtype=w.torch_dtype, gate_weights=(wg.cuda(), bg.cuda()), impl=args.layer_impl)
     ring = 8
     xs = [workloads.hidden_states(w, 0, f, device="cuda") for f in range(ring)]
     for i in range(args.profile_gates):
@@ -566,6 +566,8 @@ def main():
                          "30-layer stacks built from them (one JSON line, not the headline)")
     ap.add_argument("--profile-gates", type=int, default=0,
                     help="profiling case of the gate projection: this many launches (no timing)")
+    ap.add_argument("--layer-impl", default="auto", choices=["auto", "simt"],
+                    help="kernels of the gate profiling case: tensor cores (bf16) or SIMT")
     ap.add_argument("--profile-teacher", type=int, default=0,
                     help="profiling case of the teacher layer with this many cached frames "
                          "(read-only passes as --profile-passes; no timing, no JSON line)")

@@ -72,6 +72,7 @@ struct arl2_handle {
     float* g_part = nullptr;    // [B][gate_tiles(L)][H]
     unsigned* g_count = nullptr;  // [B], zero between launches
     void* stage_x = nullptr;    // host entry: staging of x [B][L][D]
+    arl2::GateTc* gtc = nullptr;  // tensor-core gate projection (bf16), else the SIMT kernel
     int* err = nullptr;       // device error word
     unsigned long long launches = 0;  // kernels enqueued by this handle
 };
@@ -107,6 +108,7 @@ void release(arl2_handle* h) {
     if (!h) return;
     if (h->tc) arl2::attn_tc_destroy(h->tc);
     if (h->up) arl2::update_tc_destroy(h->up);
+    if (h->gtc) arl2::gate_tc_destroy(h->gtc);
     delete h->maps;
     void* ptrs[] = {h->w_all, h->S, h->Mt, h->Sb, h->part_s, h->attn_ws, h->qp, h->kp,
                     h->vp, h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], h->stage_tok[3],
@@ -255,13 +257,15 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
         if (s == ARL2_OK) s = dalloc(h, &h->g_alpha, (size_t)dm.B * dm.H * sizeof(float));
         if (s == ARL2_OK) s = dalloc(h, &h->g_beta, (size_t)dm.B * dm.H * dm.L * sizeof(float));
         if (s == ARL2_OK)
-            s = dalloc(h, &h->g_part, (size_t)dm.B * arl2::gate_tiles(dm.L) * dm.H * sizeof(float));
+            s = dalloc(h, &h->g_part, (size_t)dm.B * arl2::gate_part_count(dm.L) * dm.H * sizeof(float));
         if (s == ARL2_OK) s = dalloc(h, &h->g_count, (size_t)dm.B * sizeof(unsigned));
         if (s == ARL2_OK && cfg->host_staging)
             s = dalloc(h, &h->stage_x, (size_t)dm.B * dm.L * h->hidden * h->esz);
     }
     if (s == ARL2_OK && arl2::simt_init() != cudaSuccess) s = ARL2_ERR_CUDA;
     if (s == ARL2_OK && h->w_gate && arl2::gate_init() != cudaSuccess) s = ARL2_ERR_CUDA;
+    if (s == ARL2_OK && h->w_gate && use_tc)  // nullptr (shapes it does not take): the SIMT kernel
+        h->gtc = arl2::gate_tc_create(dm.B, dm.L, h->hidden, dm.H, h->w_gate, arl2::gate_padded_outputs(dm.H));
     if (s == ARL2_OK && use_tc) {
         h->maps = new (std::nothrow) arl2::TokenMapCache(dm);
         h->tc = arl2::attn_tc_create(dm, h->attn_ws, cfg->max_ctas);
@@ -406,9 +410,11 @@ arl2_status arl2_gates_apply(arl2_handle* h, const void* x, float* alpha, float*
     if (s != ARL2_OK) return s;
     const Dims& dm = h->dm;
     ++h->launches;
-    if (arl2::launch_gate_proj(h->dtype == ARL2_BF16, x, h->w_gate, h->b_gate, dm.B, dm.L, h->hidden, dm.H, beta,
-                               h->g_part, alpha, h->g_count, stream) != cudaSuccess)
-        return ARL2_ERR_CUDA;
+    const cudaError_t e =
+        h->gtc ? arl2::gate_tc_launch(h->gtc, x, h->b_gate, beta, h->g_part, alpha, h->g_count, h->err, stream)
+               : arl2::launch_gate_proj(h->dtype == ARL2_BF16, x, h->w_gate, h->b_gate, dm.B, dm.L, h->hidden, dm.H,
+                                        beta, h->g_part, alpha, h->g_count, stream);
+    if (e != cudaSuccess) return ARL2_ERR_CUDA;
     return ARL2_OK;
 }
 

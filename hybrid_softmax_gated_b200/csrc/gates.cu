@@ -267,7 +267,12 @@ int gate_tiles(int L) { return (L + kGTok - 1) / kGTok; }
 
 bool gate_shape_ok(int D, int H) { return D >= 8 && D % 8 == 0 && H >= 1 && 2 * H <= 8 * kGMaxU; }
 
-int gate_padded_outputs(int H) { return 8 * pick_u(H); }
+int gate_padded_outputs(int H) {
+    // rows of the transposed weights: the SIMT tile's 8U, and the 32-row
+    // multiple the tensor-core kernel reads (both zero past 2H)
+    const int simt = 8 * pick_u(H), tc = gate_tc_outputs(H);
+    return simt > tc ? simt : tc;
+}
 
 cudaError_t launch_gate_transpose(bool bf16, const void* w, void* wt, int D, int H, cudaStream_t st) {
     const int O = 2 * H, Opad = gate_padded_outputs(H);

@@ -94,4 +94,15 @@ cudaError_t launch_gate_proj(bool bf16, const void* x, const void* wt, const flo
                              int H, float* beta, float* part_a, float* alpha, unsigned* count,
                              cudaStream_t st);
 
+// The tensor-core form for bf16 (gates_tc.cu): wt as above, wt_rows rows.
+struct GateTc;
+int gate_tc_outputs(int H);  // padded outputs N of its products: 32, 64 or 96
+// alpha-logit partials per stream that either kernel writes (part_a holds
+// B * gate_part_count(L) * H floats)
+int gate_part_count(int L);
+GateTc* gate_tc_create(int B, int L, int D, int H, const void* wt, int wt_rows);  // nullptr: not usable
+void gate_tc_destroy(GateTc* g);
+cudaError_t gate_tc_launch(GateTc* g, const void* x, const float* bias, float* beta, float* part_a, float* alpha,
+                           unsigned* count, int* err, cudaStream_t st);
+
 }  // namespace arl2

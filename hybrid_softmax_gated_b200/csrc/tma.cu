@@ -57,6 +57,17 @@ bool tma_encode_token_rows(CUtensorMap* m, const void* p, int B, int H, int rows
     return encode4(m, p, dims, strides, box);
 }
 
+bool tma_encode_rows_2d(CUtensorMap* m, const void* p, long long inner, long long rows, long long outer,
+                        int box_rows) {
+    if (inner < 64 || (inner * 2) % 16 != 0 || rows < 1 || outer < 1 || box_rows < 1 || box_rows > 256)
+        return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)outer, 1};
+    const cuuint64_t strides[3] = {(cuuint64_t)inner * 2, (cuuint64_t)(inner * 2 * rows),
+                                   (cuuint64_t)(inner * 2 * rows * outer)};
+    const cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
+    return encode4(m, p, dims, strides, box);
+}
+
 bool tma_encode_tiles(CUtensorMap* m, const void* p, int outer) {
     const cuuint64_t dims[4] = {128, 128, (cuuint64_t)outer, 1};
     const cuuint64_t strides[3] = {128 * 2, 128 * 128 * 2, (cuuint64_t)outer * 128 * 128 * 2};

@@ -22,6 +22,12 @@ bool tma_encode_tokens(CUtensorMap* m, const void* p, const Dims& dm);
 // `rows` read as zeros.
 bool tma_encode_token_rows(CUtensorMap* m, const void* p, int B, int H, int rows, long long capacity);
 
+// Row-major bf16 matrices [outer][rows][inner] (inner contiguous, a
+// multiple of 8 elements): dims {inner, rows, outer, 1}; box {64, box_rows,
+// 1, 1}, rows past the end read as zeros.
+bool tma_encode_rows_2d(CUtensorMap* m, const void* p, long long inner, long long rows, long long outer,
+                        int box_rows);
+
 // Square bf16 tiles [outer][128][128] (outer = H or B*H flattened, the
 // innermost dimension contiguous): dims {128, 128, outer}; box {64, 128, 1}.
 bool tma_encode_tiles(CUtensorMap* m, const void* p, int outer);

@@ -35,12 +35,18 @@ def make(w, **kw):
     return lay, (wq, wk, wv), (wg, bg)
 
 
-@pytest.mark.parametrize("w", [BASE, small(17), small(100, B=3, H=5), workloads.WORKLOADS["tiny_fp32"],
-                               dataclasses.replace(workloads.WORKLOADS["tiny_fp32"], heads=40, head_dim=24,
-                                                   tokens=33, batch=2)],
-                         ids=["480p", "L17", "L100_B3_H5", "tiny_fp32", "fp32_H40"])
-def test_gates_apply_matches_oracle(w):
-    lay, _, (wg, bg) = make(w, impl="simt" if w.dtype == "fp32" else "auto")
+@pytest.mark.parametrize("w,impl", [
+    (BASE, "auto"), (small(17), "auto"), (small(100, B=3, H=5), "auto"), (small(300, B=2, H=20), "auto"),
+    (small(260, B=2, H=40), "auto"), (BASE, "simt"), (small(100, B=3, H=5), "simt"),
+    (workloads.WORKLOADS["tiny_fp32"], "simt"),
+    (dataclasses.replace(workloads.WORKLOADS["tiny_fp32"], heads=40, head_dim=24, tokens=33, batch=2), "simt")],
+    ids=["480p_tc", "L17_tc", "L100_B3_H5_tc", "L300_H20_tc", "L260_H40_tc", "480p_simt", "L100_simt",
+         "tiny_fp32", "fp32_H40"])
+def test_gates_apply_matches_oracle(w, impl):
+    # bf16 layers on the default path use the tensor-core kernel (2H padded
+    # to 32, 64 or 96 outputs; the hidden features split over a cluster),
+    # impl="simt" and fp32 layers the SIMT kernel
+    lay, _, (wg, bg) = make(w, impl=impl)
     try:
         for f in range(2):
             x = workloads.hidden_states(w, 0, f)
