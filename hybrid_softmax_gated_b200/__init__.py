@@ -39,7 +39,7 @@ EXPORTED = (
     "arl2_state_get", "arl2_state_set", "arl2_phi_apply", "arl2_device_status",
     "arl2_device_bytes", "arl2_kernel_launches", "arl2_state_update_noalloc", "arl2_destroy",
     "arl2_status_string", "arl2_version", "arl2_gates_apply", "arl2_frame_forward_hidden",
-    "arl2_frame_forward_hidden_host",
+    "arl2_frame_forward_hidden_host", "arl2_selftest_wait_timeout",
     "arl2_kv_create", "arl2_kv_frame_forward", "arl2_kv_frame_forward_host", "arl2_kv_reset",
     "arl2_kv_frames", "arl2_kv_cache_get", "arl2_kv_cache_set", "arl2_kv_device_status", "arl2_kv_device_bytes",
     "arl2_kv_cache_bytes", "arl2_kv_kernel_launches", "arl2_kv_destroy",
@@ -92,6 +92,7 @@ def _load() -> ctypes.CDLL:
         "arl2_gates_apply": ([H, P, P, P, P], I),
         "arl2_frame_forward_hidden": ([H, P, P, P, P, I, P, P], I),
         "arl2_frame_forward_hidden_host": ([H, P, P, P, P, I, P, P], I),
+        "arl2_selftest_wait_timeout": ([H, ctypes.c_uint, P], I),
         "arl2_kv_create": ([ctypes.POINTER(Arl2KvConfig), P, ctypes.POINTER(H)], I),
         "arl2_kv_frame_forward": ([H, P, P, P, I, P, P], I),
         "arl2_kv_frame_forward_host": ([H, P, P, P, I, P, P], I),
@@ -334,6 +335,12 @@ class Arl2Layer:
         _check(_lib.arl2_phi_apply(self.handle, {"q": 0, "k": 1, "v": 2}[which], _ptr(x), _ptr(out),
                                    _stream(stream)), "arl2_phi_apply")
         return out
+
+    def selftest_wait_timeout(self, limit_us: int, stream=None) -> None:
+        """arl2_selftest_wait_timeout: a bounded wait on a word nothing sets,
+        which gives up after limit_us and sets the error word."""
+        _check(_lib.arl2_selftest_wait_timeout(self.handle, int(limit_us), _stream(stream)),
+               "arl2_selftest_wait_timeout")
 
     def device_status(self, stream=None) -> int:
         """Synchronise and return the device status code (0, or ARL2_ERR_TIMEOUT)."""

@@ -73,6 +73,7 @@ struct arl2_handle {
     unsigned* g_count = nullptr;  // [B], zero between launches
     void* stage_x = nullptr;    // host entry: staging of x [B][L][D]
     arl2::GateTc* gtc = nullptr;  // tensor-core gate projection (bf16), else the SIMT kernel
+    int* quiet = nullptr;       // a zero word nothing ever sets (the failure-path self-test)
     int* err = nullptr;       // device error word
     unsigned long long launches = 0;  // kernels enqueued by this handle
 };
@@ -113,7 +114,8 @@ void release(arl2_handle* h) {
     void* ptrs[] = {h->w_all, h->S, h->Mt, h->Sb, h->part_s, h->attn_ws, h->qp, h->kp,
                     h->vp, h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], h->stage_tok[3],
                     h->stage_alpha, h->stage_beta, h->err, h->tl_ws, h->zero_read,
-                    h->w_gate, h->b_gate, h->g_alpha, h->g_beta, h->g_part, h->g_count, h->stage_x};
+                    h->w_gate, h->b_gate, h->g_alpha, h->g_beta, h->g_part, h->g_count, h->stage_x,
+                    h->quiet};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     delete h;
@@ -225,6 +227,7 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
         s = dalloc(h, &h->S, h->n_state * sizeof(float));
     }
     if (s == ARL2_OK) s = dalloc(h, &h->err, sizeof(int));
+    if (s == ARL2_OK) s = dalloc(h, &h->quiet, sizeof(int));
     if (use_tc) {
         const size_t parts = (size_t)dm.B * dm.H * arl2::update_tc_chunks(dm) * dm.d * dm.d;
         if (s == ARL2_OK) s = dalloc(h, &h->Mt, h->n_state * 2);
@@ -282,7 +285,8 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
         if (cudaMemcpyAsync(h->w[i], src[i], wbytes, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
             s = ARL2_ERR_CUDA;
     if (s == ARL2_OK) s = zero_state(h, stream);
-    if (s == ARL2_OK && cudaMemsetAsync(h->err, 0, sizeof(int), stream) != cudaSuccess)
+    if (s == ARL2_OK && (cudaMemsetAsync(h->err, 0, sizeof(int), stream) != cudaSuccess ||
+                         cudaMemsetAsync(h->quiet, 0, sizeof(int), stream) != cudaSuccess))
         s = ARL2_ERR_CUDA;
     if (s == ARL2_OK && h->w_gate &&
         (arl2::launch_gate_transpose(h->dtype == ARL2_BF16, cfg->w_gate, h->w_gate, h->hidden, dm.H, stream) !=
@@ -513,6 +517,16 @@ arl2_status arl2_device_status(arl2_handle* h, cudaStream_t stream) {
         }
         return ARL2_ERR_TIMEOUT;
     }
+    return ARL2_OK;
+}
+
+arl2_status arl2_selftest_wait_timeout(arl2_handle* h, unsigned limit_us, cudaStream_t stream) {
+    if (!h || limit_us == 0 || limit_us > 1000000u) return ARL2_ERR_INVALID_ARG;
+    arl2_status s = check_device(h);
+    if (s != ARL2_OK) return s;
+    ++h->launches;
+    if (arl2::launch_selftest_wait(h->quiet, (unsigned long long)limit_us * 1000ull, h->err, stream) != cudaSuccess)
+        return ARL2_ERR_CUDA;
     return ARL2_OK;
 }
 

@@ -21,6 +21,12 @@ enum : int {
     kErrTimeoutUpdate = 1 << 1,
 };
 
+// ---- failure path self-test (simt.cu) -------------------------------------
+// One thread waits for *flag to become nonzero with the same bounded spin
+// the kernels' inter-CTA waits use; after limit_ns it sets kErrTimeoutAttn
+// in *err and returns.
+cudaError_t launch_selftest_wait(const int* flag, unsigned long long limit_ns, int* err, cudaStream_t st);
+
 // ---- SIMT kernels (fp32 arithmetic; T = float or __nv_bfloat16) ----------
 
 // One-time kernel attribute setup (dynamic shared memory limits); called by

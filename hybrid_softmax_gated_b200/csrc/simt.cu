@@ -350,6 +350,28 @@ cudaError_t launch_phi_simt(bool bf16, const void* x, const void* w, bool l2norm
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------ self-test ----
+__global__ void selftest_wait_kernel(const int* __restrict__ flag, unsigned long long limit_ns, int* err) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    unsigned long long t0, t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    while (true) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v != 0) return;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (t - t0 > limit_ns) {
+            atomicOr(err, kErrTimeoutAttn);
+            return;
+        }
+    }
+}
+
+cudaError_t launch_selftest_wait(const int* flag, unsigned long long limit_ns, int* err, cudaStream_t st) {
+    selftest_wait_kernel<<<1, 32, 0, st>>>(flag, limit_ns, err);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_attn_simt_cached(bool bf16, const void* q, const void* k, const void* v,
                                     const void* kc, const void* vc, int Lc, long long cap,
                                     const float* qp, const float* S, void* out, float scale, Dims dm,

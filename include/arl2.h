@@ -195,6 +195,13 @@ arl2_status arl2_phi_apply(arl2_handle* h, int which, const void* x, void* out,
  * else ARL2_OK.  This is the one call that blocks the host. */
 arl2_status arl2_device_status(arl2_handle* h, cudaStream_t stream);
 
+/* Self-test of the failure path: one thread waits, with the bounded spin
+ * the kernels' inter-CTA waits use, for a device word that nothing ever
+ * sets; after limit_us (1 .. 1,000,000) it gives up, sets the handle's error
+ * word and returns.  arl2_device_status then reports ARL2_ERR_TIMEOUT and
+ * clears it; the context stays usable.  No fault, trap or unbounded wait. */
+arl2_status arl2_selftest_wait_timeout(arl2_handle* h, unsigned limit_us, cudaStream_t stream);
+
 /* Device bytes the handle holds (state, copies, weights, workspaces). */
 size_t arl2_device_bytes(const arl2_handle* h);
 

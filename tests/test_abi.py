@@ -59,6 +59,7 @@ def test_null_arguments_are_rejected_before_any_cuda_call():
     assert lib.arl2_state_set(None, None, None) == -1
     assert lib.arl2_phi_apply(None, 0, None, None, None) == -1
     assert lib.arl2_device_status(None, None) == -1
+    assert lib.arl2_selftest_wait_timeout(None, 1000, None) == -1
     assert lib.arl2_device_bytes(None) == 0
     assert lib.arl2_kernel_launches(None) == 0
     lib.arl2_destroy(None)
