@@ -108,7 +108,9 @@ class ClockSampler:
         try:
             uuid = str(torch.cuda.get_device_properties(device).uuid)
             ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
-            out_dir = os.path.join(ROOT, "gpurun_out") if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else "/tmp"
+            # the raw samples: ARL2_CLOCK_LOG_DIR if set (to keep them), else the temp dir
+            import tempfile
+            out_dir = os.environ.get("ARL2_CLOCK_LOG_DIR") or tempfile.gettempdir()
             self.path = os.path.join(out_dir, f"clocks_{os.getpid()}.csv")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", ident, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
