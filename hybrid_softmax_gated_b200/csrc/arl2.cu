@@ -45,7 +45,7 @@ struct arl2_handle {
     // tensor-core path (both copies are functions of S alone)
     void* Mt = nullptr;       // bf16 (W_q S)^T, read by the attention kernel
     void* Sb = nullptr;       // bf16 S, read by the update kernel
-    float* part_s = nullptr;  // fp32 update partials [B][H][chunks][d][d]
+    float* part_s = nullptr;  // fp32 update partials [B][H][chunks], d x d each
     void* attn_ws = nullptr;  // attention split-tile partials and flags
     arl2::TokenMapCache* maps = nullptr;
     arl2::AttnTc* tc = nullptr;

@@ -20,7 +20,7 @@ struct UpdateBuffers {
     float* S;           // fp32 [B][H][128][128] master state, row = key feature
     void* Sb;           // bf16 copy of S (read by the next update)
     void* Mt;           // bf16 (W_q S)^T (read by the attention kernel)
-    float* part_s;      // fp32 [B][H][chunks][128][128] workspace
+    float* part_s;      // fp32 [B][H][chunks] blocks of 128 x 128, in column quads
 };
 
 int update_tc_chunks(const Dims& dm);
