@@ -162,7 +162,8 @@ struct __align__(1024) Smem {
     // next S needs the P V of its previous block issued, so neither barrier
     // runs more than one phase ahead of its waiter.
     uint64_t s_full[2];  // one commit: S of the buffer's block is in TMEM
-    uint64_t p_full[2];  // 4 warp arrivals: P written over S (and O_b rescaled)
+    uint64_t p_half[2];  // 4 warp arrivals: P of the block's first 64 keys written (O_b rescaled)
+    uint64_t p_full[2];  // 4 warp arrivals: P of the other 64 keys written
     uint64_t drain;      // the issuer's last commit before it gives up after a failed wait
     uint64_t o_free;     // 8 warp arrivals per segment: O_0, O_1 and O_inter read out
     uint64_t ebar;       // 8 warp arrivals: epilogue exchange of row maxima and sums
@@ -225,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(ptx::smem_u32(&sm.v_full[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sm.v_empty[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sm.s_full[s]), 1);
+            ptx::mbar_init(ptx::smem_u32(&sm.p_half[s]), kWgWarps);
             ptx::mbar_init(ptx::smem_u32(&sm.p_full[s]), kWgWarps);
             ptx::mbar_init(ptx::smem_u32(&sm.stage_free[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sm.staged[s]), kSoftmaxWarps);
@@ -245,10 +247,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    // The next kernel may launch now and run its own set-up.  Nothing of this
-    // kernel touches global memory before the previous kernel has finished:
-    // every role starts with that wait (griddepcontrol.wait).
-    ptx::pdl_trigger();
+    // Nothing of this kernel touches global memory before the previous kernel
+    // has finished: every role starts with that wait (griddepcontrol.wait),
+    // and only then lets the next kernel launch, so that the state update
+    // that follows a clean pass may load the pass's inputs before its own
+    // wait.
 
     auto fail = [&]() {
         atomicOr(err, kErrTimeoutAttn);
@@ -266,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // (the whole warp runs the producer; one elected lane issues)
         // ------------------------------------------------ TMA producer --
-        ptx::pdl_wait();
+        ptx::pdl_wait_then_trigger();
         ptx::tma_prefetch_desc(&tm_q);
         ptx::tma_prefetch_desc(&tm_k);
         ptx::tma_prefetch_desc(&tm_v);
@@ -365,12 +368,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // (the whole warp runs the issuer; one elected lane issues)
         // ------------------------------------------------- UMMA issuer --
-        ptx::pdl_wait();
+        ptx::pdl_wait_then_trigger();
         const uint32_t idesc_pv = ptx::idesc_bf16_f32(kBM, kD, false, true);  // V: MN-major
         const uint32_t idesc_qm = ptx::idesc_bf16_f32(kBM, kD, false, false);
         int kc = 0, vc = 0;
         int vb = 0;           // virtual blocks so far: block vb + j of a segment uses buffer (vb + j) & 1
-        uint32_t p_par = 0;   // bit b: phase parity of p_full[b] to wait for
+        uint32_t p_par = 0;   // bit b: phase parity of p_half[b] and p_full[b] to wait for
         int prev_oi_buf = -1; // buffer holding the previous segment's O_inter
         bool ok = true;
         int si = 0;
@@ -424,8 +427,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; ok && j < n; ++j) {
                 const int buf = (vb + j) & 1;
                 const int vs = vc & 1;
-                ok = wwait(&sm.p_full[buf], (p_par >> buf) & 1) && wwait(&sm.v_full[vs], (vc >> 1) & 1);
+                const uint32_t par = (p_par >> buf) & 1;
                 p_par ^= 1u << buf;
+                ok = wwait(&sm.p_half[buf], par) && wwait(&sm.v_full[vs], (vc >> 1) & 1);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 const int ksteps = (block_keys(nc, L, Lc, sg.kv0 + j) + 15) >> 4;
@@ -433,14 +437,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t o_t = tmem + kColO + (uint32_t)buf * kD;
                 const uint32_t v_s = ptx::smem_u32(sm.v[vs]);
                 const uint32_t acc0 = j >= 2 ? 1u : 0u;
-                // O_b += P V, P from TMEM.  A full block is one short issue
-                // sequence (the issue rate of a single warp bounds the tensor pipe).
-                if (ksteps == kBN / 16) {
-                    ptx::umma_ts8_mn(o_t, p_t, mnmajor_desc(v_s, 0), idesc_pv, acc0);
+                // O_b += P V, P from TMEM, in two halves of 64 keys: the first
+                // runs while the softmax warps compute the second half's P.
+                // A full half is one short issue sequence (the issue rate of a
+                // single warp bounds the tensor pipe).
+                const int k_half = ksteps < 4 ? ksteps : 4;
+                if (k_half == 4) {
+                    ptx::umma_ts4_mn(o_t, p_t, mnmajor_desc(v_s, 0), idesc_pv, acc0);
                 } else {
-                    for (int kk = 0; kk < ksteps; ++kk)
+                    for (int kk = 0; kk < k_half; ++kk)
                         ptx::umma_f16_ts_w(o_t, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv,
                                            kk > 0 ? 1u : acc0);
+                }
+                ok = wwait(&sm.p_full[buf], par);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                if (ksteps == kBN / 16) {
+                    ptx::umma_ts4_mn(o_t, p_t + 32u, mnmajor_desc(v_s, 4), idesc_pv, 1u);
+                } else {
+                    for (int kk = 4; kk < ksteps; ++kk)
+                        ptx::umma_f16_ts_w(o_t, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv, 1u);
                 }
                 ptx::umma_commit_w(ptx::smem_u32(&sm.v_empty[vs]));
                 ++vc;
@@ -457,6 +473,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::umma_commit_w(ptx::smem_u32(&sm.drain));
             ptx::mbar_wait_bounded(ptx::smem_u32(&sm.drain), 0, &no_abort, kWaitLimitNs);
         }
+    } else if (warp == 2) {
+        // the TMEM allocator has no role in between; it triggers like the others
+        ptx::pdl_wait_then_trigger();
     } else if (warp == 3) {
         // ------------------------------------------- epilogue helper --
         if (lane == 0 && rng.n_segs > 0) {
@@ -478,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-        ptx::pdl_wait();
+        ptx::pdl_wait_then_trigger();
         bool ok = true;
         for (int si = 0; ok && si < rng.n_segs; ++si) {
             const Seg sg = seg_at(sch, rng, si);
@@ -521,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= 4) {
         // ---------------------------------------- softmax + epilogue --
         ptx::setmaxnreg_inc<kRegsHigh>();
-        ptx::pdl_wait();
+        ptx::pdl_wait_then_trigger();
         const int wg = (warp - 4) >> 2;               // S/P buffer, O accumulator and key blocks
         const int row = ((warp & 3) << 5) + lane;     // tile row = TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -592,43 +611,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float2 nm = make_float2(-m_use, -m_use);
                 float2 sum4[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
                 uint32_t pk[64];
+                // P (bf16 pairs) over the first 64 columns of the S buffer, in
+                // two halves of 64 keys, each handed to the issuer when stored
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    // SFU exponentials, with kPolyPairEvery > 0 a share on the FMA pipe
-                    const float2 a = ptx::fma2(make_float2(x[2 * i], x[2 * i + 1]), sl2, nm);
-                    float2 p;
-                    if (poly_pair(i)) {
-                        p = ptx::exp2_fma2(a);
-                    } else {
-                        p.x = ptx::ex2(a.x);
-                        p.y = ptx::ex2(a.y);
+                for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+                    for (int i = 32 * hf; i < 32 * hf + 32; ++i) {
+                        // SFU exponentials, with kPolyPairEvery > 0 a share on the FMA pipe
+                        const float2 a = ptx::fma2(make_float2(x[2 * i], x[2 * i + 1]), sl2, nm);
+                        float2 p;
+                        if (poly_pair(i)) {
+                            p = ptx::exp2_fma2(a);
+                        } else {
+                            p.x = ptx::ex2(a.x);
+                            p.y = ptx::ex2(a.y);
+                        }
+                        sum4[i & 3] = ptx::add2(sum4[i & 3], p);
+                        pk[i] = ptx::pack_bf16x2(p.x, p.y);
                     }
-                    sum4[i & 3] = ptx::add2(sum4[i & 3], p);
-                    pk[i] = ptx::pack_bf16x2(p.x, p.y);
+                    if (hf == 0 && j >= 2 && __any_sync(0xffffffffu, need)) {
+                        // rescale O_wg before the first half's P V adds to it
+                        // (after that half's exponentials, when fewer of S's
+                        // registers are live): S of this block was committed
+                        // after the P V of this warpgroup's previous block, so
+                        // that is done
+#pragma unroll 1
+                        for (int c = 0; c < 4; ++c) {
+                            uint32_t o[32];
+                            ptx::tmem_ld32(obuf + (uint32_t)c * 32, o);
+                            ptx::tmem_wait_ld();
+                            ptx::reg_fence(o);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+                            ptx::tmem_st32(obuf + (uint32_t)c * 32, o);
+                        }
+                    }
+                    ptx::tmem_st32_u(sbuf + 32u * hf, pk + 32 * hf);
+                    ptx::tmem_wait_st();
+                    ptx::tc_fence_before();
+                    warp_arrive(hf == 0 ? &sm.p_half[wg] : &sm.p_full[wg]);
                 }
                 const float2 s2 = ptx::add2(ptx::add2(sum4[0], sum4[1]), ptx::add2(sum4[2], sum4[3]));
                 l_run = l_run * corr + (s2.x + s2.y);
                 m_run = m_use;
-                // P (bf16 pairs) over the first 64 columns of the S buffer
-                ptx::tmem_st32_u(sbuf, pk);
-                ptx::tmem_st32_u(sbuf + 32, pk + 32);
-                if (j >= 2 && __any_sync(0xffffffffu, need)) {
-                    // rescale O_wg: S of this block was committed after the
-                    // P V of this warpgroup's previous block, so that is done
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        ptx::tmem_ld32(obuf + (uint32_t)c * 32, o);
-                        ptx::tmem_wait_ld();
-                        ptx::reg_fence(o);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
-                        ptx::tmem_st32(obuf + (uint32_t)c * 32, o);
-                    }
-                }
-                ptx::tmem_wait_st();
-                ptx::tc_fence_before();
-                warp_arrive(&sm.p_full[wg]);
             }
             if (!ok) break;
             // ------------------------------------------------ epilogue --
@@ -675,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float4* pbase = reinterpret_cast<float4*>(part_o) + ((size_t)sg.tile * 2 + wg) * 16 * kBM + row;
             if (sg.kind == kHead) {
                 // unnormalised O, running max and row sum -> partial, then the flag
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < 2; ++c) {
                     float acc[32];
                     uint32_t unused[32];
@@ -706,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const uint32_t stage = ptx::smem_u32(sm.q[si & 1]);  // the segment's Q slot
                 const uint32_t oi_col = tmem + lane_base + kColS + (uint32_t)((vb + n) & 1) * kBN + (uint32_t)wg * 64;
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < 2; ++c) {
                     float acc[32];
                     uint32_t oi[32];

@@ -293,6 +293,14 @@ __device__ __forceinline__ void pdl_trigger() {
 __device__ __forceinline__ void pdl_wait() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
+// Wait for the previous kernel, then let the next one launch.  A kernel that
+// triggers only after its wait never has a dependent running beside anything
+// older than itself: a dependent that reads its own inputs before its wait
+// (inputs no kernel of this chain writes) then sees them complete.
+__device__ __forceinline__ void pdl_wait_then_trigger() {
+    pdl_wait();
+    pdl_trigger();
+}
 
 // ---- register reallocation between warpgroups ------------------------------
 // Every warp of a warpgroup executes the same one.  The increases of a CTA
@@ -491,6 +499,27 @@ __device__ __forceinline__ void umma_ss8_kk(uint32_t d_tmem, uint64_t a0, uint64
         "add.u32 x, %1, 1030;\n\tadd.u32 y, %3, 1030;\n\tmov.b64 a, {x, %2};\n\tmov.b64 b, {y, %4};\n\t"
         "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, one;\n\t}" ::"r"(d_tmem),
         "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "r"(idesc), "r"(acc0)
+        : "memory");
+}
+// A from TMEM (a_tmem, 8 columns of bf16 pairs per k-step), B MN-major:
+// four k-steps (64 deep), for a product issued in two halves.
+__device__ __forceinline__ void umma_ts4_mn(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0, uint32_t idesc,
+                                            uint32_t acc0) {
+    const uint32_t blo = (uint32_t)b0, bhi = (uint32_t)(b0 >> 32);
+    asm volatile(
+        "{\n\t.reg .pred e, p, one;\n\t.reg .b64 b;\n\t.reg .b32 t, y;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "setp.eq.b32 one, %5, %5;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "mov.b64 b, {%2, %3};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b, %4, p;\n\t"
+        "add.u32 t, %1, 8;\n\tadd.u32 y, %2, 128;\n\tmov.b64 b, {y, %3};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, one;\n\t"
+        "add.u32 t, %1, 16;\n\tadd.u32 y, %2, 256;\n\tmov.b64 b, {y, %3};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, one;\n\t"
+        "add.u32 t, %1, 24;\n\tadd.u32 y, %2, 384;\n\tmov.b64 b, {y, %3};\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, one;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(blo), "r"(bhi), "r"(idesc), "r"(acc0)
         : "memory");
 }
 // A from TMEM (a_tmem, 8 columns of bf16 pairs per k-step), B MN-major.

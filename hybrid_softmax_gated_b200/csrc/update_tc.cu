@@ -115,12 +115,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    // Set-up done: let the next kernel launch.  Only the producer waits for
-    // the previous kernel, and only before loading S_{N-1}: K, V, beta and
-    // the feature maps are never written by the kernels this one may overlap
-    // (the attention pass before it reads them too), so the projections and
-    // K' run while that kernel drains.  Everything this kernel writes comes
-    // after S_{N-1} has landed, i.e. after the wait.
+    // Set-up done: let the next kernel launch.  This kernel always follows
+    // the clean pass's attention kernel, which lets it launch only after its
+    // own wait: everything older than that kernel is complete, and that
+    // kernel writes none of K, V, beta or the feature maps.  So only the
+    // producer waits, and only before loading S_{N-1}; the projections and
+    // K' run while the attention kernel drains.  Everything this kernel
+    // writes comes after S_{N-1} has landed, i.e. after the wait.
     ptx::pdl_trigger();
     auto fail = [&]() {
         atomicOr(err, kErrTimeoutUpdate);
@@ -233,28 +234,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t xk = ptx::smem_u32(sm.xk[c]), xv = ptx::smem_u32(sm.xv[c]);
         bool ok = wwait(&sm.proj[c]);
         if (ok) {
-            // K' = Kp / max(|Kp|, 1e-6) -> bf16 into xk (the K tile is consumed)
+            // K' = Kp / max(|Kp|, 1e-6) -> bf16 into xk (the K tile is consumed).
+            // The loops over 32-column chunks stay rolled: this code runs once
+            // per launch, and every unrolled copy would be fetched cold.
             ptx::tc_fence_after();
-            uint32_t raw[4][32];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) ptx::tmem_ld32(col + q * 32, raw[q]);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int q = 0; q < 4; ++q) ptx::reg_fence(raw[q]);
             float ss = 0.f;
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t raw[32];
+                ptx::tmem_ld32(col + q * 32, raw);
+                ptx::tmem_wait_ld();
+                ptx::reg_fence(raw);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-                for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(raw[q][i]), __uint_as_float(raw[q][i]), ss);
+                for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(raw[i]), __uint_as_float(raw[i]), ss);
+            }
             const float inv = 1.f / fmaxf(sqrtf(ss), 1e-6f);
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t raw[32];
+                ptx::tmem_ld32(col + q * 32, raw);
+                ptx::tmem_wait_ld();
+                ptx::reg_fence(raw);
 #pragma unroll
-            for (int c16 = 0; c16 < 16; ++c16) {
-                const uint32_t* s = &raw[c16 >> 2][(c16 & 3) * 8];
-                ptx::st_shared_v4(xk + ptx::tile_chunk_offset(r, c16),
-                                  ptx::pack_bf16x2(__uint_as_float(s[0]) * inv, __uint_as_float(s[1]) * inv),
-                                  ptx::pack_bf16x2(__uint_as_float(s[2]) * inv, __uint_as_float(s[3]) * inv),
-                                  ptx::pack_bf16x2(__uint_as_float(s[4]) * inv, __uint_as_float(s[5]) * inv),
-                                  ptx::pack_bf16x2(__uint_as_float(s[6]) * inv, __uint_as_float(s[7]) * inv));
+                for (int g = 0; g < 4; ++g) {
+                    const uint32_t* s = &raw[g * 8];
+                    ptx::st_shared_v4(xk + ptx::tile_chunk_offset(r, q * 4 + g),
+                                      ptx::pack_bf16x2(__uint_as_float(s[0]) * inv, __uint_as_float(s[1]) * inv),
+                                      ptx::pack_bf16x2(__uint_as_float(s[2]) * inv, __uint_as_float(s[3]) * inv),
+                                      ptx::pack_bf16x2(__uint_as_float(s[4]) * inv, __uint_as_float(s[5]) * inv),
+                                      ptx::pack_bf16x2(__uint_as_float(s[6]) * inv, __uint_as_float(s[7]) * inv));
+                }
             }
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
@@ -264,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
             // beta R = beta (Vp - K' S) -> bf16 into xv (the V tile is consumed)
             ptx::tc_fence_after();
-#pragma unroll
+#pragma unroll 1
             for (int q = 0; q < 4; ++q) {
                 uint32_t vp[32], ks[32];
                 ptx::tmem_ld32(col + 128 + q * 32, vp);
@@ -294,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // bytes of a warp's 32 rows
             ptx::tc_fence_after();
             float4* blk = reinterpret_cast<float4*>(part_s + ((size_t)bh * n_parts + pair) * kD * kD);
-#pragma unroll
+#pragma unroll 1
             for (int q = 0; q < 2; ++q) {
                 uint32_t ds[32];
                 ptx::tmem_ld32(tmem + lane_base + kColDS + 64u * c + q * 32, ds);
