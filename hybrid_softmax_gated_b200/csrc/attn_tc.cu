@@ -396,12 +396,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return wwait(&sm.o_free, (si - 1) & 1);
             };
             // K-ring item i: S = Q K_i^T (i < n) or O_inter = Q (W_q S) (i == n),
-            // into buffer (vb + i) & 1
-            auto issue_item = [&](int i) -> bool {
+            // into buffer (vb + i) & 1.  item_ready waits for what the item
+            // needs besides the tensor pipe's order (its buffer's previous
+            // contents read out, its K-ring tile), item_issue issues it.
+            auto item_ready = [&](int i) -> bool {
+                return make_free((vb + i) & 1) && wwait(&sm.k_full[kc & 1], (kc >> 1) & 1);
+            };
+            auto item_issue = [&](int i) {
                 const int buf = (vb + i) & 1;
-                if (!make_free(buf)) return false;
                 const int s = kc & 1;
-                if (!wwait(&sm.k_full[s], (kc >> 1) & 1)) return false;
                 ptx::tc_fence_after();
                 const uint32_t k_s = ptx::smem_u32(sm.k[s]);
                 const uint32_t d = tmem + kColS + (uint32_t)buf * kBN;
@@ -420,16 +423,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::umma_commit_w(ptx::smem_u32(&sm.q_empty[qs]));
                 }
                 ++kc;
-                return true;
             };
-            for (int i = 0; ok && i < 2 && i < nk; ++i) ok = issue_item(i);
+            for (int i = 0; ok && i < 2 && i < nk; ++i) {
+                ok = item_ready(i);
+                if (ok) item_issue(i);
+            }
             if (ok) ok = make_free(-1);  // the first P V of each O_b starts it afresh
             for (int j = 0; ok && j < n; ++j) {
                 const int buf = (vb + j) & 1;
                 const int vs = vc & 1;
                 const uint32_t par = (p_par >> buf) & 1;
                 p_par ^= 1u << buf;
-                ok = wwait(&sm.p_half[buf], par) && wwait(&sm.v_full[vs], (vc >> 1) & 1);
+                // (V first: it has landed long before P, whose hand-off
+                // should start the products without a further check)
+                ok = wwait(&sm.v_full[vs], (vc >> 1) & 1) && wwait(&sm.p_half[buf], par);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 const int ksteps = (block_keys(nc, L, Lc, sg.kv0 + j) + 15) >> 4;
@@ -449,7 +456,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ptx::umma_f16_ts_w(o_t, p_t + (uint32_t)kk * 8u, mnmajor_desc(v_s, kk), idesc_pv,
                                            kk > 0 ? 1u : acc0);
                 }
-                ok = wwait(&sm.p_full[buf], par);
+                // The next item into this buffer follows the P V that reads it;
+                // what else it needs is awaited now, while P is completed.
+                const bool next = j + 2 < nk;
+                ok = (!next || item_ready(j + 2)) && wwait(&sm.p_full[buf], par);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 if (ksteps == kBN / 16) {
@@ -460,8 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ptx::umma_commit_w(ptx::smem_u32(&sm.v_empty[vs]));
                 ++vc;
-                // The next item into this buffer follows the P V that reads it.
-                if (j + 2 < nk) ok = issue_item(j + 2);
+                if (next) item_issue(j + 2);
             }
             if (!ok) break;
             prev_oi_buf = kInter && sg.kind != kHead ? (vb + n) & 1 : -1;
