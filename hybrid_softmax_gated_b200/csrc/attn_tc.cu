@@ -621,9 +621,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float2 sum4[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
                 uint32_t pk[64];
                 // P (bf16 pairs) over the first 64 columns of the S buffer, in
-                // two halves of 64 keys, each handed to the issuer when stored
+                // two halves of 64 keys, each handed to the issuer when stored.
+                // A block of at most 64 keys (a frame's ragged last block) has
+                // no second half: its P V reads the first half only.
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
+                    if (hf == 1 && valid <= kBN / 2) {
+                        warp_arrive(&sm.p_full[wg]);
+                        continue;
+                    }
 #pragma unroll
                     for (int i = 32 * hf; i < 32 * hf + 32; ++i) {
                         // SFU exponentials, with kPolyPairEvery > 0 a share on the FMA pipe
