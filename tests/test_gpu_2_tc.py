@@ -1,7 +1,7 @@
 """GPU parity of the tensor-core (tcgen05) path, bf16 with head_dim 128.
 
 Covers ragged token counts (one token, a partial tile, exact tiles, a
-tile plus one), several streams and heads, and the method's invariants on
+tile plus one, a last block of 64 and of 65 keys), several streams and heads, and the method's invariants on
 the GPU: read-only passes leave the state bit-identical, streams are
 independent, token permutation permutes the output, checkpoint/resume is
 exact.
@@ -26,8 +26,10 @@ def small(L, B=2, H=2, frames=3, passes=2):
                                passes=passes)
 
 
-@pytest.mark.parametrize("L", [1, 17, 128, 129, 300, 515])
+@pytest.mark.parametrize("L", [1, 17, 128, 129, 192, 193, 300, 515])
 def test_tc_stream_matches_oracle_everywhere(L):
+    # 192 and 193: a last key block of exactly 64 keys (its softmax skips the
+    # second half of P) and of 65 (it does not)
     run_and_check(small(L))
 
 
