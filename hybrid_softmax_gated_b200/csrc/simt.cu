@@ -341,8 +341,8 @@ cudaError_t launch_phi_simt(bool bf16, const void* x, const void* w, bool l2norm
     const size_t smem = sizeof(float) * ((size_t)dm.d * 128 + (size_t)kPhiRows * dm.d);
     const dim3 grid((dm.L + kPhiRows - 1) / kPhiRows, dm.H, dm.B);
     if (bf16) {
-        phi_simt_kernel<__nv_bfloat16><<<grid, kPhiThreads, smem, st>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)w, l2norm,
-                                     out_f, (__nv_bfloat16*)out_t, dm);
+        phi_simt_kernel<__nv_bfloat16><<<grid, kPhiThreads, smem, st>>>(
+            (const __nv_bfloat16*)x, (const __nv_bfloat16*)w, l2norm, out_f, (__nv_bfloat16*)out_t, dm);
     } else {
         phi_simt_kernel<float><<<grid, kPhiThreads, smem, st>>>((const float*)x, (const float*)w, l2norm, out_f,
                                      (float*)out_t, dm);

@@ -311,8 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::reg_fence(ds);
 #pragma unroll
                 for (int g = 0; g < 8; ++g)
-                    blk[(size_t)(16 * c + 8 * q + g) * kD + r] = make_float4(__uint_as_float(ds[4 * g]), __uint_as_float(ds[4 * g + 1]),
-                                         __uint_as_float(ds[4 * g + 2]), __uint_as_float(ds[4 * g + 3]));
+                    blk[(size_t)(16 * c + 8 * q + g) * kD + r] =
+                        make_float4(__uint_as_float(ds[4 * g]), __uint_as_float(ds[4 * g + 1]),
+                                    __uint_as_float(ds[4 * g + 2]), __uint_as_float(ds[4 * g + 3]));
             }
         } else {
             fail();
