@@ -54,15 +54,18 @@ def frame_flops(w: workloads.Workload) -> float:
     return B * (w.passes * per_pass + 8.0 * L * d * d * H)
 
 
-def measured_traffic() -> int | None:
+def measured_traffic(workload: str) -> int | None:
     """DRAM bytes per launch of the fused kernel from the last ncu capture
     (profiles/attn_tc_traffic.json), or None once the kernel source has
-    changed since that capture."""
+    changed since that capture, or for a workload other than the captured
+    one."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "attn_tc_traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
+        if d["workload"].split()[0] != workload:
+            return None
         h = hashlib.sha256()
         for rel in d["source_files"]:
             with open(os.path.join(ROOT, rel), "rb") as f:
@@ -811,7 +814,7 @@ def main():
         achieved = attn_flops(w) / (k_ms / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": measured_traffic(), "kernel": "attn_tc_kernel",
+                    "frac": achieved / peak, "traffic": measured_traffic(w.name), "kernel": "attn_tc_kernel",
                     "kernel_ms": k_ms, "flops_per_launch": attn_flops(w),
                     "peak_kind": f"bf16 sustained ({peaks['source']})",
                     "frac_of_burst": achieved / peaks["bf16_tflops"]}
