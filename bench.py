@@ -243,6 +243,17 @@ def oracle_frame_seconds(w: workloads.Workload, budget_s: float = 12.0):
     return per_frame, threads, desc
 
 
+METRIC = "hybrid-attn frames/s (12h x 128d, 1560 tok/frame) & % of B200 BF16 tensor peak"
+
+
+def arm_config(args, w: workloads.Workload, ws: int) -> dict:
+    """The `config` object of the bench line, the same for both arms."""
+    return {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
+            "tokens_per_frame": w.tokens, "frames_per_step": w.frames, "passes": w.passes,
+            "parallelism": f"replicas{ws}", "l2": "inputs larger than L2 (1.2 GB ring)",
+            "gating": args.gating, "access": args.access, "gates": args.gates}
+
+
 def run_reference(args, w: workloads.Workload):
     """--impl reference: the CPU oracle as it stands, on a bounded sample per step."""
     ws, rank, _ = dist_env()
@@ -282,12 +293,11 @@ def run_reference(args, w: workloads.Workload):
     sample = (f"per step: one full clean-pass state update plus {R} output rows x {w.passes} passes "
               f"of one {w.name} frame, rows scaled by L/R to a whole frame")
     line = {
-        "impl": "reference", "metric": "hybrid-attn frames/s", "value": value, "unit": "frames/s",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "frames/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": spf * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
-                   "tokens_per_frame": w.tokens, "frames": w.frames, "passes": w.passes},
+        "config": arm_config(args, w, ws),
         "cpu_baseline": {"value": value, "unit": "frames/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -826,14 +836,11 @@ def main():
                "sample": desc}
 
     line = {
-        "metric": "hybrid-attn frames/s (12h x 128d, 1560 tok/frame) & % of B200 BF16 tensor peak",
+        "metric": METRIC,
         "value": value, "unit": "frames/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
-                   "tokens_per_frame": w.tokens, "frames_per_step": w.frames, "passes": w.passes,
-                   "parallelism": f"replicas{ws}", "l2": "inputs larger than L2 (1.2 GB ring)",
-                   "gating": args.gating, "access": args.access, "gates": args.gates},
+        "config": arm_config(args, w, ws),
         "tokens_per_s": value * w.tokens,
         "tflops_per_frame_algorithmic": frame_flops(w) / 1e12,
         "roofline": roofline, "clocks": clk,
