@@ -14,8 +14,11 @@
 // process exits.  Host code cannot use its name as a device address, so the
 // first call on each device looks the address up with cudaGetSymbolAddress
 // (with that device current) and caches it; that first call also sets the
-// kernels' shared-memory limits.  Every call shares the array and leaves
-// its contents behind; calls whose work overlaps on the GPU race on it.
+// kernels' shared-memory limits.  Both are kept for the life of the process:
+// after a cudaDeviceReset the cached address and attributes are stale, so
+// the call must not be used across one.  Every call shares the array and
+// leaves its contents behind; calls whose work overlaps on the GPU race on
+// it.
 #include "arl2.h"
 #include "internal.h"
 
@@ -26,6 +29,10 @@ namespace {
 
 constexpr size_t kMaxElems = ARL2_NOALLOC_MAX_ELEMENTS;
 constexpr int kMaxDevices = 64;
+// The same caps as arl2_create: heads and batch are grid dimensions of the
+// SIMT kernels (at most 65535 each).
+constexpr int kMaxHeads = 1024;
+constexpr int kMaxBatch = 65535;
 
 // [0, kMaxElems): k' (fp32); [kMaxElems, 2 kMaxElems): v', then r.
 static __device__ __align__(256) float g_update_scratch[2 * kMaxElems];
@@ -66,7 +73,9 @@ extern "C" arl2_status arl2_state_update_noalloc(int batch, int heads, int head_
                                                  float* state, cudaStream_t stream) {
     if (!k || !v || !w_k || !w_v || !alpha || !beta || !state) return ARL2_ERR_INVALID_ARG;
     if (dtype != ARL2_BF16 && dtype != ARL2_FP32) return ARL2_ERR_INVALID_ARG;
-    if (batch < 1 || heads < 1 || tokens < 1 || head_dim < 1 || head_dim > 128) return ARL2_ERR_SHAPE;
+    if (batch < 1 || batch > kMaxBatch || heads < 1 || heads > kMaxHeads || tokens < 1 || head_dim < 1 ||
+        head_dim > 128)
+        return ARL2_ERR_SHAPE;
     const size_t elems = (size_t)batch * (size_t)tokens * (size_t)heads * (size_t)head_dim;
     if (elems > kMaxElems) return ARL2_ERR_SHAPE;
     if (!aligned16(k) || !aligned16(v) || !aligned16(w_k) || !aligned16(w_v) || !aligned16(state))

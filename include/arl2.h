@@ -232,12 +232,15 @@ unsigned long long arl2_kernel_launches(const arl2_handle* h);
  *
  * The first call on each device looks up the scratch array's device address
  * (cudaGetSymbolAddress, with that device current) and sets kernel
- * attributes; make that first call before any stream capture.  Every call
- * shares the one scratch array and leaves its contents behind, so calls
+ * attributes; make that first call before any stream capture.  That set-up
+ * is cached for the life of the process, so do not use this call across a
+ * cudaDeviceReset (the cached address and attributes would be stale).  Every
+ * call shares the one scratch array and leaves its contents behind, so calls
  * whose work overlaps on the GPU (other streams, other threads) race: keep
  * them ordered.  Errors: INVALID_ARG (null pointer, bad dtype), SHAPE (a
- * dimension out of range, or B*L*H*d > ARL2_NOALLOC_MAX_ELEMENTS), ALIGN,
- * CUDA; nothing is enqueued on an error other than CUDA. */
+ * dimension out of range: batch above 65535, heads above 1024, head_dim
+ * above 128, or B*L*H*d > ARL2_NOALLOC_MAX_ELEMENTS), ALIGN, CUDA; nothing
+ * is enqueued on an error other than CUDA. */
 arl2_status arl2_state_update_noalloc(int batch, int heads, int head_dim, int tokens,
                                       arl2_dtype dtype, const void* k, const void* v,
                                       const void* w_k, const void* w_v, const float* alpha,

@@ -144,3 +144,18 @@ def test_gate_projection_config_is_validated_before_cuda():
     assert lib.arl2_gates_apply(None, None, None, None, None) == -1
     assert lib.arl2_frame_forward_hidden(None, None, None, None, None, 1, None, None) == -1
     assert lib.arl2_frame_forward_hidden_host(None, None, None, None, None, 1, None, None) == -1
+
+
+def test_noalloc_update_arguments_are_validated_before_cuda():
+    lib = arl2._lib
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: validation fails first
+    f = lambda *dims, dt=arl2.ARL2_FP32, ptr=fake: lib.arl2_state_update_noalloc(
+        *dims, dt, ptr, ptr, ptr, ptr, ptr, ptr, ptr, None)
+    assert f(1, 1, 16, 16, ptr=None) == -1
+    assert f(1, 1, 16, 16, dt=9) == -1
+    for bad in [(0, 1, 16, 16), (1, 0, 16, 16), (1, 1, 0, 16), (1, 1, 129, 16), (1, 1, 16, 0),
+                (1, 70000, 1, 1), (70000, 1, 1, 1), (1, 1025, 1, 1)]:
+        assert f(*bad) == -2, bad
+    tokens = arl2.NOALLOC_MAX_ELEMENTS // (12 * 128) + 1
+    assert f(1, 12, 128, tokens) == -2
+    assert f(1, 1, 16, 16, ptr=ctypes.c_void_p(0x1004)) == -3
