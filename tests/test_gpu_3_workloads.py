@@ -6,11 +6,13 @@ times, against the CPU oracle on sampled output rows and the full state.
   frame.
 - 720p: 30 frames x 4 passes; every row of the first pass, 16 random rows
   elsewhere, the full state after each frame.
-- long stream (240 frames): device memory and per-frame time stay flat,
-  the state stays finite and bounded, and the last frame matches the
-  oracle when the oracle starts from the GPU's own state.
-- 30-layer stack with 4 streams: layers 0 and 29 against the oracle for
-  the first frames; every layer's streams independent of each other.
+- long stream (240 frames): device memory and per-frame time stay flat;
+  the oracle carries its own state through all 240 clean passes and the
+  GPU state matches it every 20 frames and at the end; sampled rows of
+  frames 0, 1, 120 and 239 match the oracle's outputs.
+- 30-layer stack with 4 streams: layer 0 over all 60 frames, layers 0, 7,
+  15, 22 and 29 over 4 frames, against the oracle (sampled rows, full
+  state); every layer's streams independent of each other.
 """
 import time
 
@@ -42,32 +44,54 @@ def test_720p_stream_sampled_parity():
     print(f"720p worst output err {eo:.3e}, worst state err {es:.3e}")
 
 
-def test_long_stream_memory_and_time_flat_and_last_frame_parity():
+def test_long_stream_memory_and_time_flat_and_state_trajectory_parity():
+    """240 frames x 4 passes.  The oracle carries its own state from S_0
+    through all 240 clean passes (technical summary section 2.1 "State
+    Update", section 2.2 "Clean-Pass Updates"); the GPU state is compared
+    with it in full every 20 frames and after the last frame, and 64 random
+    output rows of every pass of frames 0, 1, 120 and 239 with the oracle's
+    outputs from the oracle's state.  Device memory and per-frame time must
+    not grow with the frame index (section 4, "Efficiency": constant memory)."""
     w = W["long_stream_bf16"]
     lay, (wq, wk, wv) = make_layer(w)
+    S_ref = oracle.zero_state(w.batch, w.heads, w.head_dim)
+    check_rows = {0, 1, 120, w.frames - 1}
+    check_state = set(range(19, w.frames, 20)) | {w.frames - 1}
+    rng = np.random.default_rng(11)
+    worst_o = worst_s = 0.0
     try:
-        free0, _ = torch.cuda.mem_get_info()
         alloc0 = torch.cuda.memory_allocated()
         times, frees = [], []
         start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        last = w.frames - 1
         for f in range(w.frames):
-            a, b = (t.cuda() for t in workloads.frame_gates(w, 0, f))
+            a, b = workloads.frame_gates(w, 0, f)
             ins = [workloads.pass_inputs(w, 0, f, p, device="cuda") for p in range(w.passes)]
-            if f == last:
-                S_prev = lay.state_get().cpu().numpy()
             start.record()
             outs = []
             for p in range(w.passes):
                 q, k, v = ins[p]
-                outs.append(lay.forward(q, k, v, a, b, clean_pass=workloads.is_clean(w, p)))
+                outs.append(lay.forward(q, k, v, a.cuda(), b.cuda(), clean_pass=workloads.is_clean(w, p)))
             stop.record()
             stop.synchronize()
             times.append(start.elapsed_time(stop))
             frees.append(torch.cuda.mem_get_info()[0])
-            if f == last:
-                S_gpu = lay.state_get().cpu().numpy()
-            del outs
+            if f in check_rows:
+                for p in range(w.passes):
+                    q, k, v = (x.cpu() for x in ins[p])
+                    rt = rng.choice(w.tokens, size=64, replace=False)
+                    rb = np.zeros_like(rt)
+                    ref = oracle.rows(q, k, v, wq, S_ref, rb, rt)
+                    e = err(outs[p].float().cpu().numpy()[rb, rt], ref)
+                    worst_o = max(worst_o, e)
+                    assert e <= TOL["bf16"], f"frame {f} pass {p}: output max-abs-rel {e:.3e}"
+            # the oracle's own trajectory: its update from its own state
+            k, v = ins[w.passes - 1][1].cpu(), ins[w.passes - 1][2].cpu()
+            S_ref = oracle.state_update(k, v, wk, wv, a, b, S_ref)
+            if f in check_state:
+                e = err(lay.state_get().cpu().numpy(), S_ref)
+                worst_s = max(worst_s, e)
+                assert e <= TOL["bf16"], f"state after frame {f}: max-abs-rel {e:.3e}"
+            del outs, ins
         assert lay.device_status() == 0
         # memory: nothing grows with the frame index
         assert max(frees) - min(frees) <= 64 << 20
@@ -75,30 +99,31 @@ def test_long_stream_memory_and_time_flat_and_last_frame_parity():
         # time: the second half is not slower than the first
         t = np.array(times[5:])
         assert np.median(t[len(t) // 2:]) <= 1.25 * np.median(t[: len(t) // 2])
-        assert np.all(np.isfinite(S_gpu)) and np.max(np.abs(S_gpu)) < 10.0
-        # last frame: oracle from the GPU's own pre-frame state
-        q, k, v = (x.cpu() for x in ins[w.passes - 1])
-        a, b = workloads.frame_gates(w, 0, last)
-        rng = np.random.default_rng(7)
-        rt = rng.choice(w.tokens, size=64, replace=False)
-        rb = np.zeros_like(rt)
-        ref = oracle.rows(q, k, v, wq, S_prev, rb, rt)
-        # replay the last clean pass from the state the stream had before it
-        lay.state_set(torch.from_numpy(S_prev).cuda())
-        o = lay.forward(ins[-1][0], ins[-1][1], ins[-1][2], a.cuda(), b.cuda(), clean_pass=True)
-        assert err(o.float().cpu().numpy()[rb, rt], ref) <= TOL["bf16"]
-        S_ref = oracle.state_update(k, v, wk, wv, a, b, S_prev)
-        assert err(lay.state_get().cpu().numpy(), S_ref) <= TOL["bf16"]
-        print(f"long stream: median frame {np.median(t):.3f} ms, free-mem spread "
-              f"{(max(frees) - min(frees)) / 2**20:.1f} MiB")
+        print(f"long stream: worst output err {worst_o:.3e}, worst state err {worst_s:.3e}, "
+              f"median frame {np.median(t):.3f} ms, free-mem spread {(max(frees) - min(frees)) / 2**20:.1f} MiB")
     finally:
         lay.close()
 
 
-def test_stack30_layers_against_oracle_and_streams_independent():
+def test_stack30_layer0_whole_trajectory_against_oracle():
+    """Layer 0 of the 30-layer stack, 4 streams, all 60 frames: 16 random
+    rows of every pass and the full state after every clean pass."""
     w = W["stack30_bf16"]
-    for layer in (0, w.layers - 1):
-        run_and_check(w, layer=layer, frames=2, full_rows=lambda f, p: False, sample_rows=32)
+    eo, es = run_and_check(w, layer=0, full_rows=lambda f, p: False, sample_rows=16, device_inputs=True)
+    print(f"stack30 layer 0, 60 frames: worst output err {eo:.3e}, worst state err {es:.3e}")
+
+
+@pytest.mark.parametrize("layer", [0, 7, 15, 22, 29])
+def test_stack30_layers_against_oracle(layer):
+    """Five layers spread over the stack (own weights, gates and states), 4
+    streams, the first 4 frames: 32 random rows of every pass and the full
+    state after every clean pass."""
+    w = W["stack30_bf16"]
+    run_and_check(w, layer=layer, frames=4, full_rows=lambda f, p: False, sample_rows=32, device_inputs=True)
+
+
+def test_stack30_streams_independent():
+    w = W["stack30_bf16"]
     # all 30 layers: 4-stream runs equal single-stream runs of the same inputs
     # (states bit-exact; outputs up to the summation order of tiles that the
     # persistent schedule splits differently for 4 and for 1 stream)
