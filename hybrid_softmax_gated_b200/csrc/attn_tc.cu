@@ -685,6 +685,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float a0 = has0 ? ptx::ex2(m0 - m_seg) : 0.f;
             const float a1 = has1 ? ptx::ex2(m1 - m_seg) : 0.f;
             const float l_seg = a0 * l0 + a1 * l1;
+            // partial of (tile, column half): float4 chunk i of row r at [i][r], so
+            // that the 32 lanes of a warp touch 512 consecutive bytes
+            float4* pbase = reinterpret_cast<float4*>(part_o) + ((size_t)sg.tile * 2 + wg) * 16 * kBM + row;
+            // A tail piece merges the head partial the previous CTA wrote at its
+            // start (warp 3 acquires its flag): its 16 float4 of this thread's
+            // row half are loaded now, so that their L2 latency overlaps the
+            // wait for the last product and the accumulator loads.
+            float4 ph[4];  // chunk 0 now; each chunk loads the next one's first
+            float2 ml = make_float2(0.f, 0.f);
+            if (sg.kind == kTail) {
+                ok = wwait(&sm.head_ready, 0);
+                if (!ok) break;
+                ml = __ldcg(reinterpret_cast<const float2*>(part_ml + ((size_t)sg.tile * kBM + row) * 2));
+#pragma unroll
+                for (int i = 0; i < 4; ++i) ph[i] = __ldcg(pbase + (size_t)i * kBM);
+            }
             // the segment's last P V: its commit covers every product before it
             ok = wwait(&sm.v_empty[(vc0 + n - 1) & 1], ((vc0 + n - 1) >> 1) & 1);
             if (!ok) break;
@@ -710,9 +726,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     acc[i] = has1 ? fmaf(a1, __uint_as_float(o1[i]), v0) : v0;
                 }
             };
-            // partial of (tile, column half): float4 chunk i of row r at [i][r], so
-            // that the 32 lanes of a warp touch 512 consecutive bytes
-            float4* pbase = reinterpret_cast<float4*>(part_o) + ((size_t)sg.tile * 2 + wg) * 16 * kBM + row;
             if (sg.kind == kHead) {
                 // unnormalised O, running max and row sum -> partial, then the flag
 #pragma unroll 1
@@ -730,20 +743,68 @@ __global__ void __launch_bounds__(kThreads, 1)
                         make_float2(m_seg, l_seg);
                 // warp 3 publishes it: these writes happen before its release
                 warp_arrive(&sm.staged[si & 1]);
-            } else {
-                float a_t = 1.f, a_h = 0.f, inv_l = 1.f / l_seg;
-                if (sg.kind == kTail) {
-                    // the head piece of this tile was written by the previous CTA
-                    // at its start; warp 3 has acquired its flag
-                    ok = wwait(&sm.head_ready, 0);
-                    if (!ok) break;
-                    const float2 ml = __ldcg(reinterpret_cast<const float2*>(
-                        part_ml + ((size_t)sg.tile * kBM + row) * 2));
-                    const float mm = fmaxf(ml.x, m_seg);
-                    a_h = ptx::ex2(ml.x - mm);
-                    a_t = ptx::ex2(m_seg - mm);
-                    inv_l = 1.f / (a_h * ml.y + a_t * l_seg);
+            } else if (sg.kind == kTail) {
+                // merge with the head partial: four chunks of 16 columns,
+                // unrolled so that the preloaded partial stays in registers
+                const float mm = fmaxf(ml.x, m_seg);
+                const float a_h = ptx::ex2(ml.x - mm);
+                const float a_t = ptx::ex2(m_seg - mm);
+                const float inv_l = 1.f / (a_h * ml.y + a_t * l_seg);
+                const uint32_t stage = ptx::smem_u32(sm.q[si & 1]);  // the segment's Q slot
+                const uint32_t o0c = tmem + lane_base + kColO + (uint32_t)wg * 64;
+                const uint32_t oi_col = tmem + lane_base + kColS + (uint32_t)((vb + n) & 1) * kBN + (uint32_t)wg * 64;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float4 pn[4];
+                    if (c < 3) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) pn[i] = __ldcg(pbase + (size_t)((c + 1) * 4 + i) * kBM);
+                    }
+                    uint32_t o0[16], o1[16], oi[16];
+                    ptx::tmem_ld16(o0c + (uint32_t)c * 16, o0);
+                    ptx::tmem_ld16(o0c + kD + (uint32_t)c * 16, o1);
+                    if (kInter) ptx::tmem_ld16(oi_col + (uint32_t)c * 16, oi);
+                    ptx::tmem_wait_ld();
+                    ptx::reg_fence16(o0);
+                    ptx::reg_fence16(o1);
+                    if (kInter) ptx::reg_fence16(oi);
+                    float acc[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float v0 = has0 ? a0 * __uint_as_float(o0[i]) : 0.f;
+                        acc[i] = (has1 ? fmaf(a1, __uint_as_float(o1[i]), v0) : v0) * a_t;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float4 p4 = ph[i];
+                        acc[4 * i] = fmaf(a_h, p4.x, acc[4 * i]);
+                        acc[4 * i + 1] = fmaf(a_h, p4.y, acc[4 * i + 1]);
+                        acc[4 * i + 2] = fmaf(a_h, p4.z, acc[4 * i + 2]);
+                        acc[4 * i + 3] = fmaf(a_h, p4.w, acc[4 * i + 3]);
+                    }
+#pragma unroll
+                    for (int gq = 0; gq < 2; ++gq) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i = gq * 8 + e * 2;
+                            const float i0 = kInter ? __uint_as_float(oi[i]) : 0.f;
+                            const float i1 = kInter ? __uint_as_float(oi[i + 1]) : 0.f;
+                            w[e] = ptx::pack_bf16x2(fmaf(acc[i], inv_l, i0), fmaf(acc[i + 1], inv_l, i1));
+                        }
+                        ptx::st_shared_v4(stage + ptx::tile_chunk_offset(row, wg * 8 + c * 2 + gq), w[0], w[1],
+                                          w[2], w[3]);
+                    }
+                    if (c < 3) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) ph[i] = pn[i];
+                    }
                 }
+                ptx::fence_proxy_async_smem();
+                // staged (and the partial read): warp 3 stores it
+                warp_arrive(&sm.staged[si & 1]);
+            } else {
+                const float inv_l = 1.f / l_seg;
                 const uint32_t stage = ptx::smem_u32(sm.q[si & 1]);  // the segment's Q slot
                 const uint32_t oi_col = tmem + lane_base + kColS + (uint32_t)((vb + n) & 1) * kBN + (uint32_t)wg * 64;
 #pragma unroll 1
@@ -751,18 +812,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float acc[32];
                     uint32_t oi[32];
                     load_acc(c, acc, std::bool_constant<kInter>{}, oi_col, oi);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[i] *= a_t;
-                    if (sg.kind == kTail) {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float4 ph = __ldcg(pbase + (size_t)(c * 8 + i) * kBM);
-                            acc[4 * i] = fmaf(a_h, ph.x, acc[4 * i]);
-                            acc[4 * i + 1] = fmaf(a_h, ph.y, acc[4 * i + 1]);
-                            acc[4 * i + 2] = fmaf(a_h, ph.z, acc[4 * i + 2]);
-                            acc[4 * i + 3] = fmaf(a_h, ph.w, acc[4 * i + 3]);
-                        }
-                    }
                     // bf16 output row chunk -> the staging tile (128-byte swizzle)
 #pragma unroll
                     for (int gq = 0; gq < 4; ++gq) {
