@@ -603,6 +603,115 @@ def stack_curve(args, w: workloads.Workload) -> int:
     return 0
 
 
+def stack30(args, w: workloads.Workload) -> int:
+    """The batched 30-layer stack: w.layers hybrid layers, each with its own
+    handle (own phi maps, gates and fp32 states for w.batch streams), run
+    frame by frame, pass by pass, layer by layer over w.frames frames; the
+    clean pass of every layer updates its states.  One CUDA graph per frame
+    (all layers, all passes).  Inputs cycle through a ring of per-(layer,
+    pass) input sets larger than L2, and each layer's gates through four
+    frames of its own draws.  Prints one JSON line: stream-frames/s through
+    the whole stack, the fused kernel's time per launch at this batch (event
+    pair around a layer's back-to-back read-only passes), peak device
+    memory, and the SM clocks sampled during the timed region."""
+    from hybrid_softmax_gated_b200 import Arl2Layer
+    B, L, H, d = w.batch, w.tokens, w.heads, w.head_dim
+    per_set = 3 * B * L * H * d * 2
+    ring = max(4, (400 << 20) // per_set + 1)
+    ins = [workloads.pass_inputs(w, i % w.layers, 0, i // w.layers, device="cuda") for i in range(ring)]
+    layers, gates = [], []
+    for l in range(w.layers):
+        wq, wk, wv = workloads.phi_weights(w, l)
+        layers.append(Arl2Layer(B, H, d, L, wq.cuda(), wk.cuda(), wv.cuda(), dtype=w.torch_dtype))
+        gates.append([tuple(t.cuda() for t in workloads.frame_gates(w, l, f)) for f in range(4)])
+    outs = [torch.empty_like(ins[0][0]) for _ in range(2)]
+    st = torch.cuda.current_stream()
+    cap = torch.cuda.Stream()
+
+    def frame(f):
+        for p in range(w.passes):
+            clean = workloads.is_clean(w, p)
+            for l, lay in enumerate(layers):
+                q, k, v = ins[(f * w.passes * w.layers + p * w.layers + l) % ring]
+                a, b = gates[l][f % 4]
+                lay.forward(q, k, v, a, b, clean_pass=clean, out=outs[l & 1])
+
+    launches0 = sum(lay.kernel_launches() for lay in layers)
+    graphs = []
+    for f in range(w.frames):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            frame(f)
+        graphs.append(g)
+    launches_per_run = sum(lay.kernel_launches() for lay in layers) - launches0
+    for _ in range(max(1, args.warmup // 3)):  # the whole stream once per warm-up round
+        for g in graphs:
+            g.replay()
+    torch.cuda.synchronize()
+    for lay in layers:
+        lay.state_reset()
+    clocks = ClockSampler(torch.cuda.current_device())
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    clocks.start()
+    e0.record(st)
+    for g in graphs:
+        g.replay()
+    e1.record(st)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    bad = [lay.device_status() for lay in layers]
+    if any(bad):
+        raise SystemExit(f"device status {bad}")
+    del graphs
+    # the fused kernel at this batch: layer 0's read-only passes back to back
+    n_k = max(1, w.passes - 1) * 8
+    kg = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(kg, stream=cap):
+        for i in range(n_k):
+            layers[0].forward(*ins[i % ring], out=outs[0])
+    kg.replay()
+    torch.cuda.synchronize()
+    k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    k0.record(st)
+    kg.replay()
+    k1.record(st)
+    torch.cuda.synchronize()
+    k_ms = k0.elapsed_time(k1) / n_k
+    del kg
+    peaks = load_peaks()
+    achieved = attn_flops(w) / (k_ms / 1e3) / 1e12
+    value = B * w.frames / (ms / 1e3)
+    line = {
+        "metric": "hybrid-attn stream-frames/s through a 30-layer stack (12h x 128d, 1560 tok/frame, 4 streams)",
+        "value": value, "unit": "frames/s", "n_gpus": 1, "steps": 1, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "layers": w.layers, "batch": B, "heads": H, "head_dim": d,
+                   "tokens_per_frame": L, "frames": w.frames, "passes": w.passes,
+                   "l2": f"inputs larger than L2 ({ring} input sets of {per_set >> 20} MiB)",
+                   "step": "the whole stream: frames x passes x layers, one CUDA graph per frame"},
+        "layer_frames_per_s": value * w.layers,
+        "tflops_algorithmic": w.layers * B * w.frames * frame_flops(dataclasses_replace(w, batch=1)) / (ms / 1e3) / 1e12,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "kernel": "attn_tc_kernel", "kernel_ms": k_ms,
+                     "flops_per_launch": attn_flops(w), "peak_kind": f"bf16 burst ({peaks['source']})"},
+        "clocks": clk,
+        "gpu_launches": launches_per_run,
+        "peak_device_bytes": torch.cuda.max_memory_allocated() + sum(lay.device_bytes() for lay in layers),
+    }
+    for lay in layers:
+        lay.close()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def dataclasses_replace(w, **kw):
+    import dataclasses
+    return dataclasses.replace(w, **kw)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -652,6 +761,8 @@ def main():
         return profile_case(args, w)
     if args.stack_curve:
         return stack_curve(args, w)
+    if w.layers > 1:
+        return stack30(args, w)
     if ws > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
