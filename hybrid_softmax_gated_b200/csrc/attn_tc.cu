@@ -51,9 +51,9 @@
 // Online softmax with lazy rescaling: the running row max only moves when
 // it grows by more than 2^8; the final 1/l uses the same max as the
 // numerator, so the result is exact up to rounding.  Exponentials run on
-// the SFU (ex2.approx); the packed f32x2 polynomial (exp2_fma2) can take a
-// share of them (kPolyPairEvery), which measured slower here: the softmax
-// warps are bound by instruction issue, not by the SFU.
+// the SFU (ex2.approx).  A share on the FMA pipe (a Cody-Waite reduced
+// polynomial in packed f32x2 arithmetic) measured slower: it costs several
+// issue slots per exponential where the SFU costs one.
 // Outputs leave through a TMA store staged in the segment's Q slot; split
 // partials are stored so that a warp's lanes write consecutive 16 bytes.
 #include "attn_tc.h"
@@ -89,12 +89,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;  // S/P buffers at 0, 128; O_0, O_1 at 256, 384
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
-// One pair of exponentials in kPolyPairEvery runs on the FMA pipe (0: none).
-constexpr int kPolyPairEvery = 0;
-__device__ __forceinline__ constexpr bool poly_pair(int i) {
-    constexpr int every = kPolyPairEvery > 0 ? kPolyPairEvery : 1;
-    return kPolyPairEvery > 0 && i % every == every - 1;
-}
 
 enum SegKind : int { kFull = 0, kHead = 1, kTail = 2 };
 
@@ -632,15 +626,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
 #pragma unroll
                     for (int i = 32 * hf; i < 32 * hf + 32; ++i) {
-                        // SFU exponentials, with kPolyPairEvery > 0 a share on the FMA pipe
+                        // SFU exponentials
                         const float2 a = ptx::fma2(make_float2(x[2 * i], x[2 * i + 1]), sl2, nm);
                         float2 p;
-                        if (poly_pair(i)) {
-                            p = ptx::exp2_fma2(a);
-                        } else {
-                            p.x = ptx::ex2(a.x);
-                            p.y = ptx::ex2(a.y);
-                        }
+                        p.x = ptx::ex2(a.x);
+                        p.y = ptx::ex2(a.y);
                         sum4[i & 3] = ptx::add2(sum4[i & 3], p);
                         pk[i] = ptx::pack_bf16x2(p.x, p.y);
                     }

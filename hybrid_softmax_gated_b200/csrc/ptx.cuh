@@ -344,23 +344,6 @@ __device__ __forceinline__ void st_release_gpu(int* p, int v) {
 }
 
 // ---- math -----------------------------------------------------------------
-// 2^x on the FMA and integer pipes instead of the SFU: Cody-Waite style
-// reduction x = n + f, n = rint(x), f in [-1/2, 1/2], and 2^x = 2^n P(f)
-// with P the degree-3 polynomial fitted by fit_exp2_poly.py (relative error
-// below 1e-4).  Inputs are clamped to >= -126 so that 2^n stays a normal
-// scale; results below 2^-126 are not needed by the softmax.
-__device__ __forceinline__ float exp2_fma(float x) {
-    constexpr float kRound = 12582912.f;  // 1.5 * 2^23: x + kRound holds rint(x)
-    x = fmaxf(x, -126.f);
-    const float t = x + kRound;
-    const float f = x - (t - kRound);
-    float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
-    p = fmaf(p, f, 0.6932609677314758f);
-    p = fmaf(p, f, 0.9999280571937561f);
-    const int n = __float_as_int(t) - 0x4B400000;  // rint(x)
-    return __int_as_float(__float_as_int(p) + (n << 23));
-}
-
 // ---- packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction, two lanes of data)
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
     float2 d;
@@ -402,24 +385,6 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
 }
-// exp2_fma on a pair, the arithmetic in f32x2 form.  The exponent is added
-// as t_bits << 23: t = x + 1.5 * 2^23 holds rint(x) + 0x4B400000 in its bit
-// pattern, and 0x4B400000 << 23 vanishes modulo 2^32.
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-    constexpr float kRound = 12582912.f;
-    x.x = fmaxf(x.x, -126.f);
-    x.y = fmaxf(x.y, -126.f);
-    const float2 r = make_float2(kRound, kRound);
-    const float2 t = add2(x, r);
-    const float2 f = sub2(x, sub2(t, r));
-    float2 p = fma2(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
-                    make_float2(0.2426111251115799f, 0.2426111251115799f));
-    p = fma2(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
-    p = fma2(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
-    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
