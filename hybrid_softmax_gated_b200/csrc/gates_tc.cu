@@ -39,30 +39,6 @@ constexpr int kMaxSplit = 8;    // cluster size (portable bound)
 constexpr int kThreads = 128;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-// Every thread of every CTA of the cluster; shared-memory writes before it
-// are visible to the cluster's reads after it.
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                     : "memory");
-}
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t a, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t a) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(a)
-                 : "memory");
-    return v;
-}
 
 __device__ __forceinline__ float gate_sigmoid(float z) { return 1.f / (1.f + expf(-z)); }
 
@@ -97,7 +73,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                   ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tile = blockIdx.x, b = blockIdx.y, n_tiles = gridDim.x;
-    const uint32_t rank = cluster_ctarank();
+    const uint32_t rank = ptx::cluster_ctarank();
     const int n_split = gridDim.z;  // the cluster spans z
     const int nch = (D + kKC - 1) / kKC;
     const int per = (nch + n_split - 1) / n_split;
@@ -202,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::tc_fence_before();
     __syncthreads();
-    cluster_sync();  // #1: every rank's tile is written
+    ptx::cluster_sync();  // #1: every rank's tile is written
 
     // Rank r sums rows [R r, R r + R) of the tile (R = 128 / ranks) over
     // every rank's slice, in rank order, one group of 4 columns of one row
@@ -216,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float4 t[kMaxSplit];
 #pragma unroll
         for (int q = 0; q < kMaxSplit; ++q)
-            if (q < n_split) t[q] = ld_shared_cluster_v4(mapa_shared(a, (uint32_t)q));
+            if (q < n_split) t[q] = ptx::ld_shared_cluster_v4(ptx::mapa_shared(a, (uint32_t)q));
         float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int q = 0; q < kMaxSplit; ++q)
@@ -228,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         *reinterpret_cast<float4*>(&sm.red[rr][4 * g]) = sum;
     }
-    cluster_sync();  // #2: every remote read is done; ranks may go on alone
+    ptx::cluster_sync();  // #2: every remote read is done; ranks may go on alone
     __syncthreads();
 
     // beta of the rank's rows, and their per-head sum of alpha logits
