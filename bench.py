@@ -959,18 +959,19 @@ def main():
     k_ms = float(np.mean(kernel_ms))
     if args.access == "token":
         # the ablation's read-only pass: the fused kernel for the intra-frame
-        # term, then fp32 SIMT phi maps and the chunked sequential scan; its
-        # algorithmic work is the intra term plus, per token, the three phi
-        # maps and the sequential read, residual and update (6 d^2 per head)
+        # term, then the tensor-core chunk preparation and the sequential
+        # chunk scan; its algorithmic work is the intra term plus, per token,
+        # the three phi maps and the sequential read, residual and update
+        # (6 d^2 per head)
         L, d, H, B = w.tokens, w.head_dim, w.heads, w.batch
         flops = (4.0 * L * L * d * H + 6.0 * L * d * d * H + 6.0 * L * d * d * H) * B
         achieved = flops / (k_ms / 1e3) / 1e12
-        peak = fp32_simt_tflops()
-        roofline = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+        peak = peaks["bf16_tflops"]
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": None,
-                    "kernel": "token-level pass (attn_tc_kernel, phi_simt x3, tl_prep, tl_scan)",
+                    "kernel": "token-level pass (attn_tc_kernel, tl_tc_prep_kernel, tl_tc_scan_kernel)",
                     "kernel_ms": k_ms, "flops_per_launch": flops,
-                    "peak_kind": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1965 MHz (unit counts x clock)"}
+                    "peak_kind": f"bf16 burst ({peaks['source']})"}
     else:
         # The kernel is timed in a replay of tens of milliseconds, the regime
         # of the burst GEMM figure; the sustained (seconds-long, power-capped)

@@ -18,6 +18,7 @@
 #include "internal.h"
 #include "attn_tc.h"
 #include "tma.h"
+#include "token_level_tc.h"
 #include "update_tc.h"
 
 #include <cmath>
@@ -60,7 +61,9 @@ struct arl2_handle {
     float* stage_beta = nullptr;
     int alpha_per_key = 0;    // elementwise gating: alpha [B][H][d] instead of [B][H]
     int token_level = 0;      // token-level (sequential) access instead of frame-level
-    float* tl_ws = nullptr;   // token-level chunk workspace
+    float* tl_ws = nullptr;   // token-level chunk workspace (SIMT path)
+    void* tltc_ws = nullptr;  // token-level chunk tiles (tensor-core path)
+    arl2::TlTc* tltc = nullptr;
     void* zero_read = nullptr;  // zero state for the intra-only attention launch
                                 // (bf16 Mt on the tensor-core path, fp32 S on SIMT)
     // gate projections (optional): weights, and the gates they produce
@@ -110,12 +113,13 @@ void release(arl2_handle* h) {
     if (h->tc) arl2::attn_tc_destroy(h->tc);
     if (h->up) arl2::update_tc_destroy(h->up);
     if (h->gtc) arl2::gate_tc_destroy(h->gtc);
+    if (h->tltc) arl2::tl_tc_destroy(h->tltc);
     delete h->maps;
     void* ptrs[] = {h->w_all, h->S, h->Mt, h->Sb, h->part_s, h->attn_ws, h->qp, h->kp,
                     h->vp, h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], h->stage_tok[3],
                     h->stage_alpha, h->stage_beta, h->err, h->tl_ws, h->zero_read,
                     h->w_gate, h->b_gate, h->g_alpha, h->g_beta, h->g_part, h->g_count, h->stage_x,
-                    h->quiet};
+                    h->quiet, h->tltc_ws};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     delete h;
@@ -235,15 +239,19 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
         if (s == ARL2_OK) s = dalloc(h, &h->part_s, parts * sizeof(float));
         if (s == ARL2_OK) s = dalloc(h, &h->attn_ws, arl2::attn_tc_workspace_bytes(dm));
     }
-    if (!use_tc || h->token_level) {
+    if (!use_tc) {
         if (s == ARL2_OK) s = dalloc(h, &h->qp, h->n_tok * sizeof(float));
         if (s == ARL2_OK) s = dalloc(h, &h->kp, h->n_tok * sizeof(float));
         if (s == ARL2_OK) s = dalloc(h, &h->vp, h->n_tok * sizeof(float));
     }
     if (h->token_level) {
-        if (s == ARL2_OK) s = dalloc(h, &h->tl_ws, arl2::tl_workspace_floats(dm) * sizeof(float));
+        if (use_tc) {
+            if (s == ARL2_OK) s = dalloc(h, &h->tltc_ws, arl2::tl_tc_workspace_bytes(dm));
+        } else {
+            if (s == ARL2_OK) s = dalloc(h, &h->tl_ws, arl2::tl_workspace_floats(dm) * sizeof(float));
+            if (s == ARL2_OK && arl2::tl_init() != cudaSuccess) s = ARL2_ERR_CUDA;
+        }
         if (s == ARL2_OK) s = dalloc(h, &h->zero_read, h->n_state * (use_tc ? 2 : sizeof(float)));
-        if (s == ARL2_OK && arl2::tl_init() != cudaSuccess) s = ARL2_ERR_CUDA;
     }
     if (s == ARL2_OK && cfg->host_staging) {
         for (int i = 0; i < 4 && s == ARL2_OK; ++i) s = dalloc(h, &h->stage_tok[i], h->n_tok * h->esz);
@@ -275,6 +283,10 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
         const arl2::UpdateBuffers ub{h->w_all, h->S, h->Sb, h->Mt, h->part_s};
         h->up = arl2::update_tc_create(dm, ub);
         if (!h->maps || !h->maps->ok() || !h->tc || !h->up) s = ARL2_ERR_CUDA;
+        if (s == ARL2_OK && h->token_level) {
+            h->tltc = arl2::tl_tc_create(dm, h->w_all, h->tltc_ws);
+            if (!h->tltc) s = ARL2_ERR_CUDA;
+        }
     }
     if (s != ARL2_OK) {
         release(h);
@@ -320,12 +332,16 @@ static arl2_status token_level_pass(arl2_handle* h, const void* q, const void* k
     const bool bf16 = h->dtype == ARL2_BF16;
     const Dims& dm = h->dm;
     if (h->use_tc) {
-        ++h->launches;
+        // the intra-frame term (the attention kernel reading a zero state),
+        // then the token-level reads and states on the tensor cores
+        h->launches += 3;
         if (arl2::attn_tc_launch(h->tc, *h->maps, q, k, v, h->zero_read, out, h->scale, h->err, st) !=
                 cudaSuccess ||
-            arl2::launch_phi_simt(bf16, q, h->w[0], false, h->qp, nullptr, dm, st) != cudaSuccess)
+            arl2::tl_tc_launch(h->tltc, *h->maps, q, k, v, alpha, h->alpha_per_key, beta, h->S, out, clean,
+                               h->err, st) != cudaSuccess)
             return ARL2_ERR_CUDA;
-        ++h->launches;
+        if (clean) return refresh_derived(h, st);
+        return ARL2_OK;
     } else {
         h->launches += 2;
         if (arl2::launch_phi_simt(bf16, q, h->w[0], false, h->qp, nullptr, dm, st) != cudaSuccess ||

@@ -19,6 +19,7 @@ struct Dims {
 enum : int {
     kErrTimeoutAttn = 1 << 0,
     kErrTimeoutUpdate = 1 << 1,
+    kErrTimeoutTokenLevel = 1 << 2,
 };
 
 // ---- failure path self-test (simt.cu) -------------------------------------
