@@ -401,7 +401,7 @@ def profile_case(args, w: workloads.Workload) -> int:
     from hybrid_softmax_gated_b200 import Arl2Layer
     wq, wk, wv = workloads.phi_weights(w, 0)
     lay = Arl2Layer(w.batch, w.heads, w.head_dim, w.tokens, wq.cuda(), wk.cuda(), wv.cuda(),
-                    dtype=w.torch_dtype)
+                    dtype=w.torch_dtype, access=args.access)
     per_set = 3 * w.batch * w.tokens * w.heads * w.head_dim * (2 if w.dtype == "bf16" else 4)
     ring = max(2, (160 << 20) // per_set + 1)
     ins = [workloads.pass_inputs(w, 0, 0, i, device="cuda") for i in range(ring)]
@@ -409,7 +409,9 @@ def profile_case(args, w: workloads.Workload) -> int:
     out = torch.empty_like(ins[0][0])
     lay.forward(*ins[0], a, b, clean_pass=True, out=out)
     for i in range(args.profile_passes):
-        lay.forward(*ins[(i + 1) % ring], out=out)
+        # (token-level access reads through the gates on every pass)
+        gates = (a, b) if args.access == "token" else ()
+        lay.forward(*ins[(i + 1) % ring], *gates, out=out)
     torch.cuda.synchronize()
     st = lay.device_status()
     lay.close()
