@@ -160,12 +160,14 @@ class Arl2Layer:
 
     w_q, w_k, w_v: CUDA tensors [H, d, d] in the layer dtype (bf16 or fp32),
     row = input feature.  The handle copies them and owns the fp32 state
-    S [B, H, d, d] (zero at creation).
+    S [B, H, d, d] (zero at creation).  host_staging: 0 none, 1 staging
+    buffers for the host-buffer calls, 2 two sets of them whose copies
+    overlap the neighbouring calls' work (arl2_config.host_staging).
     """
 
     def __init__(self, batch: int, heads: int, head_dim: int, tokens: int, w_q, w_k, w_v, *,
                  dtype: torch.dtype = torch.bfloat16, softmax_scale: float = 0.0,
-                 host_staging: bool = False, impl: str = "auto", max_ctas: int = 0,
+                 host_staging: int = 0, impl: str = "auto", max_ctas: int = 0,
                  gating: str = "headwise", access: str = "frame", gate_weights=None, stream=None):
         if dtype not in (torch.bfloat16, torch.float32):
             raise ValueError("dtype must be torch.bfloat16 or torch.float32")
@@ -191,7 +193,7 @@ class Arl2Layer:
         cfg = Arl2Config(batch, heads, head_dim, tokens,
                          ARL2_BF16 if dtype == torch.bfloat16 else ARL2_FP32,
                          w_q.data_ptr(), w_k.data_ptr(), w_v.data_ptr(), float(softmax_scale),
-                         1 if host_staging else 0,
+                         int(host_staging),
                          {"auto": ARL2_IMPL_AUTO, "simt": ARL2_IMPL_SIMT}[impl], int(max_ctas),
                          {"headwise": ARL2_GATE_HEADWISE, "elementwise": ARL2_GATE_ELEMENTWISE}[gating],
                          {"frame": ARL2_ACCESS_FRAME, "token": ARL2_ACCESS_TOKEN}[access],

@@ -55,10 +55,19 @@ struct arl2_handle {
     float* qp = nullptr;      // fp32 workspaces [B][L][H][d]
     float* kp = nullptr;
     float* vp = nullptr;
-    // host staging
-    void* stage_tok[4] = {nullptr, nullptr, nullptr, nullptr};  // q, k, v, out
-    float* stage_alpha = nullptr;
-    float* stage_beta = nullptr;
+    // host staging: one slot (host_staging = 1), or two whose copies run on
+    // the handle's own streams (host_staging = 2, see host_pass)
+    int stage_slots = 0;
+    int stage_next = 0;                   // slot of the next host call
+    void* stage_tok[2][4] = {};           // [slot] q, k, v, out
+    float* stage_alpha[2] = {};
+    float* stage_beta[2] = {};
+    void* stage_x[2] = {};                // [slot] x [B][L][D] (gate projections)
+    cudaStream_t copy_in = nullptr;       // two slots: input copies
+    cudaStream_t copy_out = nullptr;      // two slots: output copies
+    cudaEvent_t ev_in[2] = {};            // [slot] input copies done
+    cudaEvent_t ev_fwd[2] = {};           // [slot] the pass that read the slot done
+    cudaEvent_t ev_out[2] = {};           // [slot] output copy done
     int alpha_per_key = 0;    // elementwise gating: alpha [B][H][d] instead of [B][H]
     int token_level = 0;      // token-level (sequential) access instead of frame-level
     float* tl_ws = nullptr;   // token-level chunk workspace (SIMT path)
@@ -74,7 +83,6 @@ struct arl2_handle {
     float* g_beta = nullptr;    // [B][H][L]
     float* g_part = nullptr;    // [B][gate_tiles(L)][H]
     unsigned* g_count = nullptr;  // [B], zero between launches
-    void* stage_x = nullptr;    // host entry: staging of x [B][L][D]
     arl2::GateTc* gtc = nullptr;  // tensor-core gate projection (bf16), else the SIMT kernel
     int* quiet = nullptr;       // a zero word nothing ever sets (the failure-path self-test)
     int* err = nullptr;       // device error word
@@ -116,12 +124,23 @@ void release(arl2_handle* h) {
     if (h->tltc) arl2::tl_tc_destroy(h->tltc);
     delete h->maps;
     void* ptrs[] = {h->w_all, h->S, h->Mt, h->Sb, h->part_s, h->attn_ws, h->qp, h->kp,
-                    h->vp, h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], h->stage_tok[3],
-                    h->stage_alpha, h->stage_beta, h->err, h->tl_ws, h->zero_read,
-                    h->w_gate, h->b_gate, h->g_alpha, h->g_beta, h->g_part, h->g_count, h->stage_x,
+                    h->vp, h->err, h->tl_ws, h->zero_read,
+                    h->w_gate, h->b_gate, h->g_alpha, h->g_beta, h->g_part, h->g_count,
                     h->quiet, h->tltc_ws};
     for (void* p : ptrs)
         if (p) cudaFree(p);
+    for (int sl = 0; sl < 2; ++sl) {
+        for (void* p : h->stage_tok[sl])
+            if (p) cudaFree(p);
+        void* more[] = {h->stage_alpha[sl], h->stage_beta[sl], h->stage_x[sl]};
+        for (void* p : more)
+            if (p) cudaFree(p);
+        cudaEvent_t evs[] = {h->ev_in[sl], h->ev_fwd[sl], h->ev_out[sl]};
+        for (cudaEvent_t e : evs)
+            if (e) cudaEventDestroy(e);
+    }
+    if (h->copy_in) cudaStreamDestroy(h->copy_in);
+    if (h->copy_out) cudaStreamDestroy(h->copy_out);
     delete h;
 }
 
@@ -159,6 +178,56 @@ arl2_status clean_update(arl2_handle* h, const void* k, const void* v, const flo
         arl2::launch_accum_simt(h->kp, h->vp, alpha, h->alpha_per_key, beta, h->S, h->dm, st) != cudaSuccess)
         return ARL2_ERR_CUDA;
     return ARL2_OK;
+}
+
+struct HostCopy {
+    void* dst;
+    const void* src;
+    size_t bytes;
+};
+
+// One pass on host buffers through staging slot `slot`: the input copies,
+// then `pass` (which enqueues the pass on `stream`, writing the slot's output
+// staging), then the copy of the output back to `out`.  With one slot every
+// copy runs on `stream`, in order.  With two, the input copies run on the
+// handle's copy-in stream once the pass that last read the slot is done,
+// the pass waits for them, the output copy runs on the copy-out stream, and
+// `stream` waits for that: the call is still complete when `stream` reaches
+// its end, while the next call's input copies overlap this pass and its
+// output copy.  They may also start before earlier work on `stream` ends, so
+// the host inputs must hold their values when the call is made.
+template <typename Pass>
+arl2_status host_pass(arl2_handle* h, int slot, const HostCopy* in, int n_in, void* out, cudaStream_t stream,
+                      Pass&& pass) {
+    const bool piped = h->stage_slots == 2;
+    const cudaStream_t cin = piped ? h->copy_in : stream;
+    if (piped && cudaStreamWaitEvent(cin, h->ev_fwd[slot], 0) != cudaSuccess) return ARL2_ERR_CUDA;
+    for (int i = 0; i < n_in; ++i)
+        if (cudaMemcpyAsync(in[i].dst, in[i].src, in[i].bytes, cudaMemcpyHostToDevice, cin) != cudaSuccess)
+            return ARL2_ERR_CUDA;
+    if (piped && (cudaEventRecord(h->ev_in[slot], cin) != cudaSuccess ||
+                  cudaStreamWaitEvent(stream, h->ev_in[slot], 0) != cudaSuccess))
+        return ARL2_ERR_CUDA;
+    const arl2_status s = pass();
+    if (s != ARL2_OK) return s;
+    const cudaStream_t cout = piped ? h->copy_out : stream;
+    if (piped && (cudaEventRecord(h->ev_fwd[slot], stream) != cudaSuccess ||
+                  cudaStreamWaitEvent(cout, h->ev_fwd[slot], 0) != cudaSuccess))
+        return ARL2_ERR_CUDA;
+    if (cudaMemcpyAsync(out, h->stage_tok[slot][3], h->n_tok * h->esz, cudaMemcpyDeviceToHost, cout) !=
+        cudaSuccess)
+        return ARL2_ERR_CUDA;
+    if (piped && (cudaEventRecord(h->ev_out[slot], cout) != cudaSuccess ||
+                  cudaStreamWaitEvent(stream, h->ev_out[slot], 0) != cudaSuccess))
+        return ARL2_ERR_CUDA;
+    return ARL2_OK;
+}
+
+// The staging slot of the next host call.
+int next_slot(arl2_handle* h) {
+    const int slot = h->stage_next;
+    h->stage_next = h->stage_slots == 2 ? slot ^ 1 : 0;
+    return slot;
 }
 
 }  // namespace
@@ -253,11 +322,22 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
         }
         if (s == ARL2_OK) s = dalloc(h, &h->zero_read, h->n_state * (use_tc ? 2 : sizeof(float)));
     }
-    if (s == ARL2_OK && cfg->host_staging) {
-        for (int i = 0; i < 4 && s == ARL2_OK; ++i) s = dalloc(h, &h->stage_tok[i], h->n_tok * h->esz);
+    h->stage_slots = cfg->host_staging == 2 ? 2 : (cfg->host_staging ? 1 : 0);
+    for (int sl = 0; sl < h->stage_slots && s == ARL2_OK; ++sl) {
+        for (int i = 0; i < 4 && s == ARL2_OK; ++i) s = dalloc(h, &h->stage_tok[sl][i], h->n_tok * h->esz);
         if (s == ARL2_OK)
-            s = dalloc(h, &h->stage_alpha, (size_t)dm.B * dm.H * (h->alpha_per_key ? dm.d : 1) * sizeof(float));
-        if (s == ARL2_OK) s = dalloc(h, &h->stage_beta, (size_t)dm.B * dm.H * dm.L * sizeof(float));
+            s = dalloc(h, &h->stage_alpha[sl], (size_t)dm.B * dm.H * (h->alpha_per_key ? dm.d : 1) * sizeof(float));
+        if (s == ARL2_OK) s = dalloc(h, &h->stage_beta[sl], (size_t)dm.B * dm.H * dm.L * sizeof(float));
+    }
+    if (s == ARL2_OK && h->stage_slots == 2) {
+        if (cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking) != cudaSuccess)
+            s = ARL2_ERR_CUDA;
+        for (int sl = 0; sl < 2 && s == ARL2_OK; ++sl)
+            if (cudaEventCreateWithFlags(&h->ev_in[sl], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&h->ev_fwd[sl], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&h->ev_out[sl], cudaEventDisableTiming) != cudaSuccess)
+                s = ARL2_ERR_CUDA;
     }
     const size_t gate_w_bytes =
         cfg->w_gate ? (size_t)cfg->hidden_dim * arl2::gate_padded_outputs(dm.H) * h->esz : 0;
@@ -270,8 +350,8 @@ arl2_status arl2_create(const arl2_config* cfg, cudaStream_t stream, arl2_handle
         if (s == ARL2_OK)
             s = dalloc(h, &h->g_part, (size_t)dm.B * arl2::gate_part_count(dm.L) * dm.H * sizeof(float));
         if (s == ARL2_OK) s = dalloc(h, &h->g_count, (size_t)dm.B * sizeof(unsigned));
-        if (s == ARL2_OK && cfg->host_staging)
-            s = dalloc(h, &h->stage_x, (size_t)dm.B * dm.L * h->hidden * h->esz);
+        for (int sl = 0; sl < h->stage_slots && s == ARL2_OK; ++sl)
+            s = dalloc(h, &h->stage_x[sl], (size_t)dm.B * dm.L * h->hidden * h->esz);
     }
     if (s == ARL2_OK && arl2::simt_init() != cudaSuccess) s = ARL2_ERR_CUDA;
     if (s == ARL2_OK && h->w_gate && arl2::gate_init() != cudaSuccess) s = ARL2_ERR_CUDA;
@@ -392,34 +472,25 @@ arl2_status arl2_frame_forward_host(arl2_handle* h, const void* q, const void* k
                                     const float* alpha, const float* beta, int clean_pass,
                                     void* out, cudaStream_t stream) {
     if (!h || !q || !k || !v || !out) return ARL2_ERR_INVALID_ARG;
-    if (!h->stage_tok[0]) return ARL2_ERR_INVALID_ARG;
+    if (h->stage_slots == 0) return ARL2_ERR_INVALID_ARG;
     const bool gates = clean_pass || h->token_level;  // the passes that read alpha and beta
     if (gates && (!alpha || !beta)) return ARL2_ERR_INVALID_ARG;
     arl2_status s = check_device(h);
     if (s != ARL2_OK) return s;
+    const Dims& dm = h->dm;
+    const int sl = next_slot(h);
+    void* const* st = h->stage_tok[sl];
     const size_t tb = h->n_tok * h->esz;
-    const void* src[3] = {q, k, v};
-    for (int i = 0; i < 3; ++i)
-        if (cudaMemcpyAsync(h->stage_tok[i], src[i], tb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
-            return ARL2_ERR_CUDA;
-    const float* a_dev = nullptr;
-    const float* b_dev = nullptr;
+    HostCopy in[5] = {{st[0], q, tb}, {st[1], k, tb}, {st[2], v, tb}, {}, {}};
+    int n_in = 3;
     if (gates) {
-        const Dims& dm = h->dm;
-        if (cudaMemcpyAsync(h->stage_alpha, alpha, (size_t)dm.B * dm.H * (h->alpha_per_key ? dm.d : 1) * sizeof(float),
-                            cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-            cudaMemcpyAsync(h->stage_beta, beta, (size_t)dm.B * dm.H * dm.L * sizeof(float),
-                            cudaMemcpyHostToDevice, stream) != cudaSuccess)
-            return ARL2_ERR_CUDA;
-        a_dev = h->stage_alpha;
-        b_dev = h->stage_beta;
+        in[n_in++] = {h->stage_alpha[sl], alpha, (size_t)dm.B * dm.H * (h->alpha_per_key ? dm.d : 1) * sizeof(float)};
+        in[n_in++] = {h->stage_beta[sl], beta, (size_t)dm.B * dm.H * dm.L * sizeof(float)};
     }
-    s = arl2_frame_forward(h, h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], a_dev, b_dev,
-                           clean_pass, h->stage_tok[3], stream);
-    if (s != ARL2_OK) return s;
-    if (cudaMemcpyAsync(out, h->stage_tok[3], tb, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
-        return ARL2_ERR_CUDA;
-    return ARL2_OK;
+    return host_pass(h, sl, in, n_in, out, stream, [&]() {
+        return arl2_frame_forward(h, st[0], st[1], st[2], gates ? h->stage_alpha[sl] : nullptr,
+                                  gates ? h->stage_beta[sl] : nullptr, clean_pass, st[3], stream);
+    });
 }
 
 arl2_status arl2_gates_apply(arl2_handle* h, const void* x, float* alpha, float* beta, cudaStream_t stream) {
@@ -452,25 +523,21 @@ arl2_status arl2_frame_forward_hidden(arl2_handle* h, const void* q, const void*
 arl2_status arl2_frame_forward_hidden_host(arl2_handle* h, const void* q, const void* k, const void* v,
                                            const void* x, int clean_pass, void* out, cudaStream_t stream) {
     if (!h || !q || !k || !v || !out) return ARL2_ERR_INVALID_ARG;
-    if (!h->stage_tok[0] || !h->w_gate) return ARL2_ERR_INVALID_ARG;
+    if (h->stage_slots == 0 || !h->w_gate) return ARL2_ERR_INVALID_ARG;
     const bool gates = clean_pass || h->token_level;
     if (gates && !x) return ARL2_ERR_INVALID_ARG;
     arl2_status s = check_device(h);
     if (s != ARL2_OK) return s;
+    const int sl = next_slot(h);
+    void* const* st = h->stage_tok[sl];
     const size_t tb = h->n_tok * h->esz;
-    const void* src[3] = {q, k, v};
-    for (int i = 0; i < 3; ++i)
-        if (cudaMemcpyAsync(h->stage_tok[i], src[i], tb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
-            return ARL2_ERR_CUDA;
-    if (gates && cudaMemcpyAsync(h->stage_x, x, (size_t)h->dm.B * h->dm.L * h->hidden * h->esz,
-                                 cudaMemcpyHostToDevice, stream) != cudaSuccess)
-        return ARL2_ERR_CUDA;
-    s = arl2_frame_forward_hidden(h, h->stage_tok[0], h->stage_tok[1], h->stage_tok[2], gates ? h->stage_x : nullptr,
-                                  clean_pass, h->stage_tok[3], stream);
-    if (s != ARL2_OK) return s;
-    if (cudaMemcpyAsync(out, h->stage_tok[3], tb, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
-        return ARL2_ERR_CUDA;
-    return ARL2_OK;
+    HostCopy in[4] = {{st[0], q, tb}, {st[1], k, tb}, {st[2], v, tb}, {}};
+    int n_in = 3;
+    if (gates) in[n_in++] = {h->stage_x[sl], x, (size_t)h->dm.B * h->dm.L * h->hidden * h->esz};
+    return host_pass(h, sl, in, n_in, out, stream, [&]() {
+        return arl2_frame_forward_hidden(h, st[0], st[1], st[2], gates ? h->stage_x[sl] : nullptr, clean_pass,
+                                         st[3], stream);
+    });
 }
 
 arl2_status arl2_state_reset(arl2_handle* h, cudaStream_t stream) {

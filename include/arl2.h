@@ -80,8 +80,10 @@ typedef enum { ARL2_GATE_HEADWISE = 0, ARL2_GATE_ELEMENTWISE = 1 } arl2_gating;
  * it with the delta rule, S <- G_i S + beta_i k'_i^T (v'_i - k'_i S), the
  * forget gate acting once with token 0 (G_0 = alpha, G_i = 1); every pass
  * reads through its own sequential states, so alpha and beta are required on
- * every pass, and only the clean pass keeps the final state.  TOKEN runs on
- * fp32 SIMT kernels for the sequential part (bf16 inputs are widened); with
+ * every pass, and only the clean pass keeps the final state.  With bf16 and
+ * d = 128 TOKEN runs on tensor-core kernels (a per-chunk preparation, then a
+ * scan over 128-token chunks with the fp32 state in TMEM and bf16 chunk
+ * operands); otherwise on fp32 SIMT kernels (bf16 inputs are widened).  With
  * bf16 its output is rounded twice (the intra-frame term, then the sum). */
 typedef enum { ARL2_ACCESS_FRAME = 0, ARL2_ACCESS_TOKEN = 1 } arl2_access;
 
@@ -97,8 +99,15 @@ typedef struct {
     const void* w_k;
     const void* w_v;
     float softmax_scale;   /* 0 selects 1/sqrt(d)                             */
-    int host_staging;      /* nonzero: allocate device staging buffers so that
-                              arl2_frame_forward_host can be used             */
+    int host_staging;      /* 0: none; 1: device staging buffers for the
+                              host-buffer calls (arl2_frame_forward_host,
+                              arl2_frame_forward_hidden_host), copies on the
+                              caller's stream; 2: two sets of them, and the
+                              copies run on the handle's own streams so that
+                              one call's input copies overlap the previous
+                              call's pass and output copy (see
+                              arl2_frame_forward_host); other nonzero values
+                              act as 1                                        */
     arl2_impl impl;
     int max_ctas;          /* 0: the tensor-core attention kernel may use every
                               SM; > 0 caps its persistent grid (co-scheduling
@@ -138,10 +147,16 @@ arl2_status arl2_frame_forward(arl2_handle* h, const void* q, const void* k, con
 
 /* arl2_frame_forward on HOST buffers: copies q, k, v (and alpha, beta on a
  * clean pass) from host memory into the handle's device staging buffers,
- * runs the pass, and copies out back to host memory, all stream-ordered on
- * `stream`.  Host buffers should be pinned for the copies to be
- * asynchronous; the caller must not touch them until the stream reaches
- * this point.  Needs a handle created with host_staging != 0
+ * runs the pass, and copies out back to host memory.  The call is complete
+ * when `stream` reaches its end; host buffers should be pinned for the
+ * copies to be asynchronous, and the caller must not touch them until then.
+ * host_staging = 1: every copy is ordered on `stream`.  host_staging = 2:
+ * consecutive calls alternate between two staging sets; the input copies
+ * run on the handle's copy-in stream (once the pass that last used the set
+ * is done) and may start before earlier work on `stream` has finished, so
+ * the host inputs must hold their values when the call is made; the pass
+ * runs on `stream` after them; the output copy runs on the copy-out stream
+ * and `stream` waits for it.  Needs a handle created with host_staging != 0
  * (INVALID_ARG otherwise). */
 arl2_status arl2_frame_forward_host(arl2_handle* h, const void* q, const void* k, const void* v,
                                     const float* alpha, const float* beta, int clean_pass,

@@ -179,3 +179,47 @@ def test_host_buffer_entry_matches_device_entry():
     finally:
         lay_h.close()
         lay_d.close()
+
+
+@pytest.mark.parametrize("L", [200, 1560])
+def test_pipelined_host_staging_matches_device_entry(L):
+    """host_staging = 2: consecutive host calls alternate staging sets, the
+    input copies overlap the previous call's pass and output copy, and no
+    synchronisation between calls; every output and the state must equal the
+    device entry's bit for bit."""
+    w = small(L, B=1, frames=3, passes=3)
+    lay_h, _ = make_layer(w, host_staging=2)
+    lay_d, _ = make_layer(w)
+    try:
+        keep, outs, refs = [], [], []
+        for f in range(w.frames):
+            a, b = workloads.frame_gates(w, 0, f)
+            ah, bh = a.pin_memory(), b.pin_memory()
+            for p in range(w.passes):
+                q, k, v = workloads.pass_inputs(w, 0, f, p)
+                clean = workloads.is_clean(w, p)
+                qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+                out_h = torch.empty_like(q).pin_memory()
+                lay_h.forward_host(qh, kh, vh, ah, bh, clean, out_h)
+                keep.append((qh, kh, vh, ah, bh))
+                outs.append(out_h)
+                refs.append(lay_d.forward(q.cuda(), k.cuda(), v.cuda(), a.cuda(), b.cuda(), clean_pass=clean))
+        torch.cuda.synchronize()
+        for i, (o, r) in enumerate(zip(outs, refs)):
+            assert torch.equal(o, r.cpu()), i
+        assert torch.equal(lay_h.state_get(), lay_d.state_get())
+        # one output buffer for every call: it holds the last pass's output
+        shared = torch.empty_like(outs[0]).pin_memory()
+        lay_h.state_reset()
+        lay_d.state_reset()
+        for f in range(w.frames):
+            a, b = workloads.frame_gates(w, 0, f)
+            for p in range(w.passes):
+                qh, kh, vh, ah, bh = keep[f * w.passes + p]
+                lay_h.forward_host(qh, kh, vh, ah, bh, workloads.is_clean(w, p), shared)
+        torch.cuda.synchronize()
+        assert torch.equal(shared, outs[-1])
+        assert lay_h.device_status() == 0
+    finally:
+        lay_h.close()
+        lay_d.close()
