@@ -958,6 +958,23 @@ def main():
     h2d = w.frames * (w.passes * 3 * tok_bytes + gate_passes * gate_bytes)
     d2h = w.frames * w.passes * tok_bytes
     e2e_value = args.e2e_steps * w.frames * w.batch * ws / (e2e_ms / 1e3)
+    # the bound the copies set: a pinned host-to-device copy of the size of a
+    # pass's inputs, best of a few, against the step's input bytes
+    probe = torch.empty(3 * tok_bytes, dtype=torch.uint8).pin_memory()
+    probe_d = torch.empty(probe.shape, dtype=torch.uint8, device="cuda")
+    h2d_gbs = 0.0
+    for _ in range(5):
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(st)
+        for _ in range(8):
+            probe_d.copy_(probe, non_blocking=True)
+        c1.record(st)
+        c1.synchronize()
+        h2d_gbs = max(h2d_gbs, 8 * probe.numel() / (c0.elapsed_time(c1) / 1e3) / 1e9)
+    del probe, probe_d
+    copy_bound = {"h2d_gbs": h2d_gbs,
+                  "frames_per_s": w.frames * w.batch * ws / (h2d / (h2d_gbs * 1e9)),
+                  "how": "pinned host-to-device copies of one pass's q, k, v bytes, back to back, best of 5"}
 
     peaks = load_peaks()
     k_ms = float(np.mean(kernel_ms))
@@ -1005,7 +1022,7 @@ def main():
         "roofline": roofline, "clocks": clk,
         "e2e": {"value": e2e_value, "unit": "frames/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "copies": "pinned host buffers, two staging sets: a call's "
-                "input copies overlap the previous call's pass and output copy"},
+                "input copies overlap the previous call's pass and output copy", "copy_bound": copy_bound},
         "gpu_launches": args.steps * launches_per_step * ws,
         "cpu_baseline": cpu,
         "peak_device_bytes": torch.cuda.max_memory_allocated() + lay.device_bytes(),
