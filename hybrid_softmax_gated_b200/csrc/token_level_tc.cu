@@ -122,9 +122,16 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     PrepSmem& sm = *reinterpret_cast<PrepSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    // chunk-major order: the last (ragged) chunks of every (stream, head)
+    // are dispatched last, so that when the grid takes more than one wave
+    // the later wave holds the chunks with the least solve work
+    const int n_bh = (int)(gridDim.x / (unsigned)nc);
+    const int c = (int)blockIdx.x / n_bh;
+    const int bhi = (int)blockIdx.x - c * n_bh;
+    const int b = bhi / H, h = bhi - b * H;
     const size_t bh = (size_t)b * H + h;
     const int t0 = c * kC;
+    const int vrows = L - t0 < kC ? L - t0 : kC;  // the chunk's tokens (rows past them are zero)
     volatile int* abort = &sm.abort;
     const int no_abort = 0;
     if (threadIdx.x == 0) {
@@ -326,6 +333,16 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         const int e = threadIdx.x;
 #pragma unroll 1
         for (int jb = r0; jb < r0 + 64; jb += 8) {
+            if (jb >= vrows) {
+                // rows of padding: k' = 0 there, so A's row is zero and T's is e_j
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const float x = jb + r == e ? 1.f : 0.f;
+                    Tf[(jb + r) * kC + e] = x;
+                    st_t_bf16(jb + r, e, x);
+                }
+                continue;
+            }
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
             for (int i = r0; i < jb; ++i) {
@@ -365,7 +382,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     // X = A21 T11 (64 x 64): thread = 4 rows j x 4 columns e
     const int mj = (threadIdx.x >> 4) * 4, me = (threadIdx.x & 15) * 4;
     float* X = At + 64 * kC;  // X[k][e] at A^T row 64 + k (e < 64)
-    if (go) {
+    // with no token past row 63, A21 = 0 and T21 = 0
+    const bool lower = go && vrows > 64;
+    if (lower) {
         float acc[4][4] = {};
 #pragma unroll 4
         for (int i = 0; i < 64; ++i) {
@@ -383,7 +402,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     }
     bar();  // #3b: X written
     // T21 = -T22 X
-    if (go) {
+    if (lower) {
         float acc[4][4] = {};
 #pragma unroll 4
         for (int k = 0; k < 64; ++k) {
@@ -401,8 +420,13 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         for (int u = 0; u < 4; ++u)
 #pragma unroll
             for (int v = 0; v < 4; ++v) st_t_bf16(64 + mj + u, me + v, -acc[u][v]);
-        ptx::fence_proxy_async_smem();  // (after every st.shared of this thread into t[6])
+    } else if (go) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) st_t_bf16(64 + mj + u, me + v, 0.f);
     }
+    if (go) ptx::fence_proxy_async_smem();  // (after every st.shared of this thread into t[6])
     bar();  // #3: T (bf16) complete
 
     // ---- phase 4: T K~ (TMEM 0) and T V' (TMEM 128)
@@ -809,7 +833,7 @@ cudaError_t tl_tc_launch(TlTc* t, TokenMapCache& maps, const void* q, const void
     const Dims& dm = t->dm;
     CUtensorMap cq, ck, cv;
     if (!maps.get(q, &cq) || !maps.get(k, &ck) || !maps.get(v, &cv)) return cudaErrorInvalidValue;
-    tl_tc_prep_kernel<<<dim3(t->nc, dm.H, dm.B), kPrepThreads, kPrepSmem, st>>>(
+    tl_tc_prep_kernel<<<dim3(t->nc * dm.H * dm.B), kPrepThreads, kPrepSmem, st>>>(
         cq, ck, cv, t->tm_w, alpha, alpha_per_key, beta, t->ws, dm.L, dm.H, t->nc, err);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
