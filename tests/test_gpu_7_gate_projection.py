@@ -137,23 +137,33 @@ def test_gate_projection_launch_count():
         lay.close()
 
 
-def test_forward_hidden_host_entry_matches_device_entry():
+@pytest.mark.parametrize("staging", [1, 2])
+def test_forward_hidden_host_entry_matches_device_entry(staging):
+    """Host-buffer passes with projected gates, staging on the caller's stream
+    (1) or double-buffered on the handle's copy streams (2), with no
+    synchronisation between calls: every output and the state equal the
+    device entry's bit for bit."""
     w = small(150, B=1)
-    lay_h, _, _ = make(w, host_staging=True)
+    lay_h, _, _ = make(w, host_staging=staging)
     lay_d, _, _ = make(w)
     try:
+        keep, outs, refs = [], [], []
         for f in range(2):
             x = workloads.hidden_states(w, 0, f)
+            xh = x.pin_memory()
             for p in range(w.passes):
                 q, k, v = workloads.pass_inputs(w, 0, f, p)
                 clean = workloads.is_clean(w, p)
+                qh, kh, vh = (t.pin_memory() for t in (q, k, v))
                 out_h = torch.empty_like(q).pin_memory()
-                lay_h.forward_hidden_host(q.pin_memory(), k.pin_memory(), v.pin_memory(),
-                                          x.pin_memory() if clean else None, clean, out_h)
-                torch.cuda.synchronize()
-                od = lay_d.forward_hidden(q.cuda(), k.cuda(), v.cuda(), x.cuda() if clean else None,
-                                          clean_pass=clean)
-                assert torch.equal(out_h, od.cpu())
+                lay_h.forward_hidden_host(qh, kh, vh, xh if clean else None, clean, out_h)
+                keep.append((qh, kh, vh, xh))
+                outs.append(out_h)
+                refs.append(lay_d.forward_hidden(q.cuda(), k.cuda(), v.cuda(), x.cuda() if clean else None,
+                                                 clean_pass=clean))
+        torch.cuda.synchronize()
+        for i, (o, r) in enumerate(zip(outs, refs)):
+            assert torch.equal(o, r.cpu()), i
         assert torch.equal(lay_h.state_get(), lay_d.state_get())
     finally:
         lay_h.close()
