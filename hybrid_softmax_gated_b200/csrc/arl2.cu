@@ -205,8 +205,11 @@ arl2_status host_pass(arl2_handle* h, int slot, const HostCopy* in, int n_in, vo
     for (int i = 0; i < n_in; ++i)
         if (cudaMemcpyAsync(in[i].dst, in[i].src, in[i].bytes, cudaMemcpyHostToDevice, cin) != cudaSuccess)
             return ARL2_ERR_CUDA;
+    // the pass waits for its inputs and for the slot's previous output copy
+    // (already behind `stream` when consecutive calls share it)
     if (piped && (cudaEventRecord(h->ev_in[slot], cin) != cudaSuccess ||
-                  cudaStreamWaitEvent(stream, h->ev_in[slot], 0) != cudaSuccess))
+                  cudaStreamWaitEvent(stream, h->ev_in[slot], 0) != cudaSuccess ||
+                  cudaStreamWaitEvent(stream, h->ev_out[slot], 0) != cudaSuccess))
         return ARL2_ERR_CUDA;
     const arl2_status s = pass();
     if (s != ARL2_OK) return s;
