@@ -309,17 +309,19 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     }
     bar();  // #2: A^T written; TMEM 0-255 read out
 
-    // ---- phase 3: T = (I + A)^-1, fp32.  With A in 64-row blocks,
+    // ---- phase 3: T = (I + A)^-1, fp32.  With A in 2 x 2 blocks,
     //   T = [[T11, 0], [T21, T22]],  T11 = (I + A11)^-1,  T22 = (I + A22)^-1,
     //   T21 = -T22 A21 T11,
-    // the two diagonal blocks solved at once by forward substitution (thread
-    // = column e: T[j][e] = [j == e] - sum_{r0 <= i < j} A[j][i] T[i][e],
-    // T[i][e] = 0 for i < e, so every thread of a block runs the same rows
-    // and reads A broadcast; rows in groups of 8: the group's sums over
-    // earlier rows first, then the triangle inside the group), then the two
-    // 64 x 64 x 64 products on all 256 threads.  T fp32 [j][e] over t[4..5],
-    // its bf16 copy into t[6] (the A operand of T K~ and T V').  A^T[i][j]
-    // for i >= 64 > j is zero and unused: X = A21 T11 goes there.
+    // applied twice: the four 32-row diagonal blocks are solved at once by
+    // forward substitution (thread = column e: T[j][e] = [j == e] -
+    // sum_{r0 <= i < j} A[j][i] T[i][e], T[i][e] = 0 for i < e, so every
+    // thread of a block runs the same rows and reads A broadcast; rows in
+    // groups of 8: the group's sums over earlier rows first, then the
+    // triangle inside the group), the lower 32-block of each 64-row half
+    // follows from two 32^3 products, and the lower 64-block from two 64^3
+    // products, all on 256 threads.  T fp32 [j][e] over t[4..5], its bf16
+    // copy into t[6] (the A operand of T K~ and T V').  A^T[i][j] for
+    // i >= 64 > j is zero and unused: the products' X = A21 T11 go there.
     float* Tf = reinterpret_cast<float*>(sm.t[4]);
     auto st_t_bf16 = [&](int j, int e, float x) {
         const __nv_bfloat16 hv = __float2bfloat16_rn(x);
@@ -329,10 +331,10 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     };
     const bool go = ok && !*abort;
     if (go && threadIdx.x < kC) {
-        const int r0 = threadIdx.x & 64;  // 0: T11, 64: T22
+        const int r0 = threadIdx.x & ~31;  // the diagonal block's first row
         const int e = threadIdx.x;
 #pragma unroll 1
-        for (int jb = r0; jb < r0 + 64; jb += 8) {
+        for (int jb = r0; jb < r0 + 32; jb += 8) {
             if (jb >= vrows) {
                 // rows of padding: k' = 0 there, so A's row is zero and T's is e_j
 #pragma unroll
@@ -373,12 +375,87 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
             }
         }
     } else if (go) {
-        // T12 = 0: rows 0-63, columns 64-127
-        const int e = 64 + (threadIdx.x & 63);
+        const int u = threadIdx.x - kC;
+        // T12 = 0: rows 0-63, columns 64-127 (bf16 only: no product reads it)
+        {
+            const int e = 64 + (u & 63);
 #pragma unroll 4
-        for (int j = (threadIdx.x >> 6) & 1; j < 64; j += 2) st_t_bf16(j, e, 0.f);
+            for (int j = (u >> 6) & 1; j < 64; j += 2) st_t_bf16(j, e, 0.f);
+        }
+        // the 32-blocks above the diagonal inside each half (fp32 too: the
+        // 64-level products read T11 and T22 whole)
+        {
+            const int hb = u >> 6;
+            const int e = 64 * hb + 32 + (u & 31);
+#pragma unroll 4
+            for (int j = 64 * hb + ((u >> 5) & 1); j < 64 * hb + 32; j += 2) {
+                Tf[j * kC + e] = 0.f;
+                st_t_bf16(j, e, 0.f);
+            }
+        }
     }
-    bar();  // #3a: T11, T22 (and T12 = 0) written
+    bar();  // #3a: the diagonal 32-blocks, and zeros above them
+    {
+        // inside half hh: X' = A21' T11' (32 x 32, into A^T's unused rows),
+        // then T21' = -T22' X'; thread = 2 rows x 4 columns of one half
+        const int hh = threadIdx.x >> 7;
+        const int idx = threadIdx.x & 127;
+        const int pk = (idx >> 3) * 2, pe = (idx & 7) * 4;
+        const int o = 64 * hh;  // the half's first row and column
+        const bool lower32 = go && vrows > o + 32;  // else A21' = 0 (rows of padding) and T21' = 0
+        float* Xs = At + (64 + 32 * hh) * kC + 32 * hh;  // X'[k][e] at Xs[k * kC + e]
+        if (lower32) {
+            float acc[2][4] = {};
+#pragma unroll 4
+            for (int i = 0; i < 32; ++i) {
+                const float a0 = At[(o + i) * kC + o + 32 + pk];  // A[o + 32 + pk][o + i]
+                const float a1 = At[(o + i) * kC + o + 33 + pk];
+                const float4 t = *reinterpret_cast<const float4*>(Tf + (o + i) * kC + o + pe);
+                const float tv4[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    acc[0][v] = fmaf(a0, tv4[v], acc[0][v]);
+                    acc[1][v] = fmaf(a1, tv4[v], acc[1][v]);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+                *reinterpret_cast<float4*>(Xs + (pk + r) * kC + pe) =
+                    make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+        }
+        bar();  // #3b: X' written
+        if (lower32) {
+            float acc[2][4] = {};
+#pragma unroll 4
+            for (int m = 0; m < 32; ++m) {
+                const float t0 = Tf[(o + 32 + pk) * kC + o + 32 + m];  // T22'[pk][m]
+                const float t1 = Tf[(o + 33 + pk) * kC + o + 32 + m];
+                const float4 x = *reinterpret_cast<const float4*>(Xs + m * kC + pe);
+                const float xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    acc[0][v] = fmaf(t0, xv[v], acc[0][v]);
+                    acc[1][v] = fmaf(t1, xv[v], acc[1][v]);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    Tf[(o + 32 + pk + r) * kC + o + pe + v] = -acc[r][v];
+                    st_t_bf16(o + 32 + pk + r, o + pe + v, -acc[r][v]);
+                }
+        } else if (go) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    Tf[(o + 32 + pk + r) * kC + o + pe + v] = 0.f;
+                    st_t_bf16(o + 32 + pk + r, o + pe + v, 0.f);
+                }
+        }
+    }
+    bar();  // #3c: T11, T22 (and T12 = 0) written
     // X = A21 T11 (64 x 64): thread = 4 rows j x 4 columns e
     const int mj = (threadIdx.x >> 4) * 4, me = (threadIdx.x & 15) * 4;
     float* X = At + 64 * kC;  // X[k][e] at A^T row 64 + k (e < 64)
